@@ -1,0 +1,89 @@
+"""Scalar brute-force Sol attention for tiny inputs (test infrastructure only).
+
+An independent second statement of the same forward pass as ``sol_ref``,
+written with plain Python loops and ``math`` so that it shares no code path
+(no NumPy reductions, no einsum) with the oracle it checks.  It is meant for
+N <= 256, D <= 16.  Definitions follow the Star7 README ("MiniMax H3
+Activation Chunk & Attention Acceleration", section 工作原理 > Sol) for the
+exact + centroid split and the KV sink, the thakicloud blog ("이 기술은
+무엇인가") for the mean + tau*std threshold, and the Spark-H3 news page
+(Spark-Reweight bullet) for the log-mass bias.
+
+Inputs are nested lists or arrays indexed [b][n][h][d].
+"""
+from __future__ import annotations
+
+import math
+
+
+def _mean_rows(X, b, h, lo, hi, D):
+    acc = [0.0] * D
+    for t in range(lo, hi):
+        for c in range(D):
+            acc[c] += float(X[b][t][h][c])
+    return [a / (hi - lo) for a in acc]
+
+
+def _dot(x, y):
+    s = 0.0
+    for a, c in zip(x, y):
+        s += a * c
+    return s
+
+
+def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False):
+    """Return (O[b][n][h][d], sel[b][h][i][j]) computed row by row."""
+    s = scale if scale else 1.0 / math.sqrt(D)
+    nqb = (N + bq - 1) // bq
+    nkb = (N + bk - 1) // bk
+    n_sink = (prefix + bk - 1) // bk
+    n_dense = (prefix + bq - 1) // bq
+    O = [[[[0.0] * D for _ in range(H)] for _ in range(N)] for _ in range(B)]
+    SEL = [[None] * H for _ in range(B)]
+    for b in range(B):
+        for h in range(H):
+            kspan = [(j * bk, min(N, (j + 1) * bk)) for j in range(nkb)]
+            qspan = [(i * bq, min(N, (i + 1) * bq)) for i in range(nqb)]
+            kbar = [_mean_rows(K, b, h, lo, hi, D) for lo, hi in kspan]
+            vbar = [_mean_rows(V, b, h, lo, hi, D) for lo, hi in kspan]
+            # anchor = mean of the video queries (all rows when there is no video part)
+            alo = prefix if prefix < N else 0
+            a = _mean_rows(Q, b, h, alo, N, D)
+            bias = []
+            for j, (lo, hi) in enumerate(kspan):
+                if not lmb:
+                    bias.append(0.0)
+                    continue
+                total = 0.0
+                for t in range(lo, hi):
+                    total += math.exp(s * _dot(a, [float(x) for x in K[b][t][h]]))
+                bias.append(math.log(total / (hi - lo)) - s * _dot(a, kbar[j]))
+            sel_bh = []
+            for i, (qlo, qhi) in enumerate(qspan):
+                qbar = _mean_rows(Q, b, h, qlo, qhi, D)
+                sc = [s * _dot(qbar, kbar[j]) for j in range(nkb)]
+                mu = sum(sc) / nkb
+                var = sum((x - mu) ** 2 for x in sc) / nkb
+                thr = -math.inf if tau == -math.inf else mu + tau * math.sqrt(var)
+                row = []
+                for j in range(nkb):
+                    row.append(i < n_dense or j < n_sink or sc[j] > thr)
+                sel_bh.append(row)
+                for r in range(qlo, qhi):
+                    q = [float(x) for x in Q[b][r][h]]
+                    logits, vals = [], []
+                    for j, (lo, hi) in enumerate(kspan):
+                        if row[j]:
+                            for t in range(lo, hi):
+                                logits.append(s * _dot(q, [float(x) for x in K[b][t][h]]))
+                                vals.append([float(x) for x in V[b][t][h]])
+                        else:
+                            logits.append(s * _dot(q, kbar[j]) + math.log(hi - lo) + bias[j])
+                            vals.append(vbar[j])
+                    m = max(logits)
+                    w = [math.exp(x - m) for x in logits]
+                    z = sum(w)
+                    for c in range(D):
+                        O[b][r][h][c] = sum(wi * vi[c] for wi, vi in zip(w, vals)) / z
+            SEL[b][h] = sel_bh
+    return O, SEL

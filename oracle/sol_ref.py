@@ -1,0 +1,209 @@
+"""fp64 CPU oracle for Sol block-sparse attention (test infrastructure only).
+
+This module is test infrastructure.  Only the tests, the smoke check and the
+bench's CPU-baseline leg may import it; the product path never does, and it
+shares no code with the CUDA kernels.
+
+What it computes, step by step, in the order the sources describe it:
+
+  1. pool     -- mean of each block of consecutive rows of Q, K, V ("K/V
+                 centroids"; Star7 README "MiniMax H3 Activation Chunk &
+                 Attention Acceleration", section 工作原理 > Sol; Spark-H3 news
+                 page, "Spark-Attn이 바꾸는 것", Spark-Reweight bullet, which calls
+                 them mean-pooled key/value summaries).
+  2. scores   -- S[i, j] = s * qbar_i . kbar_j, the block score of every
+                 query-block / key-block pair (thakicloud "MiniMax-H3 ComfyUI
+                 accel stack", section "이 기술은 무엇인가": tau is measured in
+                 standard deviations above the mean of the block scores).
+  3. route    -- a key block is exact iff its score is above the row's
+                 mean + tau * std (same section; Star7 README, 工作原理 > Sol:
+                 Q64/K64 threshold routing with tau = 1.0); key blocks that hold
+                 prefix rows are an always-exact KV sink, and query blocks that
+                 hold prefix rows attend densely (Star7 README, 工作原理 > Sol,
+                 last paragraph; aikraft.ru "ComfyUI Sol-Attn", section
+                 "Нововведения версии 2.0", exact_kv / exact_kv_and_rows).
+  4. attention -- selected blocks contribute their rows exactly; each
+                 unselected block contributes one centroid term (logit
+                 s*q.kbar_j + log n_j, value vbar_j) merged into the same
+                 softmax (Star7 README, 工作原理 > Sol).
+  5. log-mass bias (optional) -- mean pooling gives exp(E[x]) instead of
+                 E[exp(x)]; a per-block bias restores the lost mass, scored
+                 against one anchor per head, the mean video query (Spark-H3
+                 news page, Spark-Reweight bullet and the compressed-branch
+                 figure caption).
+
+Readings where the sources are silent (each is listed in the design notes):
+blocks are consecutive rows tiling the whole packed sequence from row 0 (the
+only partial block is the last); the standard deviation is the population
+one over all key blocks; the comparison is strict; a key block is a sink iff
+it holds a prefix row and a query block is dense iff it holds a prefix row;
+log n_j and the centroid use the block's valid row count; the bias is
+bias_j = logsumexp_t(s*a.k_t) - log n_j - s*a.kbar_j and does not change
+routing; tau = -inf selects every block.
+
+Layouts: Q, K, V, O are float64 arrays [B, N, H, D] (BTHD); per-head block
+quantities are [B, H, n_blocks, ...].
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+
+
+def n_blocks(N: int, bs: int) -> int:
+    """Number of blocks of ``bs`` consecutive rows covering N rows."""
+    return -(-N // bs)
+
+
+def block_rows(N: int, bs: int) -> np.ndarray:
+    """Valid row count of every block (bs, or the tail count for the last)."""
+    nb = n_blocks(N, bs)
+    starts = np.arange(nb) * bs
+    return np.minimum(starts + bs, N) - starts
+
+
+def pool(X: np.ndarray, bs: int) -> np.ndarray:
+    """Block means: X [B, N, H, D] -> [B, H, n_blocks, D] (step 1)."""
+    B, N, H, D = X.shape
+    nb = n_blocks(N, bs)
+    out = np.zeros((B, H, nb, D))
+    for j in range(nb):
+        lo, hi = j * bs, min((j + 1) * bs, N)
+        out[:, :, j, :] = X[:, lo:hi, :, :].mean(axis=1)
+    return out
+
+
+def scores(qbar: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarray:
+    """Block scores S[b, h, i, j] = scale * qbar_i . kbar_j (step 2)."""
+    return scale * np.einsum("bhid,bhjd->bhij", qbar, kbar)
+
+
+def thresholds(S: np.ndarray, tau: float) -> np.ndarray:
+    """Row threshold mean + tau * std over all key blocks (population std)."""
+    mu = S.mean(axis=-1)
+    sd = np.sqrt(((S - mu[..., None]) ** 2).mean(axis=-1))
+    if tau == -math.inf:
+        return np.full_like(mu, -math.inf)
+    return mu + tau * sd
+
+
+def route(S: np.ndarray, tau: float, prefix: int, bq: int, bk: int) -> np.ndarray:
+    """Exact-block mask sel[b, h, i, j] (step 3)."""
+    thr = thresholds(S, tau)
+    sel = S > thr[..., None]
+    n_sink = n_blocks(prefix, bk)
+    n_dense = n_blocks(prefix, bq)
+    sel[..., :, :n_sink] = True
+    sel[..., :n_dense, :] = True
+    return sel
+
+
+def to_csr(sel: np.ndarray):
+    """CSR of the mask over rows in (b, h, i) order, columns ascending."""
+    rows = sel.reshape(-1, sel.shape[-1])
+    counts = rows.sum(axis=1).astype(np.int64)
+    row_ptr = np.zeros(rows.shape[0] + 1, np.int64)
+    np.cumsum(counts, out=row_ptr[1:])
+    col_idx = np.nonzero(rows)[1].astype(np.int64)   # row-major order, ascending per row
+    return row_ptr, col_idx
+
+
+def from_csr(row_ptr, col_idx, shape) -> np.ndarray:
+    """Inverse of ``to_csr``: rebuild a boolean mask of ``shape`` [B, H, nqb, nkb]."""
+    sel = np.zeros(shape, bool)
+    flat = sel.reshape(-1, shape[-1])
+    for r in range(flat.shape[0]):
+        flat[r, col_idx[row_ptr[r]:row_ptr[r + 1]]] = True
+    return sel
+
+
+def anchor(Q: np.ndarray, prefix: int) -> np.ndarray:
+    """Per-head anchor: mean of the video (non-prefix) query rows, [B, H, D]."""
+    N = Q.shape[1]
+    rows = Q[:, prefix:, :, :] if prefix < N else Q
+    return rows.mean(axis=1)
+
+
+def log_mass_bias(Q: np.ndarray, K: np.ndarray, kbar: np.ndarray, prefix: int,
+                  scale: float, bk: int) -> np.ndarray:
+    """bias[b, h, j] = log mean_t exp(s a.k_t) - s a.kbar_j over block j (step 5)."""
+    B, N, H, D = K.shape
+    a = anchor(Q, prefix)                                    # [B, H, D]
+    logits = scale * np.einsum("bnhd,bhd->bhn", K, a)        # [B, H, N]
+    nb = n_blocks(N, bk)
+    bias = np.zeros((B, H, nb))
+    for j in range(nb):
+        lo, hi = j * bk, min((j + 1) * bk, N)
+        x = logits[:, :, lo:hi]
+        m = x.max(axis=-1, keepdims=True)
+        lme = (m[..., 0] + np.log(np.exp(x - m).sum(axis=-1))) - math.log(hi - lo)
+        bias[:, :, j] = lme - scale * np.einsum("bhd,bhd->bh", a, kbar[:, :, j, :])
+    return bias
+
+
+def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
+              rows: Optional[dict] = None):
+    """Exact + centroid attention (step 4).
+
+    For every query row r of block i (per b, h): logits are s*q_r.k_t for the
+    rows t of selected key blocks, and s*q_r.kbar_j + log n_j + bias_j for each
+    unselected key block j, with values v_t and vbar_j; the output is the
+    softmax-weighted sum.  Returns (O [B, N, H, D], lse [B, H, N]) where lse is
+    the natural-log normaliser.  ``rows`` optionally maps (b, h) to an array
+    of query rows to compute; other rows are left NaN.
+    """
+    B, N, H, D = Q.shape
+    nqb, nkb = sel.shape[-2], sel.shape[-1]
+    nk = block_rows(N, bk)
+    logn = np.log(nk.astype(np.float64))
+    O = np.full((B, N, H, D), np.nan)
+    lse = np.full((B, H, N), np.nan)
+    for b in range(B):
+        for h in range(H):
+            want = None if rows is None else rows.get((b, h))
+            if rows is not None and want is None:
+                continue
+            for i in range(nqb):
+                lo, hi = i * bq, min((i + 1) * bq, N)
+                r = np.arange(lo, hi)
+                if want is not None:
+                    r = np.intersect1d(r, want)
+                    if r.size == 0:
+                        continue
+                s_j = sel[b, h, i]
+                key_rows = np.concatenate([np.arange(j * bk, min((j + 1) * bk, N))
+                                           for j in np.nonzero(s_j)[0]] or [np.zeros(0, int)])
+                cent = np.nonzero(~s_j)[0]
+                q = Q[b, r, h, :]
+                lg = np.concatenate([scale * q @ K[b, key_rows, h, :].T,
+                                     scale * q @ kbar[b, h, cent, :].T
+                                     + (logn[cent] + bias[b, h, cent])[None, :]], axis=1)
+                vals = np.concatenate([V[b, key_rows, h, :], vbar[b, h, cent, :]], axis=0)
+                m = lg.max(axis=1, keepdims=True)
+                p = np.exp(lg - m)
+                l = p.sum(axis=1, keepdims=True)
+                O[b, r, h, :] = (p @ vals) / l
+                lse[b, h, r] = (m + np.log(l))[:, 0]
+    return O, lse
+
+
+def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: int = 64,
+                scale: Optional[float] = None, log_mass_bias_on: bool = False,
+                mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None):
+    """The whole forward pass; returns a dict of every intermediate."""
+    D = Q.shape[-1]
+    s = (1.0 / math.sqrt(D)) if not scale else float(scale)
+    qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
+    S = scores(qbar, kbar, s)
+    thr = thresholds(S, tau)
+    sel = route(S, tau, prefix, bq, bk)
+    if log_mass_bias_on:
+        bias = log_mass_bias(Q, K, kbar, prefix, s, bk)
+    else:
+        bias = np.zeros(kbar.shape[:3])
+    used = sel if mask_override is None else mask_override
+    O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows)
+    return dict(qbar=qbar, kbar=kbar, vbar=vbar, S=S, thr=thr, sel=sel, bias=bias,
+                O=O, lse=lse, scale=s)
