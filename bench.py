@@ -1,0 +1,349 @@
+"""Benchmark: Sol block-sparse attention forward (pool -> route -> attention) on B200.
+
+One step = one full forward pass (sol_pool, sol_route, sol_attn_fwd) of one
+synthetic sequence resident in HBM.  With --gpus N (one process per GPU,
+launched by torch.distributed.run) every rank runs its own sequence of the
+batch (weak scaling, no collective on the data path); the job value is the
+total work over the slowest rank's time.
+
+Metric: effective TFLOP/s = 4 * D * H * sum over query rows of the exact keys
+they attend (centroid terms excluded) / time per step, with ms per call.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_video_sol_b200 import synth  # noqa: E402
+
+WORKLOADS = {
+    "h56_n32768": lambda: synth.h56_sweep(32768),
+    "h56_n16384": lambda: synth.h56_sweep(16384),
+    "h56_n8192": lambda: synth.h56_sweep(8192),
+    "h56_n4096": synth.h56_n4096,
+    "h56_joint": synth.h56_joint,
+    "tiny": synth.tiny,
+}
+METRIC = "Sol-Attn ms/call & effective TFLOP/s at H=56,N=32768,d=128 bf16; % roofline"
+L2_BYTES = 126 * 2 ** 20
+
+
+def exact_work(row_ptr: np.ndarray, col_idx: np.ndarray, B: int, H: int, N: int) -> int:
+    """sum over query rows of the exact keys they attend (rows x keys), from the CSR."""
+    nb = -(-N // 64)
+    nrows = np.minimum(np.arange(nb) * 64 + 64, N) - np.arange(nb) * 64
+    keys = np.zeros(B * H * nb, np.int64)
+    cnt = np.diff(row_ptr)
+    rowid = np.repeat(np.arange(B * H * nb), cnt)
+    np.add.at(keys, rowid, nrows[col_idx])
+    return int((keys.reshape(B * H, nb) * nrows[None, :]).sum())
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm=pk["hbm_gbs"], bf16=pk["bf16_tflops"], bf16_sus=pk.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "block_sparse_video_sol_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None, None
+    with open(path) as f:
+        t = json.load(f).get(kernel)
+    if not t or source_hash(t["sources"]) != t["source_sha"]:
+        return None, None
+    return t["bytes_per_launch"], t.get("note")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock / throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        loaded = sorted(sm)[len(sm) // 4:] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def oracle_sample(w: synth.Workload, heads, b_offset=0):
+    """Time the fp64 oracle on a head subset of the workload; returns (seconds, rows x keys)."""
+    from oracle import sol_ref
+    q, k, v = (synth.bf16_bits_to_f64(x) for x in synth.generate(w, heads=heads, b_offset=b_offset))
+    t0 = time.perf_counter()
+    out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=w.log_mass_bias)
+    dt = time.perf_counter() - t0
+    nk = sol_ref.block_rows(w.N, 64)
+    work = int(sum(((nk[None, :] * out["sel"][b, h]).sum(1) * nk).sum()
+                   for b in range(w.B) for h in range(len(heads))))
+    return dt, work
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    heads = list(range(min(args.ref_heads or 1, w.H)))
+    for _ in range(args.warmup):
+        oracle_sample(w, heads[:1])
+    times, works = [], []
+    for _ in range(args.steps):
+        dt, work = oracle_sample(w, heads)
+        times.append(dt)
+        works.append(work)
+    sec = float(np.mean(times))
+    # scale the sample to the whole step (all heads) for the per-call time
+    ms_call = sec * 1e3 * w.H / len(heads)
+    val = 4 * w.D * float(np.mean(works)) / sec / 1e12
+    sample = f"{len(heads)} of {w.H} heads of {w.name} per step (full pool/route/attention of those heads)"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
+                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=300))
+    from block_sparse_video_sol_b200 import sol
+
+    # this rank's sequence: batch element `rank` of a world-size batch (pinned host copies for e2e)
+    shape = (w.B, w.N, w.H, w.D)
+    host = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    synth.generate(w, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host), b_offset=rank * w.B)
+    q, k, v = (h.to(dev) for h in host)
+    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias)
+    buf = sol.alloc_buffers(p, dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 1
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        sol.sol_pool(p, q, k, v, buf.ws)
+        if ev:
+            ev[1].record()
+        sol.sol_route(p, buf.ws, buf.row_ptr, buf.col_idx)
+        if ev:
+            ev[2].record()
+        sol.sol_attn_fwd(p, q, k, v, buf.ws, buf.row_ptr, buf.col_idx, buf.o)
+        if ev:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    sol.sol_last_device_status()
+    rp = buf.row_ptr.cpu().numpy().astype(np.int64)
+    ci = buf.col_idx[:int(rp[-1])].cpu().numpy().astype(np.int64)
+    work = exact_work(rp, ci, w.B, w.H, w.N)
+    nb = -(-w.N // 64)
+    density = rp[-1] / (w.B * w.H * nb * nb)
+    flop = 4.0 * w.D * work   # work is summed over every (b, h)
+    cent_flop = 4.0 * w.D * w.B * w.H * w.N * nb
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record()
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sol.sol_last_device_status()
+    total_ms = t0.elapsed_time(t1)
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
+    pool_ms, route_ms, attn_ms = per.mean(axis=0)
+
+    # e2e through the C ABI with host buffers: H2D of q, k, v + forward + D2H of o, every step
+    o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = o_host.numel() * o_host.element_size()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        for dst, src in zip((q, k, v), host):
+            dst.copy_(src, non_blocking=True)
+        step()
+        o_host.copy_(buf.o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    t = torch.tensor([total_ms, e2e_ms, flop], dtype=torch.float64, device=dev)
+    if world > 1:
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = t.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        total_ms, e2e_ms, flop_all = mx[0].item(), mx[1].item(), sm[2].item()
+    else:
+        flop_all = flop
+    if rank == 0:
+        peaks = read_peaks()
+        ms_step = total_ms / args.steps
+        value = flop_all / (ms_step * 1e-3) / 1e12
+        attn_tf = flop / (attn_ms * 1e-3) / 1e12
+        traffic, tnote = profiled_traffic("sol_attn_fwd")
+        in_bytes = 3 * w.B * w.N * w.H * w.D * 2
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
+                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, "global_batch": w.B * world,
+                       "parallelism": f"dp{world} (one sequence per GPU)",
+                       "l2": f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB), no flush"},
+            "roofline": {"kernel": "sol_attn_fwd", "bound": "tensor", "achieved": attn_tf,
+                         "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16"],
+                         "peak_source": f"{peaks['source']} bf16 burst", "traffic": traffic,
+                         "traffic_note": tnote},
+            "kernels": {
+                "sol_pool": {"ms": pool_ms, "GB/s": in_bytes / (pool_ms * 1e-3) / 1e9,
+                             "frac_hbm": in_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm"]},
+                "sol_route": {"ms": route_ms,
+                              "TFLOP/s_fp32": 2.0 * w.B * w.H * nb * nb * w.D / (route_ms * 1e-3) / 1e12},
+                "sol_attn_fwd": {"ms": attn_ms, "TFLOP/s_effective": attn_tf,
+                                 "TFLOP/s_incl_centroids": (flop + cent_flop) / (attn_ms * 1e-3) / 1e12},
+            },
+            "density": float(density), "exact_flop_per_step": flop, "clocks": clocks.summary(),
+            "e2e": {"value": flop_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            heads = list(range(min(args.ref_heads or 4, w.H)))
+            dt, swork = oracle_sample(w, heads)
+            line["cpu_baseline"] = {"value": 4 * w.D * swork / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
+                                    "kind": "oracle",
+                                    "sample": f"{len(heads)} of {w.H} heads of {w.name} ({dt:.1f} s)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="h56_n32768", choices=sorted(WORKLOADS))
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--log-mass-bias", action="store_true")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-heads", type=int, default=None,
+                    help="heads per oracle sample (default: 1 for --impl reference steps, 4 for cpu_baseline)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]()
+    if args.tau is not None or args.log_mass_bias:
+        import dataclasses
+        w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau,
+                                log_mass_bias=args.log_mass_bias,
+                                name=f"{w.name}_tau{args.tau if args.tau is not None else w.tau:g}"
+                                     + ("_lmb" if args.log_mass_bias else ""))
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,253 @@
+// C ABI of libsol.so (declared in include/sol.h): argument validation, the
+// architecture check, workspace layout and the launch sequence of each stage.
+//
+// Precedent for the boundary: the Star7 README "MiniMax H3 Activation Chunk &
+// Attention Acceleration", section 环境与分发, describes a native library that
+// receives only tensor addresses, shapes and the current CUDA stream, does not
+// link the PyTorch C++ ABI, and on an architecture mismatch stops with an
+// error naming the required and the detected compute capability, with no
+// fallback.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace sol {
+
+namespace {
+
+__device__ int g_status = 0;
+
+thread_local char t_err[512] = "";
+
+sol_status fail(sol_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+sol_status fail(sol_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof(t_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+sol_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SOL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Per-device architecture check, done once per device.
+constexpr int kMaxDevices = 64;
+int g_arch_ok[kMaxDevices];   // 0 unknown, 1 ok, -1 refused
+int g_arch_cc[kMaxDevices];
+int* g_status_ptr[kMaxDevices];
+std::mutex g_arch_mu;
+
+// Checks the current device once and records the device address of its
+// status word (the host name of a __device__ variable is not an address).
+sol_status check_arch(int** status = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_arch_mu);
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_arch_cc[dev] = major * 10 + minor;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    if (g_arch_ok[dev] > 0) {
+      void* addr = nullptr;
+      e = cudaGetSymbolAddress(&addr, g_status);
+      if (e != cudaSuccess) { g_arch_ok[dev] = 0; return cuda_fail(e, "cudaGetSymbolAddress(status)"); }
+      g_status_ptr[dev] = static_cast<int*>(addr);
+    }
+  }
+  if (g_arch_ok[dev] < 0)
+    return fail(SOL_ERR_UNSUPPORTED, "libsol requires compute capability 10.0 (sm_100a, B200); device %d is %d.%d",
+                dev, g_arch_cc[dev] / 10, g_arch_cc[dev] % 10);
+  if (status) *status = g_status_ptr[dev];
+  return SOL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape/argument validation shared by every entry point (no CUDA calls).
+sol_status validate(const sol_params* p) {
+  if (!p) return fail(SOL_ERR_INVALID_ARG, "params is NULL");
+  if (p->B < 0 || p->N < 0 || p->H <= 0) return fail(SOL_ERR_INVALID_ARG, "bad shape B=%d N=%d H=%d", p->B, p->N, p->H);
+  if (p->D != 64 && p->D != 128) return fail(SOL_ERR_UNSUPPORTED, "head dim %d unsupported (64 or 128)", p->D);
+  if (p->q_block != kBlock || p->k_block != kBlock)
+    return fail(SOL_ERR_UNSUPPORTED, "block sizes %d/%d unsupported (the GPU path takes 64/64)", p->q_block, p->k_block);
+  if (isnan(p->tau) || p->tau == INFINITY) return fail(SOL_ERR_INVALID_ARG, "tau must be finite or -inf");
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return fail(SOL_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (p->prefix_len < 0 || p->prefix_len > p->N) return fail(SOL_ERR_INVALID_ARG, "prefix_len %d outside [0, N]", p->prefix_len);
+  if (p->log_mass_bias != 0 && p->log_mass_bias != 1) return fail(SOL_ERR_INVALID_ARG, "log_mass_bias must be 0 or 1");
+  const int64_t nb = (p->N + kBlock - 1) / kBlock;
+  if (nb > kMaxKeyBlocks) return fail(SOL_ERR_UNSUPPORTED, "N=%d exceeds the supported %d rows", p->N, kMaxKeyBlocks * kBlock);
+  if ((int64_t)p->B * p->H * nb * nb >= (int64_t)INT32_MAX)
+    return fail(SOL_ERR_UNSUPPORTED, "B*H*blocks^2 exceeds int32 CSR indexing");
+  const int64_t s[6] = {p->in_stride_b, p->in_stride_n, p->in_stride_h, p->out_stride_b, p->out_stride_n, p->out_stride_h};
+  for (int i = 0; i < 6; ++i)
+    if (s[i] < 0 || (s[i] & 7)) return fail(SOL_ERR_INVALID_ARG, "stride %lld must be >= 0 and a multiple of 8 elements", (long long)s[i]);
+  return SOL_OK;
+}
+
+float eff_scale(const sol_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->D); }
+bool empty(const sol_params* p) { return p->B == 0 || p->N == 0; }
+
+}  // namespace
+}  // namespace sol
+
+using namespace sol;
+
+extern "C" {
+
+size_t sol_workspace_bytes(const sol_params* p) {
+  if (validate(p) != SOL_OK || empty(p)) return 0;
+  return ws_layout(*p).total;
+}
+
+sol_status sol_workspace_offsets(const sol_params* p, int64_t offsets[8]) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (!offsets) return fail(SOL_ERR_INVALID_ARG, "offsets is NULL");
+  const WsLayout L = ws_layout(*p);
+  const size_t o[8] = {L.qbar, L.kbar, L.kbar16, L.vbar16, L.cbias, L.anchor, L.mask, L.counts};
+  for (int i = 0; i < 8; ++i) offsets[i] = (int64_t)o[i];
+  return SOL_OK;
+}
+
+int64_t sol_col_capacity(const sol_params* p) {
+  if (validate(p) != SOL_OK || empty(p)) return 0;
+  const int64_t nb = (p->N + kBlock - 1) / kBlock;
+  return (int64_t)p->B * p->H * nb * nb;
+}
+
+sol_status sol_pool(const sol_params* p, const void* q, const void* k, const void* v, void* ws, size_t ws_bytes,
+                    void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!q || !k || !v || !ws) return fail(SOL_ERR_INVALID_ARG, "sol_pool: NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return fail(SOL_ERR_INVALID_ARG, "sol_pool: q/k/v not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SOL_ERR_INVALID_ARG, "sol_pool: workspace not 256-byte aligned");
+  const WsLayout L = ws_layout(*p);
+  if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_pool: workspace %zu < %zu bytes", ws_bytes, L.total);
+  if ((s = check_arch()) != SOL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PoolArgs a{};
+  a.src[0] = static_cast<const __nv_bfloat16*>(q);
+  a.src[1] = static_cast<const __nv_bfloat16*>(k);
+  a.src[2] = static_cast<const __nv_bfloat16*>(v);
+  a.sb = p->in_stride_b; a.sn = p->in_stride_n; a.sh = p->in_stride_h;
+  a.B = p->B; a.N = p->N; a.H = p->H; a.nb = L.nqb; a.prefix = p->prefix_len;
+  a.scale = eff_scale(p);
+  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
+  a.kbar16 = at<__nv_bfloat16>(ws, L.kbar16); a.vbar16 = at<__nv_bfloat16>(ws, L.vbar16);
+  a.cbias = at<float>(ws, L.cbias); a.anchor = at<float>(ws, L.anchor);
+  cudaError_t e;
+  if (!p->log_mass_bias) {
+    a.tensor_mask = 7; a.with_bias = 0;
+    if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch");
+  } else {
+    // Q (and V) first: the anchor (mean video query) must exist before the K pass.
+    a.tensor_mask = 5; a.with_bias = 0;
+    if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (q, v)");
+    e = launch_anchor(a.src[0], a.sb, a.sn, a.sh, a.qbar, p->B, p->N, p->H, p->D, L.nqb, p->prefix_len,
+                      at<float>(ws, L.anchor), st);
+    if (e != cudaSuccess) return cuda_fail(e, "sol_pool anchor launch");
+    a.tensor_mask = 2; a.with_bias = 1;
+    if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (k + bias)");
+  }
+  return SOL_OK;
+}
+
+sol_status sol_route(const sol_params* p, void* ws, size_t ws_bytes, int32_t* row_ptr, int32_t* col_idx, void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!ws || !row_ptr || !col_idx) return fail(SOL_ERR_INVALID_ARG, "sol_route: NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SOL_ERR_INVALID_ARG, "sol_route: workspace not 256-byte aligned");
+  const WsLayout L = ws_layout(*p);
+  if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_route: workspace %zu < %zu bytes", ws_bytes, L.total);
+  if ((s = check_arch()) != SOL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouteArgs a{};
+  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
+  a.B = p->B; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
+  a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
+  a.n_dense = a.n_sink;
+  a.scale = eff_scale(p); a.tau = p->tau;
+  a.mask = at<uint32_t>(ws, L.mask); a.counts = at<int32_t>(ws, L.counts);
+  cudaError_t e = launch_route(a, p->D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_route launch");
+  e = launch_scan_compact(a.mask, a.counts, p->B * p->H * L.nqb, L.mask_words, row_ptr, col_idx, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_route scan/compact launch");
+  return SOL_OK;
+}
+
+sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const void* v, const void* ws,
+                        size_t ws_bytes, const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                        void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!q || !k || !v || !ws || !row_ptr || !col_idx || !o) return fail(SOL_ERR_INVALID_ARG, "sol_attn_fwd: NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(SOL_ERR_INVALID_ARG, "sol_attn_fwd: q/k/v/o not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SOL_ERR_INVALID_ARG, "sol_attn_fwd: workspace not 256-byte aligned");
+  const WsLayout L = ws_layout(*p);
+  if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_attn_fwd: workspace %zu < %zu bytes", ws_bytes, L.total);
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
+  AttnArgs a{};
+  a.status = status;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.sb = p->in_stride_b; a.sn = p->in_stride_n; a.sh = p->in_stride_h;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.ob = p->out_stride_b; a.on = p->out_stride_n; a.oh = p->out_stride_h;
+  a.lse = lse;
+  a.kbar16 = at<__nv_bfloat16>(ws, L.kbar16); a.vbar16 = at<__nv_bfloat16>(ws, L.vbar16);
+  a.cbias = at<float>(ws, L.cbias);
+  a.row_ptr = row_ptr; a.col_idx = col_idx;
+  a.B = p->B; a.N = p->N; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb;
+  a.scale = eff_scale(p);
+  cudaError_t e = launch_attn(a, p->D, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sol_attn_fwd launch");
+  return SOL_OK;
+}
+
+sol_status sol_last_device_status(void* stream) {
+  sol_status s0 = check_arch();
+  if (s0 != SOL_OK) return s0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "device status read");
+  if (v == 0) return SOL_OK;
+  return fail((sol_status)v, "device status: %s", sol_status_string((sol_status)v));
+}
+
+const char* sol_status_string(sol_status s) {
+  switch (s) {
+    case SOL_OK: return "SOL_OK";
+    case SOL_ERR_INVALID_ARG: return "SOL_ERR_INVALID_ARG";
+    case SOL_ERR_UNSUPPORTED: return "SOL_ERR_UNSUPPORTED";
+    case SOL_ERR_WORKSPACE: return "SOL_ERR_WORKSPACE";
+    case SOL_ERR_CUDA: return "SOL_ERR_CUDA";
+    case SOL_ERR_TIMEOUT: return "SOL_ERR_TIMEOUT";
+  }
+  return "SOL_ERR_UNKNOWN";
+}
+
+const char* sol_last_error_text(void) { return t_err; }
+
+}  // extern "C"

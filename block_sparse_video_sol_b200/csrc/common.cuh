@@ -1,0 +1,105 @@
+// Shared definitions of the Sol CUDA path: workspace layout, kernel argument
+// blocks, device status word and small PTX helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/sol.h"
+
+namespace sol {
+
+constexpr int kBlock = 64;          // rows per query / key block on the GPU path
+constexpr int kMaxKeyBlocks = 1024; // ceil(N/64) limit of the routing kernel (N <= 65536)
+
+// Device status word (one per device, owned by the C-ABI layer): kernels set
+// it on an expired bounded wait or a bad CSR entry; sol_last_device_status()
+// reads and clears it.  The first code raised wins.
+__device__ __forceinline__ void raise_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Private workspace layout (byte offsets from the workspace base, 256-aligned).
+struct WsLayout {
+  int nqb, nkb, mask_words;
+  size_t qbar;      // fp32 [B,H,nqb,D]
+  size_t kbar;      // fp32 [B,H,nkb,D]
+  size_t kbar16;    // bf16 [B,H,nkb,D]
+  size_t vbar16;    // bf16 [B,H,nkb,D]
+  size_t cbias;     // fp32 [B,H,nkb]  log n_j (+ bias_j)
+  size_t anchor;    // fp32 [B,H,D]
+  size_t mask;      // uint32 [B*H*nqb, mask_words] exact-block bitmap
+  size_t counts;    // int32 [B*H*nqb]
+  size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const sol_params& p) {
+  WsLayout L{};
+  L.nqb = (p.N + kBlock - 1) / kBlock;
+  L.nkb = L.nqb;
+  L.mask_words = (L.nkb + 31) / 32;
+  size_t bh = (size_t)p.B * p.H, off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  L.qbar = take(bh * L.nqb * p.D * 4);
+  L.kbar = take(bh * L.nkb * p.D * 4);
+  L.kbar16 = take(bh * L.nkb * p.D * 2);
+  L.vbar16 = take(bh * L.nkb * p.D * 2);
+  L.cbias = take(bh * L.nkb * 4);
+  L.anchor = take(bh * p.D * 4);
+  L.mask = take(bh * L.nqb * L.mask_words * 4);
+  L.counts = take(bh * L.nqb * 4);
+  L.total = off;
+  return L;
+}
+
+template <class T> __host__ __device__ __forceinline__ T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(base) + off);
+}
+template <class T> __host__ __device__ __forceinline__ const T* at(const void* base, size_t off) {
+  return reinterpret_cast<const T*>(reinterpret_cast<const char*>(base) + off);
+}
+
+struct PoolArgs {
+  const __nv_bfloat16* src[3];   // q, k, v
+  int64_t sb, sn, sh;            // element strides of the inputs
+  int B, N, H, nb, prefix;
+  float scale;
+  int tensor_mask;               // bit t set: pool tensor t in this launch (grid.z = B * popcount)
+  int with_bias;                 // K pass also computes the log-mass bias
+  float* qbar; float* kbar; __nv_bfloat16* kbar16; __nv_bfloat16* vbar16;
+  float* cbias; const float* anchor;
+};
+
+struct RouteArgs {
+  const float* qbar; const float* kbar;
+  int B, H, nqb, nkb, mask_words, n_sink, n_dense;
+  float scale, tau;
+  uint32_t* mask; int32_t* counts;
+};
+
+struct AttnArgs {
+  const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
+  int64_t sb, sn, sh;            // input strides
+  __nv_bfloat16* o;
+  int64_t ob, on, oh;            // output strides
+  float* lse;
+  const __nv_bfloat16* kbar16; const __nv_bfloat16* vbar16; const float* cbias;
+  const int32_t* row_ptr; const int32_t* col_idx;
+  int B, N, H, nqb, nkb;
+  float scale;
+  int* status;
+};
+
+// Launchers (defined in the kernel files; return the launch error).
+cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st);
+cudaError_t launch_anchor(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh, const float* qbar,
+                          int B, int N, int H, int D, int nqb, int prefix, float* anchor, cudaStream_t st);
+cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st);
+cudaError_t launch_scan_compact(const uint32_t* mask, const int32_t* counts, int rows, int mask_words,
+                                int32_t* row_ptr, int32_t* col_idx, cudaStream_t st);
+cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st);
+
+}  // namespace sol

@@ -1,0 +1,196 @@
+// sol_route kernels: block scores, per-row threshold, exact-block bitmap,
+// then CSR lists (exclusive scan of row counts + compaction).
+//
+// Routing follows the thakicloud blog "MiniMax-H3 ComfyUI accel stack",
+// section 이 기술은 무엇인가 (tau counts standard deviations above the mean of
+// the block scores), and the Star7 README "MiniMax H3 Activation Chunk &
+// Attention Acceleration", section 工作原理 > Sol (Q64/K64 threshold routing,
+// prefix KV sink, dense prefix query rows).
+//
+// The score S = s * qbar kbar^T is a small fp32 contraction (2*nqb*nkb*D flop
+// per head).  It stays on the fp32 FMA pipe: TF32 tensor cores would put
+// ~1e-3 relative error on scores that are compared against a threshold.
+// One CTA owns 32 query blocks of one (b, h) and all key blocks; it keeps
+// its 32 x nkb score rows in shared memory so that the mean, the population
+// std and the mask come from one evaluation of S.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace sol {
+
+constexpr int kRouteTQ = 32;    // query blocks per CTA
+constexpr int kRouteCH = 256;   // key blocks per column chunk
+constexpr int kRouteDS = 32;    // head-dim slice held in shared memory
+constexpr int kRouteLdK = kRouteCH + 1;  // padded row: conflict-free transposed stores
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) {
+  extern __shared__ __align__(16) float sm[];
+  float* qT = sm;                          // [D][TQ]
+  float* kT = qT + D * kRouteTQ;           // [DS][CH+1]
+  float* S = kT + kRouteDS * kRouteLdK;    // [TQ][ldS]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRouteTQ;
+  const float* qbar = a.qbar + (int64_t)bh * a.nqb * D;
+  const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
+
+  for (int idx = tid; idx < kRouteTQ * D; idx += 256) {
+    const int r = idx % kRouteTQ, d = idx / kRouteTQ;
+    qT[d * kRouteTQ + r] = (i0 + r < a.nqb) ? qbar[(int64_t)(i0 + r) * D + d] : 0.f;
+  }
+  const int rg = warp & 3;   // rows 8*rg .. 8*rg+7
+  const int chh = warp >> 2; // columns 128*chh .. +127 of the chunk
+
+  for (int c0 = 0; c0 < a.nkb; c0 += kRouteCH) {
+    float acc[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int d0 = 0; d0 < D; d0 += kRouteDS) {
+      __syncthreads();
+      for (int idx = tid; idx < kRouteCH * (kRouteDS / 4); idx += 256) {
+        const int jj = idx / (kRouteDS / 4), dq = (idx % (kRouteDS / 4)) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c0 + jj < a.nkb) v = *reinterpret_cast<const float4*>(kbar + (int64_t)(c0 + jj) * D + d0 + dq);
+        kT[(dq + 0) * kRouteLdK + jj] = v.x;
+        kT[(dq + 1) * kRouteLdK + jj] = v.y;
+        kT[(dq + 2) * kRouteLdK + jj] = v.z;
+        kT[(dq + 3) * kRouteLdK + jj] = v.w;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int dd = 0; dd < kRouteDS; ++dd) {
+        const float4 qa = *reinterpret_cast<const float4*>(qT + (d0 + dd) * kRouteTQ + 8 * rg);
+        const float4 qb = *reinterpret_cast<const float4*>(qT + (d0 + dd) * kRouteTQ + 8 * rg + 4);
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        float kv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) kv[c] = kT[dd * kRouteLdK + 128 * chh + lane + 32 * c];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(qv[r], kv[c], acc[r][c]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int col = c0 + 128 * chh + lane + 32 * c;
+        if (col < a.nkb) S[(8 * rg + r) * ldS + col] = a.scale * acc[r][c];
+      }
+  }
+  __syncthreads();
+
+  // Row statistics and mask: warp w handles rows 4w .. 4w+3.
+  const float inv_n = 1.f / (float)a.nkb;
+  for (int rr = 0; rr < kRouteTQ / 8; ++rr) {
+    const int r = warp * (kRouteTQ / 8) + rr, i = i0 + r;
+    if (i >= a.nqb) break;
+    const float* Sr = S + r * ldS;
+    float s = 0.f;
+    for (int j = lane; j < a.nkb; j += 32) s += Sr[j];
+    const float mu = warp_sum(s) * inv_n;
+    float ss = 0.f;
+    for (int j = lane; j < a.nkb; j += 32) { const float t = Sr[j] - mu; ss = fmaf(t, t, ss); }
+    const float sd = sqrtf(warp_sum(ss) * inv_n);
+    const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
+    const bool dense = i < a.n_dense;
+    const int64_t row = (int64_t)bh * a.nqb + i;
+    int cnt = 0;
+    for (int w = 0; w < a.mask_words; ++w) {
+      const int j = w * 32 + lane;
+      const bool sel = j < a.nkb && (dense || j < a.n_sink || Sr[j] > thr);
+      const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) a.mask[row * a.mask_words + w] = bits;
+      cnt += __popc(bits);
+    }
+    if (lane == 0) a.counts[row] = cnt;
+  }
+}
+
+// Exclusive scan of the row counts in (b, h, i) order by one CTA.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int rows, int32_t* row_ptr) {
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (rows + 1023) / 1024;
+  const int lo = min(rows, tid * per), hi = min(rows, lo + per);
+  int s = 0;
+  for (int r = lo; r < hi; ++r) s += counts[r];
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_tot[lane], ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
+    }
+    warp_tot[lane] = ti - t;  // exclusive warp offsets
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - s;
+  for (int r = lo; r < hi; ++r) { row_ptr[r] = run; run += counts[r]; }
+  if (tid == 1023) row_ptr[rows] = warp_tot[31] + incl;
+}
+
+// One warp per row: bitmap words -> ascending column indices at row_ptr[row].
+__global__ void __launch_bounds__(256) compact_kernel(const uint32_t* mask, const int32_t* row_ptr, int rows,
+                                                      int mask_words, int32_t* col_idx) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  int base = row_ptr[row];
+  const uint32_t* m = mask + (int64_t)row * mask_words;
+  for (int w = 0; w < mask_words; ++w) {
+    const uint32_t bits = m[w];
+    if ((bits >> lane) & 1u) col_idx[base + __popc(bits & ((1u << lane) - 1u))] = w * 32 + lane;
+    base += __popc(bits);
+  }
+}
+
+static size_t route_smem_bytes(int D, int ldS) {
+  return sizeof(float) * ((size_t)D * kRouteTQ + (size_t)kRouteDS * kRouteLdK + (size_t)kRouteTQ * ldS);
+}
+
+cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
+  const int ldS = ((a.nkb + 3) / 4) * 4;
+  const size_t smem = route_smem_bytes(D, ldS);
+  dim3 grid((a.nqb + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
+  cudaError_t e;
+  if (D == 128) {
+    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
+  } else {
+    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan_compact(const uint32_t* mask, const int32_t* counts, int rows, int mask_words,
+                                int32_t* row_ptr, int32_t* col_idx, cudaStream_t st) {
+  scan_kernel<<<1, 1024, 0, st>>>(counts, rows, row_ptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  compact_kernel<<<(rows + 7) / 8, 256, 0, st>>>(mask, row_ptr, rows, mask_words, col_idx);
+  return cudaGetLastError();
+}
+
+}  // namespace sol

@@ -1,0 +1,186 @@
+"""Thin ctypes binding of libsol.so (the C ABI declared in include/sol.h).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of libsol.so.  Torch tensors supply device memory and the current
+stream; nothing here computes.  Importing this module loads the library and
+raises if it is missing -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsol.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libsol.so not built ({_LIB_PATH}); run `python -m block_sparse_video_sol_b200.build`")
+lib = ctypes.CDLL(_LIB_PATH)
+
+SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(6)
+
+# Every entry point declared in include/sol.h.
+EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_attn_fwd",
+           "sol_last_device_status", "sol_status_string", "sol_last_error_text")
+
+
+class sol_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("q_block", ctypes.c_int32), ("k_block", ctypes.c_int32),
+                ("tau", ctypes.c_float), ("scale", ctypes.c_float),
+                ("prefix_len", ctypes.c_int32), ("log_mass_bias", ctypes.c_int32),
+                ("in_stride_b", ctypes.c_int64), ("in_stride_n", ctypes.c_int64), ("in_stride_h", ctypes.c_int64),
+                ("out_stride_b", ctypes.c_int64), ("out_stride_n", ctypes.c_int64), ("out_stride_h", ctypes.c_int64)]
+
+
+_P = ctypes.POINTER(sol_params)
+_vp = ctypes.c_void_p
+lib.sol_workspace_bytes.argtypes = [_P]
+lib.sol_workspace_bytes.restype = ctypes.c_size_t
+lib.sol_workspace_offsets.argtypes = [_P, ctypes.POINTER(ctypes.c_int64)]
+lib.sol_workspace_offsets.restype = ctypes.c_int
+lib.sol_col_capacity.argtypes = [_P]
+lib.sol_col_capacity.restype = ctypes.c_int64
+lib.sol_pool.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+lib.sol_pool.restype = ctypes.c_int
+lib.sol_route.argtypes = [_P, _vp, ctypes.c_size_t, _vp, _vp, _vp]
+lib.sol_route.restype = ctypes.c_int
+lib.sol_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
+lib.sol_attn_fwd.restype = ctypes.c_int
+lib.sol_last_device_status.argtypes = [_vp]
+lib.sol_last_device_status.restype = ctypes.c_int
+lib.sol_status_string.argtypes = [ctypes.c_int]
+lib.sol_status_string.restype = ctypes.c_char_p
+lib.sol_last_error_text.argtypes = []
+lib.sol_last_error_text.restype = ctypes.c_char_p
+
+
+class SolError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        text = lib.sol_last_error_text().decode()
+        super().__init__(f"{where}: {lib.sol_status_string(status).decode()} ({text})")
+
+
+def _check(status: int, where: str):
+    if status != SOL_OK:
+        raise SolError(status, where)
+
+
+def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: int = 0,
+                log_mass_bias: bool = False, scale: float = 0.0, in_strides=None, out_strides=None,
+                q_block: int = 64, k_block: int = 64) -> sol_params:
+    """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D]."""
+    in_strides = in_strides or (N * H * D, H * D, D)
+    out_strides = out_strides or (N * H * D, H * D, D)
+    return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(bool(log_mass_bias)),
+                      *[int(s) for s in in_strides], *[int(s) for s in out_strides])
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def sol_workspace_bytes(p: sol_params) -> int:
+    return lib.sol_workspace_bytes(ctypes.byref(p))
+
+
+def sol_workspace_offsets(p: sol_params) -> list:
+    out = (ctypes.c_int64 * 8)()
+    _check(lib.sol_workspace_offsets(ctypes.byref(p), out), "sol_workspace_offsets")
+    return list(out)
+
+
+def workspace_views(p: sol_params, ws: torch.Tensor) -> dict:
+    """Typed views of the pooled quantities inside a workspace (see sol_workspace_offsets)."""
+    off = sol_workspace_offsets(p)
+    nb = -(-p.N // p.q_block)
+    mw = -(-nb // 32)
+    B, H, D = p.B, p.H, p.D
+
+    def view(i, dtype, shape):
+        n = math.prod(shape)
+        esz = torch.tensor([], dtype=dtype).element_size()
+        return ws[off[i]:off[i] + n * esz].view(dtype).view(*shape)
+
+    return dict(qbar=view(0, torch.float32, (B, H, nb, D)), kbar=view(1, torch.float32, (B, H, nb, D)),
+                kbar16=view(2, torch.bfloat16, (B, H, nb, D)), vbar16=view(3, torch.bfloat16, (B, H, nb, D)),
+                cbias=view(4, torch.float32, (B, H, nb)), anchor=view(5, torch.float32, (B, H, D)),
+                mask=view(6, torch.int32, (B * H * nb, mw)), counts=view(7, torch.int32, (B * H * nb,)))
+
+
+def sol_col_capacity(p: sol_params) -> int:
+    return lib.sol_col_capacity(ctypes.byref(p))
+
+
+def sol_pool(p: sol_params, q, k, v, ws: torch.Tensor, stream=None):
+    _check(lib.sol_pool(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel() * ws.element_size(),
+                        _stream(stream)), "sol_pool")
+
+
+def sol_route(p: sol_params, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, stream=None):
+    _check(lib.sol_route(ctypes.byref(p), _ptr(ws), ws.numel() * ws.element_size(), _ptr(row_ptr), _ptr(col_idx),
+                         _stream(stream)), "sol_route")
+
+
+def sol_attn_fwd(p: sol_params, q, k, v, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                 o: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None):
+    _check(lib.sol_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel() * ws.element_size(),
+                            _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(lse), _stream(stream)), "sol_attn_fwd")
+
+
+def sol_last_device_status(stream=None):
+    _check(lib.sol_last_device_status(_stream(stream)), "device status")
+
+
+@dataclass
+class Buffers:
+    """Caller-owned device buffers of one problem shape (allocated by torch)."""
+    ws: torch.Tensor
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    o: torch.Tensor
+    lse: Optional[torch.Tensor]
+
+
+def alloc_buffers(p: sol_params, device, with_lse: bool = False) -> Buffers:
+    nqb = -(-p.N // p.q_block)
+    ws = torch.empty(max(1, sol_workspace_bytes(p)), dtype=torch.uint8, device=device)
+    row_ptr = torch.empty(p.B * p.H * nqb + 1, dtype=torch.int32, device=device)
+    col_idx = torch.empty(max(1, sol_col_capacity(p)), dtype=torch.int32, device=device)
+    o = torch.empty((p.B, p.N, p.H, p.D), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device=device) if with_lse else None
+    return Buffers(ws, row_ptr, col_idx, o, lse)
+
+
+def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
+    """Enqueue pool -> route -> attention on one stream; returns ``buf``."""
+    sol_pool(p, q, k, v, buf.ws, stream)
+    sol_route(p, buf.ws, buf.row_ptr, buf.col_idx, stream)
+    sol_attn_fwd(p, q, k, v, buf.ws, buf.row_ptr, buf.col_idx, buf.o, buf.lse, stream)
+    return buf
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
+              log_mass_bias: bool = False, scale: float = 0.0, with_lse: bool = False):
+    """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
+
+    Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.
+    """
+    B, N, H, D = q.shape
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(3) != 1 or t.stride() != q.stride():
+            raise ValueError("q, k, v must be bf16 CUDA tensors with identical strides and contiguous head dim")
+    p = make_params(B, N, H, D, tau, prefix_len, log_mass_bias, scale,
+                    in_strides=(q.stride(0), q.stride(1), q.stride(2)))
+    buf = alloc_buffers(p, q.device, with_lse)
+    forward(p, q, k, v, buf)
+    return buf.o, buf

@@ -143,13 +143,14 @@ def _one_head(w: Workload, b: int, h: int, tile_idx: np.ndarray):
 
 
 def generate(w: Workload, heads: Optional[Sequence[int]] = None, threads: Optional[int] = None,
-             out: Optional[tuple] = None):
+             out: Optional[tuple] = None, b_offset: int = 0):
     """Return (q, k, v) as uint16 bf16 bit arrays in BTHD layout [B, N, len(heads), D].
 
     ``heads`` selects a subset of head indices (default: all); the values of a
     head do not depend on which other heads are generated.  ``out`` may hold
     three preallocated uint16 arrays of that shape (e.g. views of pinned host
-    memory) to be filled in place.
+    memory) to be filled in place.  ``b_offset`` shifts the batch index of the
+    random streams, so that shard r of a larger batch draws sequence b_offset + b.
     """
     heads = list(range(w.H)) if heads is None else list(heads)
     shape = (w.B, w.N, len(heads), w.D)
@@ -159,7 +160,7 @@ def generate(w: Workload, heads: Optional[Sequence[int]] = None, threads: Option
 
     def work(job):
         b, slot = job
-        q, k, v = _one_head(w, b, heads[slot], tile_idx)
+        q, k, v = _one_head(w, b_offset + b, heads[slot], tile_idx)
         out[0][b, :, slot, :] = q
         out[1][b, :, slot, :] = k
         out[2][b, :, slot, :] = v

@@ -1,0 +1,156 @@
+/*
+ * sol.h -- C ABI of libsol.so: Sol block-sparse attention forward on B200 (sm_100a).
+ *
+ * The forward pass has three stages, each one entry point, enqueued in order
+ * on one CUDA stream (or ordered by the caller):
+ *
+ *   sol_pool      block centroids of Q, K, V (+ optional log-mass bias)
+ *   sol_route     block scores, per-row mean + tau*std threshold, CSR lists
+ *                 of exact key blocks
+ *   sol_attn_fwd  exact attention over the listed key blocks, one centroid
+ *                 term per unlisted block, merged in one fp32 online softmax
+ *
+ * Method sources (web pages; no code or equations are published):
+ *   - Star7 README "MiniMax H3 Activation Chunk & Attention Acceleration",
+ *     section 工作原理 > Sol: Q64/K64 blocks, tau = 1.0 threshold routing;
+ *     selected K/V blocks exact, unselected blocks contribute through their
+ *     K/V centroids, both merged in the same FP32 online softmax; the
+ *     audio-range KV sink is kept and prefix query rows attend densely.
+ *   - thakicloud "MiniMax-H3 ComfyUI accel stack", section 이 기술은 무엇인가:
+ *     tau counts standard deviations above the mean block score; strided
+ *     views of the fused QKV projection are passed without copies.
+ *   - Spark-H3 news page (comfyui-wiki), section "Spark-Attn이 바꾸는 것",
+ *     Spark-Reweight bullet and compressed-branch figure caption: the
+ *     log-mass bias restoring E[exp(x)] over exp(E[x]), scored against one
+ *     anchor per head, the mean video query.
+ *   - Star7 README, section 环境与分发: a native library that takes only
+ *     tensor addresses, shapes and the current CUDA stream, and refuses a
+ *     mismatched architecture naming required and detected capability.
+ *
+ * Conventions (all entry points):
+ *   - Every buffer is owned by the caller.  The library never allocates
+ *     device memory and never synchronises, except sol_last_device_status.
+ *   - Argument errors are reported synchronously, before anything is
+ *     enqueued.  Launch failures map to SOL_ERR_CUDA.  The first call on a
+ *     device checks that it is compute capability 10.0 (B200, sm_100a) and
+ *     returns SOL_ERR_UNSUPPORTED otherwise; sol_last_error_text() then
+ *     names the detected capability.
+ *   - Tensors are bf16 with the head dimension contiguous.  Q, K, V share
+ *     one set of element strides (in_stride_*), so strided views into a
+ *     fused QKV buffer are accepted; O has its own (out_stride_*).  Base
+ *     addresses must be 16-byte aligned and every stride a multiple of 8
+ *     elements.
+ *   - B == 0 or N == 0 is a valid empty problem: nothing is enqueued.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).
+ */
+#ifndef SOL_H_
+#define SOL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SOL_OK = 0,
+  SOL_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, stride, alignment or tau */
+  SOL_ERR_UNSUPPORTED = 2,   /* wrong GPU architecture, head dim or block size */
+  SOL_ERR_WORKSPACE = 3,     /* workspace smaller than sol_workspace_bytes() */
+  SOL_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  SOL_ERR_TIMEOUT = 5        /* a kernel's bounded wait expired (device status) */
+} sol_status;
+
+typedef struct {
+  int32_t B, N, H, D;        /* batch, rows of the packed sequence, heads, head dim (64 or 128) */
+  int32_t q_block, k_block;  /* rows per query / key block; the GPU path takes 64 and 64 */
+  float tau;                 /* threshold in std units above the row mean; finite or -INFINITY
+                                (-INFINITY makes every block exact) */
+  float scale;               /* softmax and score scale; 0 selects 1/sqrt(D) */
+  int32_t prefix_len;        /* rows [0, prefix_len) are the packed text/audio prefix:
+                                key blocks holding any of them are always exact (KV sink),
+                                query blocks holding any of them attend densely */
+  int32_t log_mass_bias;     /* 0: centroid logit s*q.kbar_j + log n_j;
+                                1: plus bias_j = log mean_t exp(s*a.k_t) - s*a.kbar_j with
+                                   anchor a = mean of the query rows >= prefix_len */
+  int64_t in_stride_b, in_stride_n, in_stride_h;    /* element strides of Q, K, V */
+  int64_t out_stride_b, out_stride_n, out_stride_h; /* element strides of O */
+} sol_params;
+
+/* Bytes of device workspace that sol_pool / sol_route / sol_attn_fwd share for
+ * one problem of this shape (centroids, bias, routing mask, row counts).
+ * Returns 0 for an invalid or empty problem. */
+size_t sol_workspace_bytes(const sol_params* p);
+
+/* Byte offsets, from the workspace base, of the pooled quantities that
+ * sol_pool / sol_route leave in the workspace, for inspection and tests:
+ *   offsets[0] qbar   fp32 [B, H, nqb, D]     offsets[1] kbar   fp32 [B, H, nkb, D]
+ *   offsets[2] kbar   bf16 [B, H, nkb, D]     offsets[3] vbar   bf16 [B, H, nkb, D]
+ *   offsets[4] centroid-logit offset fp32 [B, H, nkb] = log n_j (+ bias_j)
+ *   offsets[5] anchor fp32 [B, H, D] (log_mass_bias only)
+ *   offsets[6] exact-block bitmap uint32 [B*H*nqb, ceil(nkb/32)]
+ *   offsets[7] row counts int32 [B*H*nqb]
+ * with nqb = nkb = ceil(N/64).  Returns SOL_ERR_INVALID_ARG for a bad p or
+ * a NULL offsets array. */
+sol_status sol_workspace_offsets(const sol_params* p, int64_t offsets[8]);
+
+/* Worst-case number of CSR column entries: B*H*ceil(N/q_block)*ceil(N/k_block). */
+int64_t sol_col_capacity(const sol_params* p);
+
+/* sol_pool: block centroids (Star7 README 工作原理 > Sol; Spark-H3 news page,
+ * Spark-Reweight bullet).
+ *   q, k, v  [B, N, H, D] bf16 device pointers, strides p->in_stride_*.
+ *   ws       device workspace of ws_bytes >= sol_workspace_bytes(p) bytes,
+ *            256-byte aligned.  Receives, per (b, h, block): qbar, kbar as
+ *            fp32, kbar and vbar as bf16, the valid row count n_j, and the
+ *            centroid-logit offset log n_j (+ bias_j when log_mass_bias).
+ * Means are over each block's valid rows, accumulated in fp32. */
+sol_status sol_pool(const sol_params* p, const void* q, const void* k, const void* v,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* sol_route: block scores and CSR lists of exact key blocks (thakicloud blog,
+ * 이 기술은 무엇인가; Star7 README 工作原理 > Sol).
+ *   ws       workspace filled by sol_pool for the same p.
+ *   row_ptr  int32 [B*H*ceil(N/q_block) + 1] device, written: exclusive scan
+ *            of the per-row counts in (b, h, i) order; row_ptr[last] = nnz.
+ *   col_idx  int32 device, capacity sol_col_capacity(p); row r's exact key
+ *            blocks, ascending, at [row_ptr[r], row_ptr[r+1]).
+ * S_ij = s * qbar_i . kbar_j in fp32; block j is exact for row i iff
+ * S_ij > mean_j S_ij + tau * std_j S_ij (population std over all key
+ * blocks), or j is a sink block, or i is a dense (prefix) query block. */
+sol_status sol_route(const sol_params* p, void* ws, size_t ws_bytes,
+                     int32_t* row_ptr, int32_t* col_idx, void* stream);
+
+/* sol_attn_fwd: exact + centroid attention (Star7 README 工作原理 > Sol).
+ *   q, k, v  as for sol_pool; ws, row_ptr, col_idx as filled by sol_pool
+ *            and sol_route for the same p (the caller may substitute its own
+ *            CSR lists with the same layout, e.g. to replay a mask).
+ *   o        [B, N, H, D] bf16 device, strides p->out_stride_*; written.
+ *   lse      optional fp32 [B, H, N] device (natural-log normaliser); NULL
+ *            to skip.
+ * Row r of query block i: logits s*q_r.k_t over the rows t of the listed
+ * key blocks, and s*q_r.kbar_j + log n_j (+ bias_j) with value vbar_j for
+ * each unlisted key block j; one fp32 online softmax over all of them.
+ * Keys at rows >= N are masked; O rows >= N are not written. */
+sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const void* v,
+                        const void* ws, size_t ws_bytes, const int32_t* row_ptr,
+                        const int32_t* col_idx, void* o, float* lse, void* stream);
+
+/* Synchronises `stream`, then reports and clears the device-side status word
+ * that kernels set when a bounded wait expires (SOL_ERR_TIMEOUT) or a CSR
+ * entry is out of range (SOL_ERR_INVALID_ARG). */
+sol_status sol_last_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sol_status_string(sol_status s);
+
+/* Text of the last error raised on this thread (argument or CUDA detail);
+ * empty string if none. */
+const char* sol_last_error_text(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOL_H_ */

@@ -1,0 +1,118 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+and compare each stage with the fp64 oracle.
+
+Criteria (bf16 I/O, fp32 accumulate):
+  * pooled centroids: fp32 means within 1e-5 relative (+1e-6 absolute) of the
+    oracle; bf16 copies within one bf16 rounding of the oracle's mean;
+  * routing: the GPU mask equals the oracle's on every block whose score is
+    more than 1e-4 from its row threshold, and the GPU CSR equals the
+    oracle's CSR of the GPU mask bit for bit;
+  * attention: with the oracle run on the GPU's mask, max |O_gpu - O_ref| <=
+    2e-2 and mean |O_gpu - O_ref| <= 2e-3.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from block_sparse_video_sol_b200 import synth
+from oracle import sol_ref
+
+MAX_ABS, MEAN_ABS, BAND = 2e-2, 2e-3, 1e-4
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None):
+    from block_sparse_video_sol_b200 import sol
+    B, N, H, D = q.shape
+    strides = in_strides or (q.stride(0), q.stride(1), q.stride(2))
+    p = sol.make_params(B, N, H, D, tau=tau, prefix_len=prefix, log_mass_bias=lmb, in_strides=strides)
+    buf = sol.alloc_buffers(p, q.device, with_lse=with_lse)
+    sol.forward(p, q, k, v, buf)
+    sol.sol_last_device_status()
+    torch.cuda.synchronize()
+    return p, buf
+
+
+def gpu_mask(p, buf):
+    nb = -(-p.N // 64)
+    rp = buf.row_ptr.cpu().numpy().astype(np.int64)
+    ci = buf.col_idx[:int(rp[-1])].cpu().numpy().astype(np.int64)
+    return rp, ci, sol_ref.from_csr(rp, ci, (p.B, p.H, nb, nb))
+
+
+def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix):
+    """Pooled quantities of the given head indices vs the oracle."""
+    from block_sparse_video_sol_b200 import sol
+    w = sol.workspace_views(p, buf.ws)
+    s = 1.0 / math.sqrt(p.D)
+    qbar, kbar, vbar = sol_ref.pool(Qd, 64), sol_ref.pool(Kd, 64), sol_ref.pool(Vd, 64)
+    g = {k: w[k][:, heads].float().cpu().numpy().astype(np.float64) for k in ("qbar", "kbar", "kbar16", "vbar16", "cbias")}
+    np.testing.assert_allclose(g["qbar"], qbar, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(g["kbar"], kbar, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(g["kbar16"], kbar, rtol=2 ** -8, atol=1e-6)
+    np.testing.assert_allclose(g["vbar16"], vbar, rtol=2 ** -8, atol=1e-6)
+    logn = np.log(sol_ref.block_rows(p.N, 64).astype(np.float64))
+    want = logn[None, None, :] + (sol_ref.log_mass_bias(Qd, Kd, kbar, prefix, s, 64) if lmb else 0.0)
+    want = np.broadcast_to(want, g["cbias"].shape)
+    np.testing.assert_allclose(g["cbias"], want, rtol=0, atol=2e-4)
+    return qbar, kbar, vbar
+
+
+def check_route(p, buf, qbar, kbar, heads, tau, prefix):
+    """Mask parity outside the threshold band, and CSR bit-exactness."""
+    s = 1.0 / math.sqrt(p.D)
+    S = sol_ref.scores(qbar, kbar, s)
+    thr = sol_ref.thresholds(S, tau)
+    sel = sol_ref.route(S, tau, prefix, 64, 64)
+    rp, ci, gm = gpu_mask(p, buf)
+    # CSR bit-exact for the GPU's own mask (every head)
+    rp_ref, ci_ref = sol_ref.to_csr(gm)
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(ci, ci_ref)
+    g = gm[:, heads]
+    far = np.abs(S - thr[..., None]) > BAND if tau != -math.inf else np.ones_like(sel)
+    bad = (g != sel) & far
+    assert not bad.any(), f"{int(bad.sum())} mask mismatches outside the {BAND} band"
+    return gm, int(((g != sel) & ~far).sum())
+
+
+def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None):
+    """O (and lse) of the given heads vs the oracle run on the GPU mask."""
+    ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, log_mass_bias_on=lmb,
+                              mask_override=gm_heads, rows=rows)
+    O = buf.o[:, :, heads].float().cpu().numpy().astype(np.float64)
+    Oref = ref["O"]
+    keep = ~np.isnan(Oref)
+    err = np.abs(O[keep] - Oref[keep])
+    assert keep.any()
+    assert err.max() <= MAX_ABS, f"max abs err {err.max()}"
+    assert err.mean() <= MEAN_ABS, f"mean abs err {err.mean()}"
+    if buf.lse is not None:
+        L = buf.lse[:, heads].cpu().numpy().astype(np.float64)
+        k2 = ~np.isnan(ref["lse"])
+        np.testing.assert_allclose(L[k2], ref["lse"][k2], rtol=0, atol=2e-3)
+    return float(err.max()), float(err.mean())
+
+
+def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
+    """Generate a workload, run it on the GPU, check pool/route/attention on `heads`."""
+    q, k, v = synth.generate(w)
+    Q, K, V = to_dev(q), to_dev(k), to_dev(v)
+    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias)
+    heads = list(range(w.H)) if heads is None else list(heads)
+    Qd, Kd, Vd = (synth.bf16_bits_to_f64(x[:, :, heads]) for x in (q, k, v))
+    qbar, kbar, _ = check_pool(p, buf, Qd, Kd, Vd, heads, w.log_mass_bias, w.prefix)
+    gm, flips = check_route(p, buf, qbar, kbar, heads, w.tau, w.prefix)
+    rows = None
+    if rows_per_head:
+        rng = np.random.default_rng(seed_rows)
+        rows = {(b, hh): np.sort(rng.choice(w.N, size=min(rows_per_head, w.N), replace=False))
+                for b in range(w.B) for hh in range(len(heads))}
+    errs = check_attention(p, buf, Qd, Kd, Vd, gm[:, heads], heads, w.tau, w.prefix, w.log_mass_bias, rows)
+    return dict(flips=flips, errs=errs, nnz=int(buf.row_ptr[-1].item()), p=p, buf=buf)

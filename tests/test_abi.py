@@ -1,0 +1,89 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry
+point, and validates arguments synchronously (no compute is launched)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sol():
+    from block_sparse_video_sol_b200 import build
+    build.build()
+    from block_sparse_video_sol_b200 import sol as mod
+    return mod
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(sol_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported(sol):
+    declared = _declared()
+    assert {"sol_pool", "sol_route", "sol_attn_fwd"} <= declared
+    for name in declared:
+        assert hasattr(sol.lib, name), name
+    assert declared == set(sol.EXPORTS)
+
+
+def test_status_strings(sol):
+    for code, name in enumerate(["SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_WORKSPACE",
+                                 "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT"]):
+        assert sol.lib.sol_status_string(code).decode() == name
+
+
+def test_workspace_sizes(sol):
+    p = sol.make_params(1, 32768, 56, 128)
+    nb = 512
+    ws = sol.sol_workspace_bytes(p)
+    # two fp32 and two bf16 centroid arrays dominate
+    assert ws >= 56 * nb * 128 * (4 + 4 + 2 + 2)
+    assert ws < 56 * nb * 128 * 12 * 1.05
+    assert sol.sol_col_capacity(p) == 56 * nb * nb
+    off = sol.sol_workspace_offsets(p)
+    assert off == sorted(off) and all(o % 256 == 0 for o in off) and off[-1] < ws
+    assert sol.sol_workspace_bytes(sol.make_params(1, 0, 56, 128)) == 0
+    assert sol.sol_workspace_bytes(sol.make_params(1, 100, 56, 96)) == 0   # bad head dim
+
+
+def _call_pool(sol, p, ws_bytes=1 << 30, ptr=4096):
+    return sol.lib.sol_pool(ctypes.byref(p), ptr, ptr, ptr, ptr, ws_bytes, None)
+
+
+def test_argument_validation_is_synchronous(sol):
+    ok = sol.make_params(1, 1000, 4, 128)
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 96)) == sol.SOL_ERR_UNSUPPORTED
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, q_block=32, k_block=32)) == sol.SOL_ERR_UNSUPPORTED
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, tau=math.nan)) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, tau=math.inf)) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, prefix_len=1001)) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, in_strides=(512000, 516, 128))) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 70000, 4, 128)) == sol.SOL_ERR_UNSUPPORTED
+    assert _call_pool(sol, ok, ptr=4100) == sol.SOL_ERR_INVALID_ARG          # misaligned
+    assert _call_pool(sol, ok, ws_bytes=10) == sol.SOL_ERR_WORKSPACE
+    assert sol.lib.sol_pool(ctypes.byref(ok), None, 4096, 4096, 4096, 1 << 30, None) == sol.SOL_ERR_INVALID_ARG
+    assert "NULL" in sol.lib.sol_last_error_text().decode()
+    assert sol.lib.sol_pool(None, None, None, None, None, 0, None) == sol.SOL_ERR_INVALID_ARG
+    # an empty problem is valid and enqueues nothing
+    assert _call_pool(sol, sol.make_params(0, 1000, 4, 128), ptr=0) == sol.SOL_OK
+    assert sol.lib.sol_route(ctypes.byref(sol.make_params(1, 0, 4, 128)), None, 0, None, None, None) == sol.SOL_OK
+    assert sol.lib.sol_attn_fwd(ctypes.byref(sol.make_params(1, 0, 4, 64)), None, None, None, None, 0,
+                                None, None, None, None, None) == sol.SOL_OK
+
+
+def test_no_gpu_reports_cuda_error(sol):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _call_pool(sol, sol.make_params(1, 1000, 4, 128))
+    assert st in (sol.SOL_ERR_CUDA, sol.SOL_ERR_UNSUPPORTED)

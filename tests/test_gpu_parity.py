@@ -1,0 +1,134 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_video_sol_b200 import synth
+from oracle import sol_ref
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from block_sparse_video_sol_b200 import build
+    build.build()
+
+
+def test_tiny_workload_full():
+    r = parity.full_check(synth.tiny())
+    assert r["flips"] <= 2
+
+
+@pytest.mark.parametrize("lmb", [False, True])
+def test_ragged_prefix_batch2_d64(lmb):
+    # N = 1000 (tail block of 40 rows), prefix 100 (mixed block 1), B = 2
+    w = synth.Workload("ragged", B=2, H=3, N=1000, D=64, grid=(9, 10, 10), n_topics=8, prefix=100,
+                       tau=0.5, seed=7, log_mass_bias=lmb)
+    parity.full_check(w)
+
+
+@pytest.mark.parametrize("lmb", [False, True])
+def test_ragged_prefix_d128(lmb):
+    w = synth.Workload("ragged128", B=1, H=4, N=777, D=128, grid=(4, 1, 191), n_topics=8, prefix=13,
+                       tau=1.0, seed=8, log_mass_bias=lmb)
+    parity.full_check(w)
+
+
+def test_h56_n4096_full():
+    r = parity.full_check(synth.h56_n4096())
+    nb = 64
+    dens = r["nnz"] / (56 * nb * nb)
+    assert 0.05 < dens < 0.3
+
+
+def test_all_exact_matches_dense_sdpa():
+    w = synth.Workload("dense", B=1, H=2, N=700, D=128, grid=(7, 10, 10), n_topics=4, tau=-math.inf, seed=9)
+    q, k, v = synth.generate(w)
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    p, buf = parity.run_gpu(Q, K, V, -math.inf, 0, False)
+    assert int(buf.row_ptr[-1]) == 2 * 11 * 11
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.float().transpose(1, 2), K.float().transpose(1, 2), V.float().transpose(1, 2)).transpose(1, 2)
+    err = (buf.o.float() - ref).abs()
+    assert err.max().item() <= parity.MAX_ABS and err.mean().item() <= parity.MEAN_ABS
+
+
+def test_prefix_equals_n_is_dense():
+    w = synth.Workload("alldense", B=1, H=2, N=300, D=64, grid=(3, 10, 10), n_topics=4, seed=10)
+    q, k, v = synth.generate(w)
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    p, buf = parity.run_gpu(Q, K, V, 1.0, 300, True)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.float().transpose(1, 2), K.float().transpose(1, 2), V.float().transpose(1, 2)).transpose(1, 2)
+    assert (buf.o.float() - ref).abs().max().item() <= parity.MAX_ABS
+
+
+def test_fused_qkv_strided_views():
+    w = synth.Workload("fused", B=2, H=4, N=640, D=128, grid=(4, 10, 16), n_topics=8, tau=1.0, seed=11)
+    q, k, v = synth.generate(w)
+    qkv = torch.empty((2, 640, 3, 4, 128), dtype=torch.bfloat16, device="cuda")
+    qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2] = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    Qv, Kv, Vv = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    assert Qv.stride(1) == 3 * 4 * 128
+    p, buf = parity.run_gpu(Qv, Kv, Vv, 1.0, 0, False)
+    p2, buf2 = parity.run_gpu(parity.to_dev(q), parity.to_dev(k), parity.to_dev(v), 1.0, 0, False)
+    assert torch.equal(buf.row_ptr, buf2.row_ptr)
+    assert torch.equal(buf.o, buf2.o)
+
+
+@pytest.mark.parametrize("N", [1, 5, 63, 64, 65])
+def test_small_and_single_block(N):
+    w = synth.Workload(f"small{N}", B=1, H=2, N=N, D=64, grid=(1, 1, N), n_topics=2, tau=0.0, seed=12 + N)
+    parity.full_check(w)
+
+
+def test_empty_problem_is_noop():
+    from block_sparse_video_sol_b200 import sol
+    p = sol.make_params(1, 0, 4, 128)
+    sol.sol_pool(p, None, None, None, torch.empty(1, dtype=torch.uint8, device="cuda"))
+    sol.sol_last_device_status()
+
+
+def test_max_key_blocks():
+    # N = 65536 is the longest sequence the routing kernel takes (1024 key blocks)
+    w = synth.Workload("maxN", B=1, H=2, N=65536, D=128, grid=(64, 32, 32), n_topics=128, seed=13)
+    parity.full_check(w, rows_per_head=300)
+
+
+def test_bad_csr_entry_is_reported_not_read():
+    from block_sparse_video_sol_b200 import sol
+    w = synth.tiny()
+    q, k, v = synth.generate(w)
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    p, buf = parity.run_gpu(Q, K, V, 1.0, 0, False)
+    bad = buf.col_idx.clone()
+    bad[0] = 10 ** 6
+    sol.sol_attn_fwd(p, Q, K, V, buf.ws, buf.row_ptr, bad, buf.o)
+    with pytest.raises(sol.SolError) as e:
+        sol.sol_last_device_status()
+    assert e.value.status == sol.SOL_ERR_INVALID_ARG
+    sol.sol_last_device_status()   # cleared
+
+
+@pytest.mark.slow
+def test_h56_n32768_sampled():
+    # full problem on the GPU; oracle on two heads, sampled rows
+    w = synth.h56_sweep(32768)
+    r = parity.full_check(w, heads=[0, 41], rows_per_head=256)
+    assert r["flips"] <= 20
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("lmb", [False, True])
+def test_joint_sequence_sampled(lmb):
+    w = synth.h56_joint()
+    if lmb:
+        w = synth.Workload(w.name + "_lmb", w.B, w.H, w.N, w.D, w.grid, w.n_topics, w.prefix, w.tau, w.seed, True)
+    r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=1)
+    assert r["flips"] <= 20
