@@ -251,3 +251,93 @@ const char* sol_status_string(sol_status s) {
 const char* sol_last_error_text(void) { return t_err; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// sol_route_static: sol_route for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc or hand the library extra device
+// buffers: a host framework that owns every device allocation through its
+// own fixed-budget pool, or a code path that must not allocate (allocation
+// can synchronise the device or fail at an inconvenient time).  For them this
+// entry point keeps sol_route's scratch -- the exact-block bitmap and the
+// per-row counts -- in one fixed array inside the library, so the caller only
+// provides the pooled input (the workspace sol_pool filled, of which only the
+// part before the bitmap is read) and the CSR outputs.
+//
+// The array holds kRouteScratchBytes (8 MiB); every GPU that loads the
+// library keeps it until the process exits.  A problem needs
+// B*H*ceil(N/64)*ceil(ceil(N/64)/32)*4 bytes of bitmap (rounded up to 256)
+// plus B*H*ceil(N/64)*4 bytes of counts; larger problems are rejected with
+// SOL_ERR_UNSUPPORTED.  Every call shares the array and it keeps the last
+// call's contents; each call writes every bitmap word and count it later
+// reads, so nothing needs clearing.  Calls whose executions overlap on the GPU
+// (different streams, or different host threads, on one device) race on the
+// array.  The first call on a device looks up the array's device address
+// (cudaGetSymbolAddress) and caches it; make that first call before any
+// stream capture.
+static constexpr size_t kRouteScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char sol_route_scratch[kRouteScratchBytes];
+
+namespace sol {
+namespace {
+
+unsigned char* g_route_scratch_ptr[kMaxDevices];
+std::mutex g_route_scratch_mu;
+
+// Device address of this device's copy of the array (the host-side name of a
+// __device__ variable is only a stand-in, never a device address).
+sol_status route_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_route_scratch_mu);
+  if (!g_route_scratch_ptr[dev]) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, sol_route_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(route scratch)");
+    g_route_scratch_ptr[dev] = static_cast<unsigned char*>(addr);
+  }
+  *out = g_route_scratch_ptr[dev];
+  return SOL_OK;
+}
+
+}  // namespace
+}  // namespace sol
+
+extern "C" sol_status sol_route_static(const sol_params* p, const void* ws, size_t ws_bytes, int32_t* row_ptr,
+                                       int32_t* col_idx, void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!ws || !row_ptr || !col_idx) return fail(SOL_ERR_INVALID_ARG, "sol_route_static: NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(SOL_ERR_INVALID_ARG, "sol_route_static: workspace not 256-byte aligned");
+  const WsLayout L = ws_layout(*p);
+  if (ws_bytes < L.mask)
+    return fail(SOL_ERR_WORKSPACE, "sol_route_static: pooled workspace %zu < %zu bytes", ws_bytes, L.mask);
+  const size_t rows = (size_t)p->B * p->H * L.nqb;
+  const size_t mask_bytes = align256(rows * L.mask_words * 4);
+  const size_t need = mask_bytes + rows * 4;
+  if (need > kRouteScratchBytes)
+    return fail(SOL_ERR_UNSUPPORTED,
+                "sol_route_static: this problem needs %zu bytes of routing scratch; the built-in array holds %zu "
+                "(use sol_route with a caller-allocated workspace)", need, kRouteScratchBytes);
+  if ((s = check_arch()) != SOL_OK) return s;
+  unsigned char* scratch = nullptr;
+  if ((s = route_scratch(&scratch)) != SOL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RouteArgs a{};
+  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
+  a.B = p->B; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
+  a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
+  a.n_dense = a.n_sink;
+  a.scale = eff_scale(p); a.tau = p->tau;
+  a.mask = reinterpret_cast<uint32_t*>(scratch);
+  a.counts = reinterpret_cast<int32_t*>(scratch + mask_bytes);
+  cudaError_t e = launch_route(a, p->D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_route_static launch");
+  e = launch_scan_compact(a.mask, a.counts, (int)rows, L.mask_words, row_ptr, col_idx, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_route_static scan/compact launch");
+  return SOL_OK;
+}

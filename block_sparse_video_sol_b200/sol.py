@@ -23,8 +23,8 @@ lib = ctypes.CDLL(_LIB_PATH)
 SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(6)
 
 # Every entry point declared in include/sol.h.
-EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_attn_fwd",
-           "sol_last_device_status", "sol_status_string", "sol_last_error_text")
+EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
+           "sol_attn_fwd", "sol_last_device_status", "sol_status_string", "sol_last_error_text")
 
 
 class sol_params(ctypes.Structure):
@@ -48,6 +48,8 @@ lib.sol_pool.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 lib.sol_pool.restype = ctypes.c_int
 lib.sol_route.argtypes = [_P, _vp, ctypes.c_size_t, _vp, _vp, _vp]
 lib.sol_route.restype = ctypes.c_int
+lib.sol_route_static.argtypes = [_P, _vp, ctypes.c_size_t, _vp, _vp, _vp]
+lib.sol_route_static.restype = ctypes.c_int
 lib.sol_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
 lib.sol_attn_fwd.restype = ctypes.c_int
 lib.sol_last_device_status.argtypes = [_vp]
@@ -129,6 +131,13 @@ def sol_pool(p: sol_params, q, k, v, ws: torch.Tensor, stream=None):
 def sol_route(p: sol_params, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, stream=None):
     _check(lib.sol_route(ctypes.byref(p), _ptr(ws), ws.numel() * ws.element_size(), _ptr(row_ptr), _ptr(col_idx),
                          _stream(stream)), "sol_route")
+
+
+def sol_route_static(p: sol_params, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                     stream=None):
+    """Routing without caller scratch (see include/sol.h); ws may hold only the pooled part."""
+    _check(lib.sol_route_static(ctypes.byref(p), _ptr(ws), ws.numel() * ws.element_size(), _ptr(row_ptr),
+                                _ptr(col_idx), _stream(stream)), "sol_route_static")
 
 
 def sol_attn_fwd(p: sol_params, q, k, v, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,

@@ -137,6 +137,26 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
                         const void* ws, size_t ws_bytes, const int32_t* row_ptr,
                         const int32_t* col_idx, void* o, float* lse, void* stream);
 
+/* sol_route_static: the routing of sol_route without any caller-provided
+ * scratch, for callers that cannot allocate device memory (a host framework
+ * that owns every device allocation through a fixed-budget pool, or a code
+ * path that must not allocate).  The pages describe no such entry point; it
+ * has no counterpart in the method's sources.
+ *   ws       the workspace sol_pool filled for the same p; only its pooled
+ *            part is read, so ws_bytes may be as small as offsets[6] of
+ *            sol_workspace_offsets (the bitmap offset).
+ *   row_ptr, col_idx  outputs exactly as for sol_route (identical values).
+ * The bitmap and row counts live in one fixed 8 MiB device array inside the
+ * library, held by every GPU that loads it until the process exits; problems
+ * needing more than 8 MiB (B*H*ceil(N/64) rows x (ceil(N/64/32) words + 1
+ * count) x 4 bytes, bitmap rounded up to 256 bytes) are rejected with
+ * SOL_ERR_UNSUPPORTED.  The library allocates nothing.  All calls share the
+ * array: calls that overlap on the GPU race on it.  The first call on a
+ * device looks up the array's device address; make it before any stream
+ * capture. */
+sol_status sol_route_static(const sol_params* p, const void* ws, size_t ws_bytes,
+                            int32_t* row_ptr, int32_t* col_idx, void* stream);
+
 /* Synchronises `stream`, then reports and clears the device-side status word
  * that kernels set when a bounded wait expires (SOL_ERR_TIMEOUT) or a CSR
  * entry is out of range (SOL_ERR_INVALID_ARG). */
