@@ -134,6 +134,29 @@ def dist_env():
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def shard_b_offset(rank: int, w: synth.Workload) -> int:
+    """Batch index of this rank's first sequence: rank r runs sequences r*B .. r*B+B-1 of the job."""
+    return rank * w.B
+
+
+def job_reduce(values, device, world: int):
+    """Max-over-ranks of the timing entries and sum of the work entry.
+
+    ``values`` = (timed ms, e2e ms, work); returns the same triple for the whole
+    job: the slowest rank's times and the total work.  Collective only when
+    world > 1 (plumbing, not the data path).
+    """
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        mx, sm = t.clone(), t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        return mx[0].item(), mx[1].item(), sm[2].item()
+    return t[0].item(), t[1].item(), t[2].item()
+
+
 def oracle_sample(w: synth.Workload, heads, b_offset=0):
     """Time the fp64 oracle on a head subset of the workload; returns (seconds, rows x keys)."""
     from oracle import sol_ref
@@ -197,7 +220,8 @@ def run_ours(args, w):
     # this rank's sequence: batch element `rank` of a world-size batch (pinned host copies for e2e)
     shape = (w.B, w.N, w.H, w.D)
     host = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-    synth.generate(w, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host), b_offset=rank * w.B)
+    synth.generate(w, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host),
+                   b_offset=shard_b_offset(rank, w))
     q, k, v = (h.to(dev) for h in host)
     p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias)
     buf = sol.alloc_buffers(p, dev)
@@ -263,15 +287,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    t = torch.tensor([total_ms, e2e_ms, flop], dtype=torch.float64, device=dev)
-    if world > 1:
-        mx = t.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = t.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        total_ms, e2e_ms, flop_all = mx[0].item(), mx[1].item(), sm[2].item()
-    else:
-        flop_all = flop
+    total_ms, e2e_ms, flop_all = job_reduce((total_ms, e2e_ms, flop), dev, world)
     if rank == 0:
         peaks = read_peaks()
         ms_step = total_ms / args.steps

@@ -47,16 +47,23 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile csrc/*.cu for sm_100a and link libsol.so; returns its path."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, trace: bool = False) -> str:
+    """Compile csrc/*.cu for sm_100a and link libsol.so; returns its path.
+
+    ``trace`` builds a separate libsol_trace.so with the attention kernel's
+    phase trace compiled in (for pipeline analysis; not used by the product).
+    """
+    out = OUT if not trace else os.path.join(PKG, "libsol_trace.so")
+    if not force and not trace and up_to_date():
         return OUT
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    if trace:
+        extra.append("-DSOL_TRACE")
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + (".trace.o" if trace else ".o"))
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -69,14 +76,15 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         for obj, log in results:
             if log.strip():
                 print(f"== {os.path.basename(obj)}\n{log}", file=sys.stderr)
-    tmp = OUT + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-cudart=static"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv,
+                trace="--trace" in sys.argv))

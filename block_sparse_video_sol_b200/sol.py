@@ -15,7 +15,7 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsol.so")
+_LIB_PATH = os.environ.get("SOL_LIB_PATH") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsol.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"libsol.so not built ({_LIB_PATH}); run `python -m block_sparse_video_sol_b200.build`")
 lib = ctypes.CDLL(_LIB_PATH)
