@@ -17,15 +17,17 @@
 // p = 0 there (its exponentials are skipped, warp-uniformly).  Then come the
 // centroid tiles: 128 centroids each, the half's selected blocks masked.
 //
-// Roles (6 warps):
-//   warp 0     TMA producer: Q once, then K and V tiles into a 2-stage ring.
+// Roles (7 warps):
+//   warp 0     TMA producer: Q once, then the K tiles into a 3-stage ring.
+//   warp 6     TMA producer: the V tiles into a 2-stage ring.
 //   warp 1     MMA issuer (one lane): S_b = Q K^T into TMEM buffer b = t%2,
-//              then O += P V with P read from TMEM (P overwrites S_b as bf16).
+//              then O += P V with P read from its own TMEM buffer.
 //   warps 2-5  softmax, one thread per row (TMEM lane): online max/sum in
 //              fp32 with lazy rescaling (O in TMEM is rescaled only when a
 //              row's max grows by more than 2^8), P written back to TMEM,
 //              final normalisation and bf16 store.
-// TMEM: S0 = columns [0,128), S1 = [128,256), O = [256, 256+D).
+// TMEM: S0 = columns [0,128), S1 = [128,256), O = [256, 256+D),
+//       P0 = [384, 448), P1 = [448, 512) (bf16 pairs).
 // Every mbarrier wait is bounded; on expiry the kernel raises
 // SOL_ERR_TIMEOUT, stops issuing, drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -36,8 +38,21 @@
 namespace sol {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 2;
+constexpr int kThreads = 224;
+constexpr int kKStages = 3;   // K tiles in flight (needed first, by QK)
+constexpr int kVStages = 2;   // V tiles in flight (needed a softmax later, by PV)
+
+// Optional phase trace (build with -DSOL_TRACE): clock64() stamps of one CTA's
+// roles for its first kTraceSteps S tiles, read back with sol_debug_trace().
+#ifdef SOL_TRACE
+constexpr int kTraceSteps = 256;
+__device__ long long g_trace[16 * kTraceSteps];
+#define SOL_TRACE_AT(slot, step) \
+  do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (step) < kTraceSteps) \
+         g_trace[(slot) * kTraceSteps + (step)] = clock64(); } while (0)
+#else
+#define SOL_TRACE_AT(slot, step) do { } while (0)
+#endif
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr float kRescale = 8.0f;   // log2 units: rescale O when the max grows by more than 2^8
 constexpr float kLog2e = 1.4426950408889634f;
@@ -50,13 +65,13 @@ struct Cfg {
   static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
   static constexpr int kChunkBytes = 128 * 128;        // one chunk of a 128-row tile
   static constexpr int kTileBytes = 128 * D * 2;       // Q, K or V tile of 128 rows
-  static constexpr int kSmemTiles = kTileBytes * (1 + 2 * kStages);
+  static constexpr int kSmemTiles = kTileBytes * (1 + kKStages + kVStages);
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done, final_mma;
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2], final_mma;
 };
 
 struct Extra {
@@ -198,8 +213,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::kTileBytes;
-  uint8_t* sV = sK + kStages * C::kTileBytes;
-  Extra& x = *reinterpret_cast<Extra*>(sV + kStages * C::kTileBytes);
+  uint8_t* sV = sK + kKStages * C::kTileBytes;
+  Extra& x = *reinterpret_cast<Extra*>(sV + kVStages * C::kTileBytes);
   Bars& bar = x.bar;
   volatile int* abort_flag = &x.abort_flag;
 
@@ -212,12 +227,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   // ---- set-up: barriers, TMEM, routing lists --------------------------------------------------
   if (tid == 0) {
     mbar_init(&bar.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar.k_full[s], 1); mbar_init(&bar.v_full[s], 1);
-      mbar_init(&bar.k_empty[s], 1); mbar_init(&bar.v_empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) { mbar_init(&bar.k_full[s], 1); mbar_init(&bar.k_empty[s], 1); }
+    for (int s = 0; s < kVStages; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.s_full[s], 1); mbar_init(&bar.s_free[s], 4); mbar_init(&bar.p_full[s], 4);
+      mbar_init(&bar.o_done[s], 1);
     }
-    for (int s = 0; s < 2; ++s) { mbar_init(&bar.s_full[s], 1); mbar_init(&bar.p_full[s], 4); }
-    mbar_init(&bar.o_done, 1);
     mbar_init(&bar.final_mma, 1);
     x.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -294,17 +309,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   const int n_ex = (x.n_union + 1) >> 1;
   const int T = n_ex + x.n_cent;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == 6) {
+    // ---------------------------------------------------------------- TMA producers
+    // warp 0: Q and the K tiles (kKStages ring); warp 6: the V tiles
+    // (kVStages ring).  Each runs ahead on its own ring.
     if (lane == 0) {
-      int nk = 0, nv = 0;   // K / V tile loads issued
+      const bool is_k = warp == 0;
+      const int nst = is_k ? kKStages : kVStages;
+      const CUtensorMap* m4 = is_k ? &mk : &mv;
+      const CUtensorMap* m3 = is_k ? &mkb : &mvb;
+      uint8_t* ring = is_k ? sK : sV;
+      int nl = 0;   // tile loads issued
       bool ok = true;
-      mbar_expect_tx(&bar.q_full, C::kTileBytes);
-      for (int hf = 0; hf < 2; ++hf)
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + c * C::kChunkBytes + hf * (C::kChunkBytes / 2), &mq, c * 64, h, 64 * (i0 + hf), b, &bar.q_full);
+      if (is_k) {
+        mbar_expect_tx(&bar.q_full, C::kTileBytes);
+        for (int hf = 0; hf < 2; ++hf)
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sQ + c * C::kChunkBytes + hf * (C::kChunkBytes / 2), &mq, c * 64, h, 64 * (i0 + hf), b,
+                        &bar.q_full);
+      }
       for (int t = 0; t < T && ok; ++t) {
-        const int s = t % kStages, n = t / kStages;
+        const int s = t % nst, n = t / nst;
         int j0 = 0, j1 = 0, ct = -1;
         if (t < n_ex) {
           j0 = x.list[2 * t] & 0xffff;
@@ -312,68 +337,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         } else {
           ct = x.cent[t - n_ex];
         }
-        ok = wait_bar(&bar.k_empty[s], (n & 1) ^ 1, abort_flag, a.status);
-        if (!ok) break;
-        mbar_expect_tx(&bar.k_full[s], C::kTileBytes);
-        ++nk;
-        uint8_t* dk = sK + s * C::kTileBytes;
+        uint64_t* empty = is_k ? &bar.k_empty[s] : &bar.v_empty[s];
+        uint64_t* full = is_k ? &bar.k_full[s] : &bar.v_full[s];
+        if (!(ok = wait_bar(empty, (n & 1) ^ 1, abort_flag, a.status))) break;
+        SOL_TRACE_AT(is_k ? 7 : 8, t);
+        mbar_expect_tx(full, C::kTileBytes);
+        ++nl;
+        uint8_t* dst = ring + s * C::kTileBytes;
         for (int c = 0; c < C::kChunks; ++c) {
           if (ct < 0) {
-            tma_load_4d(dk + c * C::kChunkBytes, &mk, c * 64, h, 64 * j0, b, &bar.k_full[s]);
-            tma_load_4d(dk + c * C::kChunkBytes + C::kChunkBytes / 2, &mk, c * 64, h, 64 * j1, b, &bar.k_full[s]);
+            tma_load_4d(dst + c * C::kChunkBytes, m4, c * 64, h, 64 * j0, b, full);
+            tma_load_4d(dst + c * C::kChunkBytes + C::kChunkBytes / 2, m4, c * 64, h, 64 * j1, b, full);
           } else {
-            tma_load_3d(dk + c * C::kChunkBytes, &mkb, c * 64, 128 * ct, (int)bh, &bar.k_full[s]);
-          }
-        }
-        ok = wait_bar(&bar.v_empty[s], (n & 1) ^ 1, abort_flag, a.status);
-        if (!ok) break;
-        mbar_expect_tx(&bar.v_full[s], C::kTileBytes);
-        ++nv;
-        uint8_t* dv = sV + s * C::kTileBytes;
-        for (int c = 0; c < C::kChunks; ++c) {
-          if (ct < 0) {
-            tma_load_4d(dv + c * C::kChunkBytes, &mv, c * 64, h, 64 * j0, b, &bar.v_full[s]);
-            tma_load_4d(dv + c * C::kChunkBytes + C::kChunkBytes / 2, &mv, c * 64, h, 64 * j1, b, &bar.v_full[s]);
-          } else {
-            tma_load_3d(dv + c * C::kChunkBytes, &mvb, c * 64, 128 * ct, (int)bh, &bar.v_full[s]);
+            tma_load_3d(dst + c * C::kChunkBytes, m3, c * 64, 128 * ct, (int)bh, full);
           }
         }
       }
       // drain: every armed load has landed before the CTA may exit
-      for (int s = 0; s < kStages; ++s) {
-        const int kc = (nk + kStages - 1 - s) / kStages, vc = (nv + kStages - 1 - s) / kStages;
-        if (kc) drain_bar(&bar.k_full[s], (kc - 1) & 1, a.status);
-        if (vc) drain_bar(&bar.v_full[s], (vc - 1) & 1, a.status);
+      for (int s = 0; s < nst; ++s) {
+        const int cnt = (nl + nst - 1 - s) / nst;
+        if (cnt) drain_bar(is_k ? &bar.k_full[s] : &bar.v_full[s], (cnt - 1) & 1, a.status);
       }
-      drain_bar(&bar.q_full, 0, a.status);
+      if (is_k) drain_bar(&bar.q_full, 0, a.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // Issue order QK(0), QK(1), QK(2), PV(0), QK(3), PV(1), QK(4), ...: the
+    // tensor pipe runs in order and issuing blocks for about as long as the
+    // MMAs take, so the QKs run ahead and S(u+1), S(u+2) are ready before the
+    // softmax needs them.  QK(g) reuses S_(g%2) once the softmax has read
+    // S(g-2) (it releases S right after loading it).
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       const uint32_t o_tmem = tmem + 256;
       bool ok = wait_bar(&bar.q_full, 0, abort_flag, a.status);
-      auto pv = [&](int u) -> bool {
-        const int s = u % kStages, n = u / kStages, bb = u & 1;
-        if (!wait_bar(&bar.p_full[bb], (u >> 1) & 1, abort_flag, a.status)) return false;
-        if (!wait_bar(&bar.v_full[s], n & 1, abort_flag, a.status)) return false;
+      auto qk = [&](int g) -> bool {
+        const int s = g % kKStages, n = g / kKStages, bb = g & 1;
+        if (!wait_bar(&bar.k_full[s], n & 1, abort_flag, a.status)) return false;
+        if (g >= 2 && !wait_bar(&bar.s_free[bb], ((g >> 1) - 1) & 1, abort_flag, a.status)) return false;
         fence_after();
-        const uint32_t vb = v_addr + s * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(o_tmem, tmem + bb * 128 + kk * 8, sdesc(vb + kk * 2048, C::kChunkBytes, 1024), id_pv,
-                 (u > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.v_empty[s]);
-        mma_commit(&bar.o_done);
-        return true;
-      };
-      for (int t = 0; t < T && ok; ++t) {
-        const int s = t % kStages, n = t / kStages, bb = t & 1;
-        ok = wait_bar(&bar.k_full[s], n & 1, abort_flag, a.status);
-        if (!ok) break;
-        fence_after();
+        SOL_TRACE_AT(4, g);
         const uint32_t kb = k_addr + s * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -382,21 +387,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         }
         mma_commit(&bar.s_full[bb]);
         mma_commit(&bar.k_empty[s]);
-        if (t >= 1) ok = pv(t - 1);
+        return true;
+      };
+      auto pv = [&](int u) -> bool {
+        const int s = u % kVStages, n = u / kVStages, bb = u & 1;
+        if (!wait_bar(&bar.p_full[bb], (u >> 1) & 1, abort_flag, a.status)) return false;
+        SOL_TRACE_AT(5, u);
+        if (!wait_bar(&bar.v_full[s], n & 1, abort_flag, a.status)) return false;
+        fence_after();
+        const uint32_t vb = v_addr + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(o_tmem, tmem + 384 + 64 * bb + kk * 8, sdesc(vb + kk * 2048, C::kChunkBytes, 1024), id_pv,
+                 (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar.v_empty[s]);
+        mma_commit(&bar.o_done[bb]);
+        return true;
+      };
+      for (int g = 0; g < 3 && g < T && ok; ++g) ok = qk(g);
+      for (int u = 0; u < T && ok; ++u) {
+        ok = pv(u);
+        if (ok && u + 3 < T) ok = qk(u + 3);
       }
-      if (ok && T > 0) pv(T - 1);
       // drain: all issued MMAs complete before TMEM is released
       mma_commit(&bar.final_mma);
       drain_bar(&bar.final_mma, 0, a.status);
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ---------------------------------------------------------------- softmax warpgroup
+    // One pass per S tile: the needed columns are read once (S is then
+    // released to the next QK), masked, maxed, exponentiated and stored as bf16
+    // P into its own TMEM buffer P_(u%2), once PV(u-2), the last reader of
+    // that buffer, is complete.  PV completions are waited for only there, for
+    // a rescale of O (PV(u-1)) and before the epilogue (PV(T-1)).  PV(v)
+    // completes o_done[v%2]; the next completion of that barrier needs P(v+2),
+    // which this warpgroup has not produced yet, so each parity wait is exact.
     const int sub = warp & 3;                 // TMEM sub-partition = rows 32*sub .. 32*sub+31
     const int r = 32 * sub + lane;            // row of the tile
     const int hf = r >> 6;                    // query block half (warp-uniform)
     const bool present = x.present[hf] != 0;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
+    const uint32_t o_addr = lane_addr + 256;
     const float sl2 = a.scale * kLog2e;
+    const bool tracer = warp == 2 && lane == 0;
     float m_run = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
@@ -404,6 +437,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       ok = __all_sync(0xffffffffu, wait_bar(&bar.s_full[bb], (t >> 1) & 1, abort_flag, a.status));
       if (!ok) break;
       fence_after();
+      if (tracer) SOL_TRACE_AT(0, t);
       // which 64-column halves of this S tile the row uses, and their additive offsets
       bool need0, need1;
       const float *add0, *add1;
@@ -422,27 +456,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         add1 = x.cent_add[slot][hf] + 64;
       }
       const uint32_t s_addr = lane_addr + bb * 128;
-      // pass 1: row max of this tile (log2 units)
-      float mt = -INFINITY;
-#pragma unroll 1
+      float sv[128];
+      if (need0) { tmem_ld32(s_addr, sv); tmem_ld32(s_addr + 32, sv + 32); }
+      if (need1) { tmem_ld32(s_addr + 64, sv + 64); tmem_ld32(s_addr + 96, sv + 96); }
+      tmem_wait_ld();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.s_free[bb]);
+      // logits in log2 units (masked / offset) and the tile's row max
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (!(hh ? need1 : need0)) continue;
         const float* ad = hh ? add1 : add0;
-        float sv[64];
-        tmem_ld32(s_addr + 64 * hh, sv);
-        tmem_ld32(s_addr + 64 * hh + 32, sv + 32);
-        tmem_wait_ld();
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (ad) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], fmaf(sv[c], sl2, ad[c]));
+          for (int c = 0; c < 64; ++c) {
+            sv[64 * hh + c] = fmaf(sv[64 * hh + c], sl2, ad[c]);
+            m4[c & 3] = fmaxf(m4[c & 3], sv[64 * hh + c]);
+          }
         } else {
+          float r4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
-          m4[0] *= sl2; m4[1] *= sl2; m4[2] *= sl2; m4[3] *= sl2;
+          for (int c = 0; c < 64; ++c) r4[c & 3] = fmaxf(r4[c & 3], sv[64 * hh + c]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], r4[q] * sl2);
         }
-        mt = fmaxf(mt, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
       }
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (tracer) SOL_TRACE_AT(1, t);
       float alpha = 1.f;
       bool resc = false;
       if (mt > m_run + kRescale || (m_run == -INFINITY && mt != -INFINITY)) {
@@ -452,62 +494,60 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         m_run = mt;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: p = 2^(x - base) as bf16 into the S columns (P aliases S)
+      if (t >= 2) {   // P_bb's previous reader, PV(t-2)
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[bb], ((t - 2) >> 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        fence_after();
+      }
+      // p = 2^(x - base) as bf16 pairs into P_bb
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+#pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
-        const float* ad = hh ? add1 : add0;
         if (hh ? need1 : need0) {
-          float sv[64];
-          tmem_ld32(s_addr + 64 * hh, sv);
-          tmem_ld32(s_addr + 64 * hh + 32, sv + 32);
-          tmem_wait_ld();
-          if (ad) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = ex2(fmaf(sv[c], sl2, ad[c]) - base);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) sv[c] = ex2(fmaf(sv[c], sl2, -base));
-          }
+          const bool scaled = (hh ? add1 : add0) != nullptr;   // logits already in log2 units
+          const float mul = scaled ? 1.f : sl2;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            l4[c & 3] += sv[2 * c] + sv[2 * c + 1];
-            pk[c] = pack_bf16(sv[2 * c], sv[2 * c + 1]);
+            const float p0 = ex2(fmaf(sv[64 * hh + 2 * c], mul, -base));
+            const float p1 = ex2(fmaf(sv[64 * hh + 2 * c + 1], mul, -base));
+            l4[c & 3] += p0 + p1;
+            pk[c] = pack_bf16(p0, p1);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
-        tmem_st32(s_addr + 32 * hh, pk);
+        tmem_st32(lane_addr + 384 + 64 * bb + 32 * hh, pk);
       }
-      tmem_wait_st();
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      if (t >= 1) {
-        ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done, (t - 1) & 1, abort_flag, a.status));
+      if (tracer) SOL_TRACE_AT(2, t);
+      // O is rescaled only once PV(t-1), the last MMA to accumulate into it, is complete
+      if (t >= 1 && __any_sync(0xffffffffu, resc)) {
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, a.status));
         if (!ok) break;
         fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const float f = resc ? alpha : 1.f;
+        const float f = resc ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tmem_ld32(lane_addr + 256 + 32 * c, ov);
-            tmem_wait_ld();
-            uint32_t ou[32];
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(o_addr + 32 * c, ov);
+          tmem_wait_ld();
+          uint32_t ou[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(ov[e] * f);
-            tmem_st32(lane_addr + 256 + 32 * c, ou);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(ov[e] * f);
+          tmem_st32(o_addr + 32 * c, ou);
         }
       }
+      tmem_wait_st();
       fence_before();
       __syncwarp();
+      if (tracer) SOL_TRACE_AT(3, t);
       if (lane == 0) mbar_arrive(&bar.p_full[bb]);
     }
-    // epilogue: O / l -> bf16
-    if (ok && T > 0) ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done, (T - 1) & 1, abort_flag, a.status));
+    // epilogue: O / l -> bf16, once the last PV is complete
+    if (ok && T > 0)
+      ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status));
     if (ok) {
       fence_after();
       const int grow = 64 * (i0 + hf) + (r & 63);
@@ -517,7 +557,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];
-        tmem_ld32(lane_addr + 256 + 32 * c, ov);
+        tmem_ld32(o_addr + 32 * c, ov);
         tmem_wait_ld();
         if (store) {
 #pragma unroll
@@ -596,3 +636,11 @@ cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st) {
 }
 
 }  // namespace sol
+
+#ifdef SOL_TRACE
+// Copies the phase trace (16 slots x 256 steps of clock64 stamps) to host memory.
+extern "C" int sol_debug_trace(long long* host, int n) {
+  const int total = 16 * sol::kTraceSteps;
+  return (int)cudaMemcpyFromSymbol(host, sol::g_trace, sizeof(long long) * (n < total ? n : total));
+}
+#endif
