@@ -61,6 +61,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
     extra = ["-Xptxas", "-v"] if ptxas_info else []
     if trace:
         extra.append("-DSOL_TRACE")
+        if os.environ.get("SOL_TRACE_WARP"):
+            extra.append("-DSOL_TRACE_WARP=" + os.environ["SOL_TRACE_WARP"])
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + (".trace.o" if trace else ".o"))

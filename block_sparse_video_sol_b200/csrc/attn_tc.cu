@@ -17,17 +17,22 @@
 // p = 0 there (its exponentials are skipped, warp-uniformly).  Then come the
 // centroid tiles: 128 centroids each, the half's selected blocks masked.
 //
-// Roles (7 warps):
-//   warp 0     TMA producer: Q once, then the K tiles into a 3-stage ring.
-//   warp 6     TMA producer: the V tiles into a 2-stage ring.
-//   warp 1     MMA issuer (one lane): S_b = Q K^T into TMEM buffer b = t%2,
-//              then O += P V with P read from its own TMEM buffer.
-//   warps 2-5  softmax, one thread per row (TMEM lane): online max/sum in
-//              fp32 with lazy rescaling (O in TMEM is rescaled only when a
-//              row's max grows by more than 2^8), P written back to TMEM,
-//              final normalisation and bf16 store.
-// TMEM: S0 = columns [0,128), S1 = [128,256), O = [256, 256+D),
-//       P0 = [384, 448), P1 = [448, 512) (bf16 pairs).
+// Roles (12 warps):
+//   warps 0-3  softmax warpgroup 0: the even S tiles t = 0, 2, 4, ...
+//   warps 4-7  softmax warpgroup 1: the odd S tiles.  One thread per row
+//              (TMEM lane), fp32 online softmax with lazy rescaling: the
+//              groups share each row's reference max (handed from step t-1
+//              to step t through an mbarrier per warp pair) and O is
+//              rescaled only when that reference grows by more than 2^8;
+//              bf16 P is written back over S.  The groups alternate, so one
+//              group's exponentials overlap the other's TMEM traffic and
+//              waits.  The epilogue normalises O and stores bf16 rows.
+//   warp 8     TMA producer: Q once, then the K tiles into a 3-stage ring.
+//   warp 9     MMA issuer (one lane): S_(t%3) = Q K^T into TMEM, then
+//              O += P V with P read from TMEM; QK runs three tiles ahead.
+//   warp 10    TMA producer: the V tiles into a 2-stage ring.
+// TMEM: S_0, S_1, S_2 = columns [0,128), [128,256), [256,384) (P = bf16 pairs
+//       over the first 64 columns of its S), O = [384, 384+D).
 // Every mbarrier wait is bounded; on expiry the kernel raises
 // SOL_ERR_TIMEOUT, stops issuing, drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -38,18 +43,29 @@
 namespace sol {
 namespace {
 
-constexpr int kThreads = 224;
+constexpr int kThreads = 384;       // 12 warps: two softmax warpgroups + one control warpgroup
+constexpr int kKWarp = 8, kMmaWarp = 9, kVWarp = 10;   // warp 11 idles
+constexpr uint32_t kOCol = 384;     // TMEM column of O; S_0, S_1, S_2 at 0, 128, 256
+// Register split (setmaxnreg): the block launches with kRegsLaunch per
+// thread; the control warpgroup gives registers back so that the softmax
+// warpgroups can hold a whole 128-column S row.  2*128*kRegsSoftmax +
+// 128*kRegsControl must not exceed 384*kRegsLaunch.
+constexpr int kRegsLaunch = 168, kRegsSoftmax = 224, kRegsControl = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch, "register split");
 constexpr int kKStages = 3;   // K tiles in flight (needed first, by QK)
 constexpr int kVStages = 2;   // V tiles in flight (needed a softmax later, by PV)
 
-// Optional phase trace (build with -DSOL_TRACE): clock64() stamps of one CTA's
-// roles for its first kTraceSteps S tiles, read back with sol_debug_trace().
+// Optional phase trace (build with -DSOL_TRACE): 32-bit clock() stamps of one
+// CTA's roles for its first kTraceSteps S tiles, kept in shared memory (a
+// global store before a release-semantics mbarrier arrive would stall it) and
+// copied out at the end; read back with sol_debug_trace().
 #ifdef SOL_TRACE
-constexpr int kTraceSteps = 256;
-__device__ long long g_trace[16 * kTraceSteps];
+constexpr int kTraceSteps = 128;
+constexpr int kTraceSlots = 24;
+__device__ unsigned int g_trace[kTraceSlots * kTraceSteps];
+#define SOL_TRACE_ON (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
 #define SOL_TRACE_AT(slot, step) \
-  do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (step) < kTraceSteps) \
-         g_trace[(slot) * kTraceSteps + (step)] = clock64(); } while (0)
+  do { if (SOL_TRACE_ON && (step) < kTraceSteps) x.trace[(slot) * kTraceSteps + (step)] = (unsigned int)clock(); } while (0)
 #else
 #define SOL_TRACE_AT(slot, step) do { } while (0)
 #endif
@@ -71,7 +87,8 @@ struct Cfg {
 struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2], final_mma;
+  uint64_t s_full[3], p_full[3], o_done[2], final_mma;
+  uint64_t ref_full[2][4];           // [group][warp]: the group's step published its reference max
 };
 
 struct Extra {
@@ -83,8 +100,13 @@ struct Extra {
   int cent[kMaxCentTiles];           // centroid tiles to visit
   int list[kMaxKeyBlocks];           // union entries: j | needA << 16 | needB << 17
   int cent_live[kMaxCentTiles][2][2];           // [slot][half][64-column half]: any live centroid
-  float cent_add[kMaxCentTiles][2][128];        // log2-unit offset of each centroid column, -inf if masked
-  float tail_add[64];                           // 0 for valid rows of the last key block, -inf beyond N
+  alignas(16) float cent_add[kMaxCentTiles][2][128];        // log2-unit offset of each centroid column, -inf if masked
+  alignas(16) float tail_add[64];                         // 0 for valid rows of the last key block, -inf beyond N
+  float2 ml[2][128];                            // per warpgroup and row: (reference, partial sum)
+  float m_ref[128];                             // per row: reference max after the latest step (log2 units)
+#ifdef SOL_TRACE
+  unsigned int trace[kTraceSlots * kTraceSteps];
+#endif
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -101,6 +123,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
 __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
                : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
   return ok != 0;
 }
@@ -156,6 +185,23 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
   asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
                :: "r"(d), "r"(a), "l"(b), "r"(id), "r"(acc));
 }
+// Warp-wide forms: the whole (converged) warp executes them and one elected
+// lane issues, so the issuing loop's values stay warp-uniform.
+__device__ __forceinline__ void mma_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile("{ .reg .pred p, e; setp.ne.b32 p, %4, 0; elect.sync _|e, 0xffffffff;\n"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
+               :: "r"(d), "l"(a), "l"(b), "r"(id), "r"(acc));
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile("{ .reg .pred p, e; setp.ne.b32 p, %4, 0; elect.sync _|e, 0xffffffff;\n"
+               "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+               :: "r"(d), "r"(a), "l"(b), "r"(id), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile("{ .reg .pred e; elect.sync _|e, 0xffffffff;\n"
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0]; }"
+               :: "r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
@@ -192,15 +238,61 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pair arithmetic (sm_100a f32x2): halves the instruction count
+// of the softmax's elementwise work.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// O row *= f for this warp's 32 rows (rarely executed; kept out of the
+// softmax loop's instruction stream).
+template <int D>
+__device__ __noinline__ void rescale_rows(uint32_t o_addr, float f) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float ov[32];
+    tmem_ld32(o_addr + 32 * c, ov);
+    tmem_wait_ld();
+    uint32_t ou[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(ov[e] * f);
+    tmem_st32(o_addr + 32 * c, ou);
+  }
 }
 
 struct TcParams {
   AttnArgs a;
   int mask_words;
 };
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -229,21 +321,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     mbar_init(&bar.q_full, 1);
     for (int s = 0; s < kKStages; ++s) { mbar_init(&bar.k_full[s], 1); mbar_init(&bar.k_empty[s], 1); }
     for (int s = 0; s < kVStages; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar.s_full[s], 1); mbar_init(&bar.s_free[s], 4); mbar_init(&bar.p_full[s], 4);
-      mbar_init(&bar.o_done[s], 1);
-    }
+    for (int s = 0; s < 3; ++s) { mbar_init(&bar.s_full[s], 1); mbar_init(&bar.p_full[s], 4); }
+    for (int s = 0; s < 2; ++s) mbar_init(&bar.o_done[s], 1);
+    for (int g = 0; g < 2; ++g)
+      for (int s = 0; s < 4; ++s) mbar_init(&bar.ref_full[g][s], 32);
     mbar_init(&bar.final_mma, 1);
     x.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&x.tmem_base)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   for (int w = tid; w < 2 * kMaxWords; w += kThreads) (&x.sel[0][0])[w] = 0u;
   const int n_tail = a.N - 64 * (a.nkb - 1);   // valid rows of the last key block
   for (int c = tid; c < 64; c += kThreads) x.tail_add[c] = c < n_tail ? 0.f : -INFINITY;
+#ifdef SOL_TRACE
+  for (int i = tid; i < kTraceSlots * kTraceSteps; i += kThreads) x.trace[i] = 0u;
+#endif
   __syncthreads();
   for (int hf = 0; hf < 2; ++hf) {
     const int i = i0 + hf;
@@ -309,12 +404,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   const int n_ex = (x.n_union + 1) >> 1;
   const int T = n_ex + x.n_cent;
 
-  if (warp == 0 || warp == 6) {
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsControl));
+  if (warp == kKWarp || warp == kVWarp) {
     // ---------------------------------------------------------------- TMA producers
-    // warp 0: Q and the K tiles (kKStages ring); warp 6: the V tiles
-    // (kVStages ring).  Each runs ahead on its own ring.
+    // Q and the K tiles (kKStages ring) from one warp, the V tiles (kVStages
+    // ring) from another; each runs ahead on its own ring.
     if (lane == 0) {
-      const bool is_k = warp == 0;
+      const bool is_k = warp == kKWarp;
       const int nst = is_k ? kKStages : kVStages;
       const CUtensorMap* m4 = is_k ? &mk : &mv;
       const CUtensorMap* m3 = is_k ? &mkb : &mvb;
@@ -360,84 +457,138 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       }
       if (is_k) drain_bar(&bar.q_full, 0, a.status);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
-    // Issue order QK(0), QK(1), QK(2), PV(0), QK(3), PV(1), QK(4), ...: the
-    // tensor pipe runs in order and issuing blocks for about as long as the
-    // MMAs take, so the QKs run ahead and S(u+1), S(u+2) are ready before the
-    // softmax needs them.  QK(g) reuses S_(g%2) once the softmax has read
-    // S(g-2) (it releases S right after loading it).
-    if (lane == 0) {
+    // Issue order QK(0), QK(1), QK(2), PV(0), QK(3), PV(1), QK(4), ...  Step t
+    // uses S_(t%3), whose first 64 columns the softmax overwrites with P(t);
+    // every PV accumulates into the one O.  QK(t+3) follows PV(t) in the
+    // (in-order) tensor pipe, so it overwrites S_(t%3) only after PV(t) has
+    // read P(t), and the commit that signals S(t+3) also covers PV(t).
+    {   // the whole warp runs the loop; one elected lane issues each MMA / commit
+      // The tensor pipe's issue queue is short, so the steady-state loop is
+      // kept free of run-time conditions around its MMA batches (a batch
+      // under a condition costs pipe time even when skipped): the first PV
+      // (which starts O) and the last three (no QK follows) are peeled off,
+      // ring positions are counters, descriptors are precomputed (one add
+      // per MMA) and every wait sits between batches.
       constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t o_tmem = tmem + 256;
-      bool ok = wait_bar(&bar.q_full, 0, abort_flag, a.status);
-      auto qk = [&](int g) -> bool {
-        const int s = g % kKStages, n = g / kKStages, bb = g & 1;
-        if (!wait_bar(&bar.k_full[s], n & 1, abort_flag, a.status)) return false;
-        if (g >= 2 && !wait_bar(&bar.s_free[bb], ((g >> 1) - 1) & 1, abort_flag, a.status)) return false;
-        fence_after();
-        SOL_TRACE_AT(4, g);
-        const uint32_t kb = k_addr + s * C::kTileBytes;
+      constexpr int NQ = D / 16;                                   // QK MMAs (k = 16 each)
+      constexpr uint64_t kStageD = (uint64_t)(C::kTileBytes >> 4); // descriptor step per ring stage
+      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024);
+      const uint64_t kd0 = sdesc(smem_u32(sK), 16, 1024);
+      const uint64_t vd0 = sdesc(smem_u32(sV), C::kChunkBytes, 1024);
+      int kst = 0, vst = 0, sq = 0, sp = 0;        // K / V ring stages, S buffers of the next QK / PV
+      uint32_t kph = 0, vph = 0, pph = 0;          // their phase parities
+      // QK(g) into S_sq from K stage kst (K must have landed)
+      auto qk = [&]() {
+        const uint64_t kd = kd0 + (uint64_t)kst * kStageD;
+        const uint32_t d = tmem + 128 * sq;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + bb * 128, sdesc(q_addr + off, 16, 1024), sdesc(kb + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < NQ; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
+          mma_ss_w(d, qd + off, kd + off, id_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bar.s_full[bb]);
-        mma_commit(&bar.k_empty[s]);
-        return true;
+        mma_commit_w(&bar.s_full[sq]);
+        mma_commit_w(&bar.k_empty[kst]);
+        if (++kst == kKStages) { kst = 0; kph ^= 1u; }
+        sq = sq == 2 ? 0 : sq + 1;
       };
-      auto pv = [&](int u) -> bool {
-        const int s = u % kVStages, n = u / kVStages, bb = u & 1;
-        if (!wait_bar(&bar.p_full[bb], (u >> 1) & 1, abort_flag, a.status)) return false;
-        SOL_TRACE_AT(5, u);
-        if (!wait_bar(&bar.v_full[s], n & 1, abort_flag, a.status)) return false;
-        fence_after();
-        const uint32_t vb = v_addr + s * C::kTileBytes;
+      // PV(u) from P in S_sp and V stage vst into O (P and V must be ready)
+      auto pv = [&](int u, bool first) {
+        const uint64_t vd = vd0 + (uint64_t)vst * kStageD;
+        const uint32_t pa = tmem + 128 * sp;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(o_tmem, tmem + 384 + 64 * bb + kk * 8, sdesc(vb + kk * 2048, C::kChunkBytes, 1024), id_pv,
-                 (u > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.v_empty[s]);
-        mma_commit(&bar.o_done[bb]);
-        return true;
+          mma_ts_w(tmem + kOCol, pa + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), id_pv, (first && kk == 0) ? 0u : 1u);
+        mma_commit_w(&bar.v_empty[vst]);
+        mma_commit_w(&bar.o_done[u & 1]);
+        if (++vst == kVStages) { vst = 0; vph ^= 1u; }
+        if (sp == 2) { sp = 0; pph ^= 1u; } else { ++sp; }
       };
-      for (int g = 0; g < 3 && g < T && ok; ++g) ok = qk(g);
-      for (int u = 0; u < T && ok; ++u) {
-        ok = pv(u);
-        if (ok && u + 3 < T) ok = qk(u + 3);
+      // every wait's outcome is made warp-uniform, so all lanes leave the loop together
+      auto wait_k = [&]() {
+        const bool r = __all_sync(0xffffffffu, wait_bar(&bar.k_full[kst], kph, abort_flag, a.status));
+        fence_after();
+        return r;
+      };
+      auto wait_pv = [&]() {
+        const bool r = __all_sync(0xffffffffu, wait_bar(&bar.p_full[sp], pph, abort_flag, a.status) &&
+                                                   wait_bar(&bar.v_full[vst], vph, abort_flag, a.status));
+        fence_after();
+        return r;
+      };
+      bool ok = __all_sync(0xffffffffu, wait_bar(&bar.q_full, 0, abort_flag, a.status));
+      const int nq0 = T < 3 ? T : 3;
+      for (int g = 0; g < nq0 && ok; ++g) {
+        if ((ok = wait_k())) qk();
       }
-      // drain: all issued MMAs complete before TMEM is released
-      mma_commit(&bar.final_mma);
+      const int n_steady = T > 3 ? T - 3 : 0;    // PV(u) followed by QK(u+3)
+      if (ok && T > 0 && (ok = wait_pv())) {
+        SOL_TRACE_AT(5, 0);
+        pv(0, true);
+        if (n_steady > 0 && (ok = wait_k())) qk();
+      }
+      for (int u = 1; u < n_steady && ok; ++u) {
+        if (!(ok = wait_pv())) break;
+        SOL_TRACE_AT(5, u);
+        pv(u, false);
+        SOL_TRACE_AT(13, u);
+        if (!(ok = wait_k())) break;
+        SOL_TRACE_AT(4, u + 3);
+        qk();
+        SOL_TRACE_AT(11, u + 3);
+      }
+      for (int u = n_steady > 1 ? n_steady : 1; u < T && ok; ++u) {
+        if (!(ok = wait_pv())) break;
+        pv(u, false);
+      }
+      // all issued MMAs complete before the epilogue reads O and TMEM is released
+      mma_commit_w(&bar.final_mma);
       drain_bar(&bar.final_mma, 0, a.status);
     }
-  } else if (warp >= 2 && warp <= 5) {
-    // ---------------------------------------------------------------- softmax warpgroup
-    // One pass per S tile: the needed columns are read once (S is then
-    // released to the next QK), masked, maxed, exponentiated and stored as bf16
-    // P into its own TMEM buffer P_(u%2), once PV(u-2), the last reader of
-    // that buffer, is complete.  PV completions are waited for only there, for
-    // a rescale of O (PV(u-1)) and before the epilogue (PV(T-1)).  PV(v)
-    // completes o_done[v%2]; the next completion of that barrier needs P(v+2),
-    // which this warpgroup has not produced yet, so each parity wait is exact.
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsSoftmax));
+    // ---------------------------------------------------------------- softmax warpgroups
+    // Warpgroup w (warps 4w .. 4w+3) takes the steps t = w, w+2, w+4, ...,
+    // one thread per row (TMEM lane), so one group exponentiates while the
+    // other waits on TMEM.  Both feed the one accumulator O, so they share
+    // each row's reference max m (log2 units): step t reads the reference
+    // left by step t-1 (the other group), raises it only when its tile's max
+    // exceeds it by more than 2^8 (lazy rescaling), publishes it at once and
+    // then exponentiates against it.  A raise rescales O after PV(t-1), the
+    // last product taken against the old reference.  Each group keeps its
+    // partial sum l_w relative to the reference of its latest step; the
+    // epilogue brings both to the final reference.
+    const int w = warp >> 2;
     const int sub = warp & 3;                 // TMEM sub-partition = rows 32*sub .. 32*sub+31
     const int r = 32 * sub + lane;            // row of the tile
     const int hf = r >> 6;                    // query block half (warp-uniform)
     const bool present = x.present[hf] != 0;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
-    const uint32_t o_addr = lane_addr + 256;
+    const uint32_t o_addr = lane_addr + kOCol;
     const float sl2 = a.scale * kLog2e;
-    const bool tracer = warp == 2 && lane == 0;
-    float m_run = -INFINITY, l = 0.f;
+#ifndef SOL_TRACE_WARP
+#define SOL_TRACE_WARP 0
+#endif
+    const bool tracer = sub == SOL_TRACE_WARP && lane == 0;
+    (void)tracer;
+    float ref_w = -INFINITY, l = 0.f;         // this group's partial sum, relative to ref_w
     bool ok = true;
-    for (int t = 0; t < T && ok; ++t) {
-      const int bb = t & 1;
-      ok = __all_sync(0xffffffffu, wait_bar(&bar.s_full[bb], (t >> 1) & 1, abort_flag, a.status));
+    int bb = w;                               // S buffer of step t: t % 3
+    for (int t = w; t < T && ok; t += 2, bb = (bb + 2) % 3) {
+#ifdef SOL_TRACE
+      if (tracer) SOL_TRACE_AT(15, t);
+#endif
+      ok = __all_sync(0xffffffffu, wait_bar(&bar.s_full[bb], (t / 3) & 1, abort_flag, a.status));
       if (!ok) break;
       fence_after();
+#ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(0, t);
+      if (lane == 0) SOL_TRACE_AT(20 + sub, t);
+#endif
+      const uint32_t s_addr = lane_addr + 128 * bb;   // S(t); P(t) is written over its first 64 columns
       // which 64-column halves of this S tile the row uses, and their additive offsets
       bool need0, need1;
       const float *add0, *add1;
@@ -455,125 +606,142 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         add0 = x.cent_add[slot][hf];
         add1 = x.cent_add[slot][hf] + 64;
       }
-      const uint32_t s_addr = lane_addr + bb * 128;
       float sv[128];
       if (need0) { tmem_ld32(s_addr, sv); tmem_ld32(s_addr + 32, sv + 32); }
       if (need1) { tmem_ld32(s_addr + 64, sv + 64); tmem_ld32(s_addr + 96, sv + 96); }
       tmem_wait_ld();
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.s_free[bb]);
-      // logits in log2 units (masked / offset) and the tile's row max
+      // logits in log2 units (offset / masked) and the tile's row max; an
+      // ordinary block's scores are scaled inside the exponent instead
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (!(hh ? need1 : need0)) continue;
         const float* ad = hh ? add1 : add0;
+        float* v = sv + 64 * hh;
         if (ad) {
+          const uint64_t sl22 = f2pack(sl2, sl2);
+          const float4* ad4 = reinterpret_cast<const float4*>(ad);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            sv[64 * hh + c] = fmaf(sv[64 * hh + c], sl2, ad[c]);
-            m4[c & 3] = fmaxf(m4[c & 3], sv[64 * hh + c]);
+          for (int c = 0; c < 16; ++c) {
+            const float4 o = ad4[c];
+            f2unpack(ffma2(f2pack(v[4 * c], v[4 * c + 1]), sl22, f2pack(o.x, o.y)), v[4 * c], v[4 * c + 1]);
+            f2unpack(ffma2(f2pack(v[4 * c + 2], v[4 * c + 3]), sl22, f2pack(o.z, o.w)), v[4 * c + 2], v[4 * c + 3]);
+            m4[c & 3] = fmax3(m4[c & 3], v[4 * c], v[4 * c + 1]);
+            m4[(c + 2) & 3] = fmax3(m4[(c + 2) & 3], v[4 * c + 2], v[4 * c + 3]);
           }
         } else {
           float r4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) r4[c & 3] = fmaxf(r4[c & 3], sv[64 * hh + c]);
+          for (int c = 0; c < 32; ++c) r4[c & 3] = fmax3(r4[c & 3], v[2 * c], v[2 * c + 1]);
 #pragma unroll
           for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], r4[q] * sl2);
         }
       }
       const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+#ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(1, t);
-      float alpha = 1.f;
-      bool resc = false;
-      if (mt > m_run + kRescale || (m_run == -INFINITY && mt != -INFINITY)) {
-        alpha = ex2(m_run - mt);            // 0 when m_run = -inf
-        resc = l > 0.f;
-        l *= alpha;
-        m_run = mt;
-      }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      if (t >= 2) {   // P_bb's previous reader, PV(t-2)
-        ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[bb], ((t - 2) >> 1) & 1, abort_flag, a.status));
+#endif
+      // the reference after step t-1, raised if this tile exceeds it by more than 2^8
+      float m_prev = -INFINITY;
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.ref_full[w ^ 1][sub], ((t - 1) >> 1) & 1, abort_flag, a.status));
         if (!ok) break;
-        fence_after();
+        m_prev = x.m_ref[r];
       }
-      // p = 2^(x - base) as bf16 pairs into P_bb
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      float m_cur = m_prev;
+      if (mt > m_prev + kRescale || (m_prev == -INFINITY && mt != -INFINITY)) m_cur = mt;
+      x.m_ref[r] = m_cur;
+      mbar_arrive(&bar.ref_full[w][sub]);
+      const bool resc = m_cur != m_prev && m_prev != -INFINITY;   // O holds terms against m_prev
+      if (m_cur != ref_w) { l *= ex2(ref_w - m_cur); ref_w = m_cur; }   // m only grows: ex2(<= 0)
+      const float base = (m_cur == -INFINITY) ? 0.f : m_cur;
+      // p = 2^(x - base) as bf16 pairs into P(t) (over S(t)'s first 64 columns)
+      float lsum = 0.f;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
         if (hh ? need1 : need0) {
-          const bool scaled = (hh ? add1 : add0) != nullptr;   // logits already in log2 units
-          const float mul = scaled ? 1.f : sl2;
+          const float mul = (hh ? add1 : add0) != nullptr ? 1.f : sl2;   // offset logits are in log2 units
+          const uint64_t mul2 = f2pack(mul, mul), nb2 = f2pack(-base, -base);
+          uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(fmaf(sv[64 * hh + 2 * c], mul, -base));
-            const float p1 = ex2(fmaf(sv[64 * hh + 2 * c + 1], mul, -base));
-            l4[c & 3] += p0 + p1;
+            float x0, x1;
+            f2unpack(ffma2(f2pack(sv[64 * hh + 2 * c], sv[64 * hh + 2 * c + 1]), mul2, nb2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc2[c & 1] = fadd2(acc2[c & 1], f2pack(p0, p1));
             pk[c] = pack_bf16(p0, p1);
           }
+          float a0, a1, a2, a3;
+          f2unpack(acc2[0], a0, a1);
+          f2unpack(acc2[1], a2, a3);
+          lsum += (a0 + a1) + (a2 + a3);
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
-        tmem_st32(lane_addr + 384 + 64 * bb + 32 * hh, pk);
+        tmem_st32(s_addr + 32 * hh, pk);
       }
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      l += lsum;
+#ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(2, t);
-      // O is rescaled only once PV(t-1), the last MMA to accumulate into it, is complete
-      if (t >= 1 && __any_sync(0xffffffffu, resc)) {
-        ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, a.status));
+#endif
+      if (__any_sync(0xffffffffu, resc)) {
+        // O = sum of PV(0..t-1) against m_prev once PV(t-1) is complete
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(&bar.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, a.status));
         if (!ok) break;
         fence_after();
-        const float f = resc ? alpha : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tmem_ld32(o_addr + 32 * c, ov);
-          tmem_wait_ld();
-          uint32_t ou[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ou[e] = __float_as_uint(ov[e] * f);
-          tmem_st32(o_addr + 32 * c, ou);
-        }
+        rescale_rows<D>(o_addr, resc ? ex2(m_prev - m_cur) : 1.f);
       }
       tmem_wait_st();
       fence_before();
       __syncwarp();
+#ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(3, t);
+      if (lane == 0) SOL_TRACE_AT(16 + sub, t);
+#endif
       if (lane == 0) mbar_arrive(&bar.p_full[bb]);
     }
-    // epilogue: O / l -> bf16, once the last PV is complete
-    if (ok && T > 0)
-      ok = __all_sync(0xffffffffu, wait_bar(&bar.o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status));
-    if (ok) {
+    // epilogue: with M the final reference, O / (l_0 2^(ref_0 - M) + l_1 2^(ref_1 - M));
+    // warpgroup w writes the columns [w D/2, (w+1) D/2)
+    x.ml[w][r] = make_float2(ref_w, l);
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bar.final_mma, 0, abort_flag, a.status));
+    named_bar_sync(1, 256);
+    if (ok && !*abort_flag && T > 0) {
       fence_after();
+      const float M = x.m_ref[r];            // written by step T-1
+      const float2 p0 = x.ml[0][r], p1 = x.ml[1][r];
+      const float L = (p0.x == -INFINITY ? 0.f : p0.y * ex2(p0.x - M)) + (p1.x == -INFINITY ? 0.f : p1.y * ex2(p1.x - M));
+      const float inv = L > 0.f ? 1.f / L : 0.f;
       const int grow = 64 * (i0 + hf) + (r & 63);
       const bool store = present && grow < a.N;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = a.o + (int64_t)b * a.ob + (int64_t)h * a.oh + (int64_t)grow * a.on;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = w * (D / 2) + 32 * c;
         float ov[32];
-        tmem_ld32(o_addr + 32 * c, ov);
+        tmem_ld32(o_addr + col, ov);
         tmem_wait_ld();
         if (store) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
-            uint4 u4 = make_uint4(pack_bf16(ov[e] * inv, ov[e + 1] * inv), pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv),
-                                  pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv), pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv));
-            *reinterpret_cast<uint4*>(orow + 32 * c + e) = u4;
+            const uint4 u4 = make_uint4(pack_bf16(ov[e] * inv, ov[e + 1] * inv), pack_bf16(ov[e + 2] * inv, ov[e + 3] * inv),
+                                        pack_bf16(ov[e + 4] * inv, ov[e + 5] * inv), pack_bf16(ov[e + 6] * inv, ov[e + 7] * inv));
+            *reinterpret_cast<uint4*>(orow + col + e) = u4;
           }
         }
       }
-      if (store && a.lse) a.lse[bh * a.N + grow] = (m_run + log2f(l)) * kLn2;
+      if (w == 0 && store && a.lse) a.lse[bh * a.N + grow] = (M + log2f(L)) * kLn2;
     }
   }
   fence_before();
   __syncthreads();
-  if (warp == 1) {
+#ifdef SOL_TRACE
+  if (SOL_TRACE_ON)
+    for (int i = tid; i < kTraceSlots * kTraceSteps; i += kThreads) g_trace[i] = x.trace[i];
+#endif
+  if (warp == kMmaWarp) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(512));
   }
@@ -624,6 +792,12 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   const size_t smem = 1024 + Cfg<D>::kSmemTiles + sizeof(Extra);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // The setmaxnreg split is sized for exactly kRegsLaunch registers per
+  // thread at launch; with any other count the softmax warpgroups' increase
+  // could not be granted, so refuse to launch.
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>)) != cudaSuccess) return e;
+  if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   dim3 grid((a.nqb + 1) / 2, a.H, a.B);
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkb, mvb, prm);
   return cudaGetLastError();
@@ -638,9 +812,9 @@ cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st) {
 }  // namespace sol
 
 #ifdef SOL_TRACE
-// Copies the phase trace (16 slots x 256 steps of clock64 stamps) to host memory.
-extern "C" int sol_debug_trace(long long* host, int n) {
-  const int total = 16 * sol::kTraceSteps;
-  return (int)cudaMemcpyFromSymbol(host, sol::g_trace, sizeof(long long) * (n < total ? n : total));
+// Copies the phase trace (16 slots x 128 steps of 32-bit clock stamps) to host memory.
+extern "C" int sol_debug_trace(unsigned int* host, int n) {
+  const int total = sol::kTraceSlots * sol::kTraceSteps;
+  return (int)cudaMemcpyFromSymbol(host, sol::g_trace, sizeof(unsigned int) * (n < total ? n : total));
 }
 #endif
