@@ -18,8 +18,13 @@
 // centroid tiles: 128 centroids each, the half's selected blocks masked.
 //
 // Roles (12 warps):
-//   warps 0-3  softmax warpgroup 0: the even S tiles t = 0, 2, 4, ...
-//   warps 4-7  softmax warpgroup 1: the odd S tiles.  One thread per row
+//   warp 0     TMA producer: Q once, then the K tiles into a 3-stage ring.
+//   warp 1     MMA issuer (the whole warp; one elected lane issues):
+//              S_(t%3) = Q K^T into TMEM, then O += P V with P read from
+//              TMEM; QK runs three tiles ahead.
+//   warp 2     TMA producer: the V tiles into a 2-stage ring.
+//   warps 4-7  softmax warpgroup 0: the even S tiles t = 0, 2, 4, ...
+//   warps 8-11 softmax warpgroup 1: the odd S tiles.  One thread per row
 //              (TMEM lane), fp32 online softmax with lazy rescaling: the
 //              groups share each row's reference max (handed from step t-1
 //              to step t through an mbarrier per warp pair) and O is
@@ -27,10 +32,6 @@
 //              bf16 P is written back over S.  The groups alternate, so one
 //              group's exponentials overlap the other's TMEM traffic and
 //              waits.  The epilogue normalises O and stores bf16 rows.
-//   warp 8     TMA producer: Q once, then the K tiles into a 3-stage ring.
-//   warp 9     MMA issuer (one lane): S_(t%3) = Q K^T into TMEM, then
-//              O += P V with P read from TMEM; QK runs three tiles ahead.
-//   warp 10    TMA producer: the V tiles into a 2-stage ring.
 // TMEM: S_0, S_1, S_2 = columns [0,128), [128,256), [256,384) (P = bf16 pairs
 //       over the first 64 columns of its S), O = [384, 384+D).
 // Every mbarrier wait is bounded; on expiry the kernel raises
@@ -44,7 +45,7 @@ namespace sol {
 namespace {
 
 constexpr int kThreads = 384;       // 12 warps: two softmax warpgroups + one control warpgroup
-constexpr int kKWarp = 8, kMmaWarp = 9, kVWarp = 10;   // warp 11 idles
+constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2;   // warp 3 idles; warps 4-11 softmax
 constexpr uint32_t kOCol = 384;     // TMEM column of O; S_0, S_1, S_2 at 0, 128, 256
 // Register split (setmaxnreg): the block launches with kRegsLaunch per
 // thread; the control warpgroup gives registers back so that the softmax
@@ -54,6 +55,9 @@ constexpr int kRegsLaunch = 168, kRegsSoftmax = 224, kRegsControl = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch, "register split");
 constexpr int kKStages = 3;   // K tiles in flight (needed first, by QK)
 constexpr int kVStages = 2;   // V tiles in flight (needed a softmax later, by PV)
+// A K stage is released by the commit that signals its S buffer and a V stage
+// by the commit that signals its PV, so the rings match those buffers.
+static_assert(kKStages == 3 && kVStages == 2, "K ring = S buffers, V ring = o_done barriers");
 
 // Optional phase trace (build with -DSOL_TRACE): 32-bit clock() stamps of one
 // CTA's roles for its first kTraceSteps S tiles, kept in shared memory (a
@@ -86,7 +90,7 @@ struct Cfg {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t k_full[kKStages], v_full[kVStages];
   uint64_t s_full[3], p_full[3], o_done[2], final_mma;
   uint64_t ref_full[2][4];           // [group][warp]: the group's step published its reference max
 };
@@ -319,8 +323,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   // ---- set-up: barriers, TMEM, routing lists --------------------------------------------------
   if (tid == 0) {
     mbar_init(&bar.q_full, 1);
-    for (int s = 0; s < kKStages; ++s) { mbar_init(&bar.k_full[s], 1); mbar_init(&bar.k_empty[s], 1); }
-    for (int s = 0; s < kVStages; ++s) { mbar_init(&bar.v_full[s], 1); mbar_init(&bar.v_empty[s], 1); }
+    for (int s = 0; s < kKStages; ++s) mbar_init(&bar.k_full[s], 1);
+    for (int s = 0; s < kVStages; ++s) mbar_init(&bar.v_full[s], 1);
     for (int s = 0; s < 3; ++s) { mbar_init(&bar.s_full[s], 1); mbar_init(&bar.p_full[s], 4); }
     for (int s = 0; s < 2; ++s) mbar_init(&bar.o_done[s], 1);
     for (int g = 0; g < 2; ++g)
@@ -353,18 +357,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   }
   __syncthreads();
   if (warp == 0) {
-    // union list with per-half tags, ascending
-    uint32_t ua = lane < mw ? x.sel[0][lane] : 0u, ub = lane < mw ? x.sel[1][lane] : 0u, u = ua | ub;
-    int cnt = __popc(u), incl = cnt;
+    // Union list with per-half tags.  The S tiles take consecutive pairs of
+    // entries, and a half's exponentials are skipped for a block it does not
+    // need, so the order balances the two halves' warps: first pairs (block
+    // only A needs, block only B needs), then the blocks both need, then the
+    // leftover single-half blocks.  (The online softmax is order-free.)
+    const uint32_t ua = lane < mw ? x.sel[0][lane] : 0u, ub = lane < mw ? x.sel[1][lane] : 0u;
+    const uint32_t oa = ua & ~ub, ob = ub & ~ua, oc = ua & ub;
+    const int ca = __popc(oa), cb = __popc(ob), cc = __popc(oc);
+    int ia = ca, ib = cb, ic = cc;   // inclusive scans over the lanes' words
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) { const int y = __shfl_up_sync(0xffffffffu, incl, o); if (lane >= o) incl += y; }
-    int pos = incl - cnt;
-    while (u) {
-      const int bit = __ffs(u) - 1;
-      u &= u - 1;
-      x.list[pos++] = (32 * lane + bit) | (int)(((ua >> bit) & 1u) << 16) | (int)(((ub >> bit) & 1u) << 17);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o),
+                yc = __shfl_up_sync(0xffffffffu, ic, o);
+      if (lane >= o) { ia += ya; ib += yb; ic += yc; }
     }
-    if (lane == 31) x.n_union = incl;
+    const int NA = __shfl_sync(0xffffffffu, ia, 31), NB = __shfl_sync(0xffffffffu, ib, 31),
+              NC = __shfl_sync(0xffffffffu, ic, 31);
+    const int npair = min(NA, NB), rest = 2 * npair + NC;   // leftovers of one kind start at rest
+    int ra = ia - ca, rb = ib - cb, rc = ic - cc;
+    for (uint32_t m = oa; m; m &= m - 1, ++ra)
+      x.list[ra < npair ? 2 * ra : rest + ra - npair] = (32 * lane + __ffs(m) - 1) | (1 << 16);
+    for (uint32_t m = ob; m; m &= m - 1, ++rb)
+      x.list[rb < npair ? 2 * rb + 1 : rest + rb - npair] = (32 * lane + __ffs(m) - 1) | (1 << 17);
+    for (uint32_t m = oc; m; m &= m - 1, ++rc)
+      x.list[2 * npair + rc] = (32 * lane + __ffs(m) - 1) | (3 << 16);
+    if (lane == 0) x.n_union = NA + NB + NC;
     // centroid tiles holding at least one block unselected by a present half
     if (lane == 0) {
       x.present[0] = 1;
@@ -404,7 +422,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   const int n_ex = (x.n_union + 1) >> 1;
   const int T = n_ex + x.n_cent;
 
-  if (warp >= 8) {
+  if (warp < 4) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsControl));
   if (warp == kKWarp || warp == kVWarp) {
     // ---------------------------------------------------------------- TMA producers
@@ -434,7 +452,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         } else {
           ct = x.cent[t - n_ex];
         }
-        uint64_t* empty = is_k ? &bar.k_empty[s] : &bar.v_empty[s];
+        // K stage t%3 is free once QK(t-3) is complete (the completion of
+        // s_full[t%3] before the one for S(t)); V stage t%2 once PV(t-2) is
+        // (o_done[t%2]): the same commits that signal the consumers.
+        uint64_t* empty = is_k ? &bar.s_full[s] : &bar.o_done[s];
         uint64_t* full = is_k ? &bar.k_full[s] : &bar.v_full[s];
         if (!(ok = wait_bar(empty, (n & 1) ^ 1, abort_flag, a.status))) break;
         SOL_TRACE_AT(is_k ? 7 : 8, t);
@@ -489,8 +510,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
           const uint64_t off = (uint64_t)(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
           mma_ss_w(d, qd + off, kd + off, id_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit_w(&bar.s_full[sq]);
-        mma_commit_w(&bar.k_empty[kst]);
+        mma_commit_w(&bar.s_full[sq]);   // also frees K stage kst (== sq)
         if (++kst == kKStages) { kst = 0; kph ^= 1u; }
         sq = sq == 2 ? 0 : sq + 1;
       };
@@ -501,16 +521,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(tmem + kOCol, pa + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), id_pv, (first && kk == 0) ? 0u : 1u);
-        mma_commit_w(&bar.v_empty[vst]);
-        mma_commit_w(&bar.o_done[u & 1]);
+        mma_commit_w(&bar.o_done[u & 1]);   // also frees V stage vst (== u % 2)
         if (++vst == kVStages) { vst = 0; vph ^= 1u; }
         if (sp == 2) { sp = 0; pph ^= 1u; } else { ++sp; }
       };
       // every wait's outcome is made warp-uniform, so all lanes leave the loop together
-      auto wait_k = [&]() {
-        const bool r = __all_sync(0xffffffffu, wait_bar(&bar.k_full[kst], kph, abort_flag, a.status));
-        fence_after();
-        return r;
+      auto wait_k = [&]() {   // TMA data: the mbarrier completion orders it, no tcgen05 fence needed
+        return __all_sync(0xffffffffu, wait_bar(&bar.k_full[kst], kph, abort_flag, a.status));
       };
       auto wait_pv = [&]() {
         const bool r = __all_sync(0xffffffffu, wait_bar(&bar.p_full[sp], pph, abort_flag, a.status) &&
@@ -551,7 +568,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsSoftmax));
     // ---------------------------------------------------------------- softmax warpgroups
-    // Warpgroup w (warps 4w .. 4w+3) takes the steps t = w, w+2, w+4, ...,
+    // Warpgroup w (warps 4w+4 .. 4w+7) takes the steps t = w, w+2, w+4, ...,
     // one thread per row (TMEM lane), so one group exponentiates while the
     // other waits on TMEM.  Both feed the one accumulator O, so they share
     // each row's reference max m (log2 units): step t reads the reference
@@ -561,7 +578,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     // last product taken against the old reference.  Each group keeps its
     // partial sum l_w relative to the reference of its latest step; the
     // epilogue brings both to the final reference.
-    const int w = warp >> 2;
+    const int w = (warp >> 2) - 1;            // softmax warpgroup 0 or 1
     const int sub = warp & 3;                 // TMEM sub-partition = rows 32*sub .. 32*sub+31
     const int r = 32 * sub + lane;            // row of the tile
     const int hf = r >> 6;                    // query block half (warp-uniform)
@@ -648,6 +665,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (!ok) break;
         m_prev = x.m_ref[r];
       }
+#ifdef SOL_TRACE
+      if (tracer) SOL_TRACE_AT(6, t);
+#endif
       float m_cur = m_prev;
       if (mt > m_prev + kRescale || (m_prev == -INFINITY && mt != -INFINITY)) m_cur = mt;
       x.m_ref[r] = m_cur;
