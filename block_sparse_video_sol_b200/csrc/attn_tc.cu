@@ -67,7 +67,20 @@ static_assert(kKStages == 3 && kVStages == 2, "K ring = S buffers, V ring = o_do
 constexpr int kTraceSteps = 128;
 constexpr int kTraceSlots = 24;
 __device__ unsigned int g_trace[kTraceSlots * kTraceSteps];
-#define SOL_TRACE_ON (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+#ifndef SOL_TRACE_BX
+#define SOL_TRACE_BX 0
+#endif
+#ifndef SOL_TRACE_BY
+#define SOL_TRACE_BY 0
+#endif
+#define SOL_TRACE_ON (blockIdx.x == SOL_TRACE_BX && blockIdx.y == SOL_TRACE_BY && blockIdx.z == 0)
+__device__ __forceinline__ unsigned int sol_gtime() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return (unsigned int)t;
+}
+// globaltimer (ns) stamps of CTA-level events in slot 9, steps 8.. (comparable across warps)
+#define SOL_GT_AT(k) do { if (SOL_TRACE_ON) x.trace[9 * kTraceSteps + 8 + (k)] = sol_gtime(); } while (0)
 #define SOL_TRACE_AT(slot, step) \
   do { if (SOL_TRACE_ON && (step) < kTraceSteps) x.trace[(slot) * kTraceSteps + (step)] = (unsigned int)clock(); } while (0)
 #else
@@ -108,6 +121,7 @@ struct Extra {
   alignas(16) float tail_add[64];                         // 0 for valid rows of the last key block, -inf beyond N
   float2 ml[2][128];                            // per warpgroup and row: (reference, partial sum)
   float m_ref[128];                             // per row: reference max after the latest step (log2 units)
+  float cbias[kMaxKeyBlocks];                   // this (b, h)'s centroid logit biases, prefetched
 #ifdef SOL_TRACE
   unsigned int trace[kTraceSlots * kTraceSteps];
 #endif
@@ -294,8 +308,17 @@ struct TcParams {
   int mask_words;
 };
 
+// bar.sync is an aligned barrier: every warp must reach it converged, so the
+// lanes of warps that ran lane-0-only work (TMA producers, set-up) are
+// re-converged first.  Without it a warp whose lanes arrive apart can let the
+// barrier complete early.
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cta_sync() {
+  __syncwarp();
+  __syncthreads();
 }
 
 template <int D>
@@ -315,6 +338,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   volatile int* abort_flag = &x.abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#ifdef SOL_TRACE
+  const unsigned int t_entry = (unsigned int)clock(), g_entry = sol_gtime();
+#endif
   const int tq = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = (int64_t)b * a.H + h;
   const int i0 = 2 * tq;
@@ -332,6 +358,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     mbar_init(&bar.final_mma, 1);
     x.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // Q does not depend on the routing: its load starts at once
+    mbar_expect_tx(&bar.q_full, C::kTileBytes);
+    for (int hf = 0; hf < 2; ++hf)
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_4d(sQ + c * C::kChunkBytes + hf * (C::kChunkBytes / 2), &mq, c * 64, h, 64 * (i0 + hf), b, &bar.q_full);
   }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&x.tmem_base)), "r"(512));
@@ -340,10 +371,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   for (int w = tid; w < 2 * kMaxWords; w += kThreads) (&x.sel[0][0])[w] = 0u;
   const int n_tail = a.N - 64 * (a.nkb - 1);   // valid rows of the last key block
   for (int c = tid; c < 64; c += kThreads) x.tail_add[c] = c < n_tail ? 0.f : -INFINITY;
+  // this (b, h)'s centroid biases, needed once the lists are built: loaded now to overlap the CSR reads
+  for (int j = tid; j < a.nkb; j += kThreads) x.cbias[j] = a.cbias[bh * a.nkb + j];
 #ifdef SOL_TRACE
   for (int i = tid; i < kTraceSlots * kTraceSteps; i += kThreads) x.trace[i] = 0u;
 #endif
-  __syncthreads();
+  cta_sync();
+#ifdef SOL_TRACE
+  if (tid == 0) SOL_GT_AT(8);
+#endif
   for (int hf = 0; hf < 2; ++hf) {
     const int i = i0 + hf;
     if (i >= a.nqb) continue;
@@ -355,7 +391,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       else raise_status(a.status, SOL_ERR_INVALID_ARG);
     }
   }
-  __syncthreads();
+  cta_sync();
+#ifdef SOL_TRACE
+  if (tid == 0) SOL_GT_AT(9);
+#endif
   if (warp == 0) {
     // Union list with per-half tags.  The S tiles take consecutive pairs of
     // entries, and a half's exponentials are skipped for a block it does not
@@ -383,42 +422,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     for (uint32_t m = oc; m; m &= m - 1, ++rc)
       x.list[2 * npair + rc] = (32 * lane + __ffs(m) - 1) | (3 << 16);
     if (lane == 0) x.n_union = NA + NB + NC;
-    // centroid tiles holding at least one block unselected by a present half
+    // centroid tiles (128 blocks = 4 bitmap words) holding at least one
+    // block unselected by a present half: lane w checks word w
+    const bool present1 = i0 + 1 < a.nqb;
+    const uint32_t vm = lane < mw ? (a.nkb - 32 * lane >= 32 ? 0xffffffffu : ((1u << (a.nkb - 32 * lane)) - 1u)) : 0u;
+    const uint32_t wb = __ballot_sync(0xffffffffu, ((~ua & vm) != 0u) || (present1 && (~ub & vm) != 0u));
     if (lane == 0) {
       x.present[0] = 1;
-      x.present[1] = (i0 + 1 < a.nqb) ? 1 : 0;
+      x.present[1] = present1 ? 1 : 0;
       int n = 0;
-      for (int ct = 0; ct * 128 < a.nkb; ++ct) {
-        bool any = false;
-        for (int w = 4 * ct; w < min(4 * ct + 4, mw); ++w) {
-          const int valid = min(32, a.nkb - 32 * w);
-          const uint32_t vm = valid >= 32 ? 0xffffffffu : ((1u << valid) - 1u);
-          any |= ((~x.sel[0][w]) & vm) != 0u;
-          if (x.present[1]) any |= ((~x.sel[1][w]) & vm) != 0u;
-        }
-        if (any) x.cent[n++] = ct;
-      }
+      for (int ct = 0; ct < 8; ++ct)
+        if ((wb >> (4 * ct)) & 0xFu) x.cent[n++] = ct;
       x.n_cent = n;
     }
   }
-  __syncthreads();
-  for (int idx = tid; idx < x.n_cent * 256; idx += kThreads) {
-    const int slot = idx >> 8, hf = (idx >> 7) & 1, c = idx & 127;
-    const int j = 128 * x.cent[slot] + c;
-    const bool live = x.present[hf] && j < a.nkb && !((x.sel[hf][j >> 5] >> (j & 31)) & 1u);
-    x.cent_add[slot][hf][c] = live ? a.cbias[bh * a.nkb + j] * kLog2e : -INFINITY;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < x.n_cent * 4; idx += kThreads) {
-    const int slot = idx >> 2, hf = (idx >> 1) & 1, hh = idx & 1;
-    int any = 0;
-    for (int c = 0; c < 64; ++c) any |= x.cent_add[slot][hf][64 * hh + c] != -INFINITY;
-    x.cent_live[slot][hf][hh] = any;
+  cta_sync();
+#ifdef SOL_TRACE
+  if (tid == 0) SOL_GT_AT(10);
+#endif
+  // Centroid offsets (log2 units; -inf where the half took the block exactly
+  // or past the last block) and, per 64-column half, whether any is live:
+  // warp w takes the (tile, query half) pairs w, w + 12, ...
+  for (int pr = warp; pr < 2 * x.n_cent; pr += kThreads / 32) {
+    const int slot = pr >> 1, hf = pr & 1;
+    bool l0 = false, l1 = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = lane + 32 * q, j = 128 * x.cent[slot] + c;
+      const bool live = x.present[hf] && j < a.nkb && !((x.sel[hf][j >> 5] >> (j & 31)) & 1u);
+      x.cent_add[slot][hf][c] = live ? x.cbias[j] * kLog2e : -INFINITY;
+      if (q < 2) l0 |= live; else l1 |= live;
+    }
+    const bool any0 = __any_sync(0xffffffffu, l0), any1 = __any_sync(0xffffffffu, l1);
+    if (lane == 0) { x.cent_live[slot][hf][0] = any0; x.cent_live[slot][hf][1] = any1; }
   }
   fence_before();
-  __syncthreads();
+  cta_sync();
   fence_after();
   const uint32_t tmem = x.tmem_base;
+#ifdef SOL_TRACE
+  if (tid == 0 && SOL_TRACE_ON) { x.trace[9 * kTraceSteps] = t_entry; x.trace[9 * kTraceSteps + 8] = g_entry; SOL_TRACE_AT(10, 0); SOL_GT_AT(1); }
+#endif
   const int n_ex = (x.n_union + 1) >> 1;
   const int T = n_ex + x.n_cent;
 
@@ -436,13 +480,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       uint8_t* ring = is_k ? sK : sV;
       int nl = 0;   // tile loads issued
       bool ok = true;
-      if (is_k) {
-        mbar_expect_tx(&bar.q_full, C::kTileBytes);
-        for (int hf = 0; hf < 2; ++hf)
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(sQ + c * C::kChunkBytes + hf * (C::kChunkBytes / 2), &mq, c * 64, h, 64 * (i0 + hf), b,
-                        &bar.q_full);
-      }
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % nst, n = t / nst;
         int j0 = 0, j1 = 0, ct = -1;
@@ -725,6 +762,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     }
     // epilogue: with M the final reference, O / (l_0 2^(ref_0 - M) + l_1 2^(ref_1 - M));
     // warpgroup w writes the columns [w D/2, (w+1) D/2)
+#ifdef SOL_TRACE
+    if (tracer) { SOL_TRACE_AT(12, w); SOL_GT_AT(2 + w); }
+#endif
     x.ml[w][r] = make_float2(ref_w, l);
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bar.final_mma, 0, abort_flag, a.status));
     named_bar_sync(1, 256);
@@ -755,9 +795,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       if (w == 0 && store && a.lse) a.lse[bh * a.N + grow] = (M + log2f(L)) * kLn2;
     }
   }
-  fence_before();
-  __syncthreads();
 #ifdef SOL_TRACE
+  if (warp >= 4 && (warp & 3) == SOL_TRACE_WARP && lane == 0) { SOL_TRACE_AT(14, (warp >> 2) - 1); SOL_GT_AT(4 + (warp >> 2) - 1); }
+#endif
+  fence_before();
+  cta_sync();
+#ifdef SOL_TRACE
+  if (tid == 0) { SOL_TRACE_AT(9, 1); SOL_GT_AT(6); }
+  if (warp == kMmaWarp && lane == 0) SOL_GT_AT(7);
+  cta_sync();
   if (SOL_TRACE_ON)
     for (int i = tid; i < kTraceSlots * kTraceSteps; i += kThreads) g_trace[i] = x.trace[i];
 #endif
@@ -832,7 +878,7 @@ cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st) {
 }  // namespace sol
 
 #ifdef SOL_TRACE
-// Copies the phase trace (16 slots x 128 steps of 32-bit clock stamps) to host memory.
+// Copies the phase trace (24 slots x 128 steps of 32-bit clock stamps) to host memory.
 extern "C" int sol_debug_trace(unsigned int* host, int n) {
   const int total = sol::kTraceSlots * sol::kTraceSteps;
   return (int)cudaMemcpyFromSymbol(host, sol::g_trace, sizeof(unsigned int) * (n < total ? n : total));

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
     for (int d0 = 0; d0 < D; d0 += kRouteDS) {
+      __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
       __syncthreads();
       for (int idx = tid; idx < kRouteCH * (kRouteDS / 4); idx += 256) {
         const int jj = idx / (kRouteDS / 4), dq = (idx % (kRouteDS / 4)) * 4;
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
         kT[(dq + 2) * kRouteLdK + jj] = v.z;
         kT[(dq + 3) * kRouteLdK + jj] = v.w;
       }
+      __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
       __syncthreads();
 #pragma unroll 4
       for (int dd = 0; dd < kRouteDS; ++dd) {
@@ -88,6 +90,7 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
         if (col < a.nkb) S[(8 * rg + r) * ldS + col] = a.scale * acc[r][c];
       }
   }
+  __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
   __syncthreads();
 
   // Row statistics and mask: warp w handles rows 4w .. 4w+3.
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int r
     if (lane >= o) incl += y;
   }
   if (lane == 31) warp_tot[warp] = incl;
+  __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
   __syncthreads();
   if (warp == 0) {
     int t = warp_tot[lane], ti = t;
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int r
     }
     warp_tot[lane] = ti - t;  // exclusive warp offsets
   }
+  __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
   __syncthreads();
   int run = warp_tot[warp] + incl - s;
   for (int r = lo; r < hi; ++r) { row_ptr[r] = run; run += counts[r]; }
