@@ -321,7 +321,7 @@ def run_ours(args, w):
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:
-            heads = list(range(min(args.ref_heads or 4, w.H)))
+            heads = list(range(min(args.ref_heads or 6, w.H)))
             dt, swork = oracle_sample(w, heads)
             line["cpu_baseline"] = {"value": 4 * w.D * swork / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(),
                                     "kind": "oracle",
@@ -342,7 +342,7 @@ def main():
     ap.add_argument("--log-mass-bias", action="store_true")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
-                    help="heads per oracle sample (default: 1 for --impl reference steps, 4 for cpu_baseline)")
+                    help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
