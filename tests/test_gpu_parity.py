@@ -47,6 +47,19 @@ def test_h56_n4096_full():
     assert 0.05 < dens < 0.3
 
 
+@pytest.mark.parametrize("tau", [0.5, 2.0])
+@pytest.mark.parametrize("lmb", [False, True])
+def test_tau_sweep_n8192(tau, lmb):
+    # the density sweep of the length-sweep workload: tau sets how many blocks
+    # each query block takes exactly, hence the mix of blocks one or both of a
+    # tile's two query blocks need (the order the kernel walks them in)
+    w = synth.h56_sweep(8192, tau=tau, log_mass_bias=lmb)
+    r = parity.full_check(w, heads=[0, 23, 55])
+    nb = 8192 // 64
+    dens = r["nnz"] / (56 * nb * nb)
+    assert (0.2 < dens < 0.5) if tau == 0.5 else (0.005 < dens < 0.1)
+
+
 def test_all_exact_matches_dense_sdpa():
     w = synth.Workload("dense", B=1, H=2, N=700, D=128, grid=(7, 10, 10), n_topics=4, tau=-math.inf, seed=9)
     q, k, v = synth.generate(w)
