@@ -31,8 +31,12 @@ def _dot(x, y):
     return s
 
 
-def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False):
-    """Return (O[b][n][h][d], sel[b][h][i][j]) computed row by row."""
+def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=False):
+    """Return (O[b][n][h][d], sel[b][h][i][j]) computed row by row.
+
+    ``rw`` replaces the centroid key/value of every block by the anchor-softmax
+    weighted summaries (and implies the log-mass bias, taken against them).
+    """
     s = scale if scale else 1.0 / math.sqrt(D)
     nqb = (N + bq - 1) // bq
     nkb = (N + bk - 1) // bk
@@ -50,14 +54,24 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False):
             alo = prefix if prefix < N else 0
             a = _mean_rows(Q, b, h, alo, N, D)
             bias = []
+            kc, vc = list(kbar), list(vbar)        # centroid key/value seen by queries
             for j, (lo, hi) in enumerate(kspan):
-                if not lmb:
+                if not (lmb or rw):
                     bias.append(0.0)
                     continue
                 total = 0.0
+                wk, wv = [0.0] * D, [0.0] * D
                 for t in range(lo, hi):
-                    total += math.exp(s * _dot(a, [float(x) for x in K[b][t][h]]))
-                bias.append(math.log(total / (hi - lo)) - s * _dot(a, kbar[j]))
+                    kt = [float(x) for x in K[b][t][h]]
+                    e = math.exp(s * _dot(a, kt))
+                    total += e
+                    for c in range(D):
+                        wk[c] += e * kt[c]
+                        wv[c] += e * float(V[b][t][h][c])
+                if rw:
+                    kc[j] = [x / total for x in wk]
+                    vc[j] = [x / total for x in wv]
+                bias.append(math.log(total / (hi - lo)) - s * _dot(a, kc[j]))
             sel_bh = []
             for i, (qlo, qhi) in enumerate(qspan):
                 qbar = _mean_rows(Q, b, h, qlo, qhi, D)
@@ -78,8 +92,8 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False):
                                 logits.append(s * _dot(q, [float(x) for x in K[b][t][h]]))
                                 vals.append([float(x) for x in V[b][t][h]])
                         else:
-                            logits.append(s * _dot(q, kbar[j]) + math.log(hi - lo) + bias[j])
-                            vals.append(vbar[j])
+                            logits.append(s * _dot(q, kc[j]) + math.log(hi - lo) + bias[j])
+                            vals.append(vc[j])
                     m = max(logits)
                     w = [math.exp(x - m) for x in logits]
                     z = sum(w)

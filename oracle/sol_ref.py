@@ -31,6 +31,15 @@ What it computes, step by step, in the order the sources describe it:
                  against one anchor per head, the mean video query (Spark-H3
                  news page, Spark-Reweight bullet and the compressed-branch
                  figure caption).
+  6. weighted summaries (optional, implies 5) -- the compressed branch's
+                 mean-pooled key/value summaries are replaced by weighted ones
+                 (same bullet).  Reading: within key block j the weights are
+                 the anchor's own softmax over the block's rows,
+                 w_t = exp(s*a.k_t) / sum_u exp(s*a.k_u); the summaries are
+                 sum_t w_t k_t and sum_t w_t v_t, and the bias is taken
+                 against the weighted key.  A query equal to the anchor then
+                 gets the block's exact contribution, mass and value alike.
+                 Routing still scores the mean-pooled kbar.
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -143,6 +152,36 @@ def log_mass_bias(Q: np.ndarray, K: np.ndarray, kbar: np.ndarray, prefix: int,
     return bias
 
 
+def reweighted_summaries(Q: np.ndarray, K: np.ndarray, V: np.ndarray, prefix: int,
+                         scale: float, bk: int):
+    """Anchor-weighted key/value summaries and their log-mass bias (step 6).
+
+    Per (b, h) and key block j with rows t: w_t = softmax_t(s a.k_t),
+    ktil_j = sum_t w_t k_t, vtil_j = sum_t w_t v_t,
+    bias_j = logsumexp_t(s a.k_t) - log n_j - s a.ktil_j.
+    Returns (ktil [B, H, nb, D], vtil [B, H, nb, D], bias [B, H, nb]).
+    """
+    B, N, H, D = K.shape
+    a = anchor(Q, prefix)                                    # [B, H, D]
+    logits = scale * np.einsum("bnhd,bhd->bhn", K, a)        # [B, H, N]
+    nb = n_blocks(N, bk)
+    ktil = np.zeros((B, H, nb, D))
+    vtil = np.zeros((B, H, nb, D))
+    bias = np.zeros((B, H, nb))
+    for j in range(nb):
+        lo, hi = j * bk, min((j + 1) * bk, N)
+        x = logits[:, :, lo:hi]
+        m = x.max(axis=-1, keepdims=True)
+        e = np.exp(x - m)
+        z = e.sum(axis=-1)                                   # [B, H]
+        w = e / z[..., None]                                 # [B, H, n]
+        ktil[:, :, j] = np.einsum("bhn,bnhd->bhd", w, K[:, lo:hi])
+        vtil[:, :, j] = np.einsum("bhn,bnhd->bhd", w, V[:, lo:hi])
+        lse = m[..., 0] + np.log(z)
+        bias[:, :, j] = lse - math.log(hi - lo) - scale * np.einsum("bhd,bhd->bh", a, ktil[:, :, j])
+    return ktil, vtil, bias
+
+
 def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
               rows: Optional[dict] = None):
     """Exact + centroid attention (step 4).
@@ -191,19 +230,28 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
 
 def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: int = 64,
                 scale: Optional[float] = None, log_mass_bias_on: bool = False,
-                mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None):
-    """The whole forward pass; returns a dict of every intermediate."""
+                mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None,
+                reweight_on: bool = False):
+    """The whole forward pass; returns a dict of every intermediate.
+
+    ``reweight_on`` (step 6) gives the centroid terms the anchor-weighted
+    summaries ``kc``/``vc`` and their bias; otherwise ``kc``/``vc`` are the
+    mean-pooled kbar/vbar.
+    """
     D = Q.shape[-1]
     s = (1.0 / math.sqrt(D)) if not scale else float(scale)
     qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
     S = scores(qbar, kbar, s)
     thr = thresholds(S, tau)
     sel = route(S, tau, prefix, bq, bk)
-    if log_mass_bias_on:
+    kc, vc = kbar, vbar
+    if reweight_on:
+        kc, vc, bias = reweighted_summaries(Q, K, V, prefix, s, bk)
+    elif log_mass_bias_on:
         bias = log_mass_bias(Q, K, kbar, prefix, s, bk)
     else:
         bias = np.zeros(kbar.shape[:3])
     used = sel if mask_override is None else mask_override
-    O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows)
-    return dict(qbar=qbar, kbar=kbar, vbar=vbar, S=S, thr=thr, sel=sel, bias=bias,
-                O=O, lse=lse, scale=s)
+    O, lse = attention(Q, K, V, used, kc, vc, bias, s, bq, bk, rows=rows)
+    return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kc, vc=vc, S=S, thr=thr, sel=sel,
+                bias=bias, O=O, lse=lse, scale=s)

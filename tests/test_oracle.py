@@ -320,3 +320,122 @@ def test_planted_mistakes_are_caught(monkeypatch):
                      ("log_mass_bias", bias_sign), ("pool", pool_sum)]:
         assert _pins_fail(monkeypatch, name, fn) > 0, name
         monkeypatch.undo()
+
+
+# ---------------------------------------------------------------- weighted summaries
+def _uniform_q(N, H, D, seed):
+    """Every query row of a head equal to one vector: the anchor itself."""
+    c = np.random.default_rng(seed).standard_normal((1, 1, H, D))
+    return np.repeat(c, N, axis=1)
+
+
+@pytest.mark.parametrize("N,bk,P", [(77, 16, 0), (77, 16, 9), (64, 8, 64), (50, 50, 3)])
+def test_reweight_anchor_query_is_exact(N, bk, P):
+    """A query equal to the anchor gets each centroid block's exact contribution
+    (mass and value), so any routing reproduces dense attention for it; the
+    mean-pooled summary with the bias gets the mass but not the value."""
+    _, K, V = rand_qkv(1, N, 2, 6, seed=14)
+    Q = _uniform_q(N, 2, 6, seed=15)
+    s = 1 / math.sqrt(6)
+    dense = dense_attention(Q, K, V, s)
+    none = np.zeros((1, 2, -(-N // 16), -(-N // bk)), bool)
+    for ov in (none, None):
+        o = sol_ref.sol_forward(Q, K, V, tau=0.3, prefix=P, bq=16, bk=bk, reweight_on=True,
+                                mask_override=ov)
+        np.testing.assert_allclose(o["O"], dense, rtol=1e-11, atol=1e-12)
+    lmb = sol_ref.sol_forward(Q, K, V, tau=0.3, prefix=P, bq=16, bk=bk, log_mass_bias_on=True,
+                              mask_override=none)
+    assert np.abs(lmb["O"] - dense).max() > 1e-3
+
+
+def test_reweight_bias_is_entropy_gap():
+    """log mean exp(x) - E_w[x] with w = softmax(x) equals H(w) - log n, so the
+    bias is the weights' entropy deficit: <= 0, and 0 exactly for uniform weights."""
+    Q, K, V = rand_qkv(2, 70, 2, 6, seed=16)
+    s = 1 / math.sqrt(6)
+    for P in (0, 11):
+        kc, vc, bias = sol_ref.reweighted_summaries(Q, K, V, P, s, 16)
+        a = sol_ref.anchor(Q, P)
+        for j in range(kc.shape[2]):
+            lo, hi = 16 * j, min(70, 16 * (j + 1))
+            x = s * np.einsum("bnhd,bhd->bhn", K[:, lo:hi], a)
+            w = np.exp(x - x.max(-1, keepdims=True))
+            w /= w.sum(-1, keepdims=True)
+            H = -(w * np.log(w)).sum(-1)
+            np.testing.assert_allclose(bias[:, :, j], H - math.log(hi - lo), rtol=1e-10,
+                                       atol=1e-12)
+            # summaries are convex combinations: inside each coordinate's range
+            for X, C in ((K, kc), (V, vc)):
+                blk = X[:, lo:hi].transpose(0, 2, 1, 3)
+                assert (C[:, :, j] <= blk.max(2) + 1e-12).all()
+                assert (C[:, :, j] >= blk.min(2) - 1e-12).all()
+        assert (bias <= 1e-13).all()
+
+
+def test_reweight_zero_anchor_is_mean_pooling():
+    """With a zero anchor the weights are uniform: the summaries are the block
+    means, the bias vanishes and the pass equals the plain one."""
+    Q, K, V = rand_qkv(1, 96, 2, 4, seed=17)
+    P = 8
+    Q[0, P + 44:] = -Q[0, P:P + 44]                       # video rows cancel in pairs
+    o = sol_ref.sol_forward(Q, K, V, tau=0.5, prefix=P, bq=16, bk=16, reweight_on=True)
+    p = sol_ref.sol_forward(Q, K, V, tau=0.5, prefix=P, bq=16, bk=16)
+    np.testing.assert_allclose(sol_ref.anchor(Q, P), 0, atol=1e-14)
+    np.testing.assert_allclose(o["kc"], p["kbar"], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(o["vc"], p["vbar"], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(o["bias"], 0, atol=1e-13)
+    np.testing.assert_allclose(o["O"], p["O"], rtol=1e-12, atol=1e-13)
+    assert (o["sel"] == p["sel"]).all()
+
+
+@pytest.mark.parametrize("tau", [-1.0, 1.0])
+def test_reweight_block_size_one_is_dense(tau):
+    Q, K, V = rand_qkv(1, 40, 2, 4, seed=18)
+    o = sol_ref.sol_forward(Q, K, V, tau=tau, prefix=3, bq=1, bk=1, reweight_on=True)
+    np.testing.assert_allclose(o["kc"], K.transpose(0, 2, 1, 3), rtol=1e-14)
+    np.testing.assert_allclose(o["vc"], V.transpose(0, 2, 1, 3), rtol=1e-14)
+    np.testing.assert_allclose(o["bias"], 0.0, atol=1e-12)
+    np.testing.assert_allclose(o["O"], dense_attention(Q, K, V, 0.5), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_reweight_matches_brute_random(seed):
+    rng = np.random.default_rng(300 + seed)
+    N = int(rng.integers(17, 90))
+    bq, bk = int(rng.choice([4, 8, 16])), int(rng.choice([4, 8, 16]))
+    P = int(rng.integers(0, N // 2))
+    tau = float(rng.choice([-0.5, 0.5, 1.0, 1.5]))
+    Q, K, V = rand_qkv(1, N, 2, 4, seed=400 + seed)
+    o = sol_ref.sol_forward(Q, K, V, tau=tau, prefix=P, bq=bq, bk=bk, reweight_on=True)
+    bo, bsel = brute.forward(Q, K, V, 1, N, 2, 4, tau, P, bq, bk, rw=True)
+    assert (o["sel"][0] == np.array(bsel[0])).all()
+    np.testing.assert_allclose(o["O"], np.array(bo), rtol=1e-11, atol=1e-12)
+
+
+def test_planted_reweight_mistakes_are_caught(monkeypatch):
+    good = sol_ref.reweighted_summaries
+
+    def unscaled_weights(Q, K, V, prefix, scale, bk):   # softmax of a.k without s
+        kc, vc, _ = good(Q, K, V, prefix, 1.0, bk)
+        _, _, bias = good(Q, K, V, prefix, scale, bk)
+        return kc, vc, bias
+
+    def bias_vs_mean(Q, K, V, prefix, scale, bk):       # bias taken against kbar
+        kc, vc, _ = good(Q, K, V, prefix, scale, bk)
+        return kc, vc, sol_ref.log_mass_bias(Q, K, sol_ref.pool(K, bk), prefix, scale, bk)
+
+    def mean_values(Q, K, V, prefix, scale, bk):        # values left mean-pooled
+        kc, _, bias = good(Q, K, V, prefix, scale, bk)
+        return kc, sol_ref.pool(V, bk), bias
+
+    for fn in (unscaled_weights, bias_vs_mean, mean_values):
+        monkeypatch.setattr(sol_ref, "reweighted_summaries", fn)
+        failures = 0
+        for test in (lambda: test_reweight_anchor_query_is_exact(77, 16, 9),
+                     lambda: test_reweight_matches_brute_random(0)):
+            try:
+                test()
+            except AssertionError:
+                failures += 1
+        assert failures > 0, fn.__name__
+        monkeypatch.undo()
