@@ -162,7 +162,8 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
     from oracle import sol_ref
     q, k, v = (synth.bf16_bits_to_f64(x) for x in synth.generate(w, heads=heads, b_offset=b_offset))
     t0 = time.perf_counter()
-    out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=w.log_mass_bias)
+    out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
+                              reweight_on=int(w.log_mass_bias) == 2)
     dt = time.perf_counter() - t0
     nk = sol_ref.block_rows(w.N, 64)
     work = int(sum(((nk[None, :] * out["sel"][b, h]).sum(1) * nk).sum()
@@ -339,7 +340,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="h56_n32768", choices=sorted(WORKLOADS))
     ap.add_argument("--tau", type=float, default=None)
-    ap.add_argument("--log-mass-bias", action="store_true")
+    ap.add_argument("--log-mass-bias", action="store_true", help="centroid terms with the log-mass bias")
+    ap.add_argument("--reweight", action="store_true",
+                    help="anchor-weighted key/value summaries with the log-mass bias")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
@@ -349,12 +352,14 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]()
-    if args.tau is not None or args.log_mass_bias:
+    if args.log_mass_bias and args.reweight:
+        ap.error("--log-mass-bias and --reweight are exclusive")
+    mode = 2 if args.reweight else int(args.log_mass_bias)
+    if args.tau is not None or mode:
         import dataclasses
-        w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau,
-                                log_mass_bias=args.log_mass_bias,
-                                name=f"{w.name}_tau{args.tau if args.tau is not None else w.tau:g}"
-                                     + ("_lmb" if args.log_mass_bias else ""))
+        w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau, log_mass_bias=mode,
+                                name=w.name + (f"_tau{args.tau:g}" if args.tau is not None else "")
+                                     + synth.mode_suffix(mode))
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -85,7 +85,7 @@ sol_status validate(const sol_params* p) {
   if (isnan(p->tau) || p->tau == INFINITY) return fail(SOL_ERR_INVALID_ARG, "tau must be finite or -inf");
   if (!(p->scale >= 0.f) || isinf(p->scale)) return fail(SOL_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->prefix_len < 0 || p->prefix_len > p->N) return fail(SOL_ERR_INVALID_ARG, "prefix_len %d outside [0, N]", p->prefix_len);
-  if (p->log_mass_bias != 0 && p->log_mass_bias != 1) return fail(SOL_ERR_INVALID_ARG, "log_mass_bias must be 0 or 1");
+  if (p->log_mass_bias < 0 || p->log_mass_bias > 2) return fail(SOL_ERR_INVALID_ARG, "log_mass_bias must be 0, 1 or 2");
   const int64_t nb = (p->N + kBlock - 1) / kBlock;
   if (nb > kMaxKeyBlocks) return fail(SOL_ERR_UNSUPPORTED, "N=%d exceeds the supported %d rows", p->N, kMaxKeyBlocks * kBlock);
   if ((int64_t)p->B * p->H * nb * nb >= (int64_t)INT32_MAX)
@@ -153,6 +153,14 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
   if (!p->log_mass_bias) {
     a.tensor_mask = 7; a.with_bias = 0;
     if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch");
+  } else if (p->log_mass_bias == 2) {
+    // Q first: the anchor weights the K and V rows of one fused pass.
+    a.tensor_mask = 1; a.with_bias = 0;
+    if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (q)");
+    e = launch_anchor(a.src[0], a.sb, a.sn, a.sh, a.qbar, p->B, p->N, p->H, p->D, L.nqb, p->prefix_len,
+                      at<float>(ws, L.anchor), st);
+    if (e != cudaSuccess) return cuda_fail(e, "sol_pool anchor launch");
+    if ((e = launch_pool_kv_reweight(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (k, v reweight)");
   } else {
     // Q (and V) first: the anchor (mean video query) must exist before the K pass.
     a.tensor_mask = 5; a.with_bias = 0;

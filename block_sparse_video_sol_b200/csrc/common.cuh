@@ -68,7 +68,7 @@ struct PoolArgs {
   int B, N, H, nb, prefix;
   float scale;
   int tensor_mask;               // bit t set: pool tensor t in this launch (grid.z = B * popcount)
-  int with_bias;                 // K pass also computes the log-mass bias
+  int with_bias;                 // K pass also computes the log-mass bias (mean summaries)
   float* qbar; float* kbar; __nv_bfloat16* kbar16; __nv_bfloat16* vbar16;
   float* cbias; const float* anchor;
 };
@@ -95,6 +95,7 @@ struct AttnArgs {
 
 // Launchers (defined in the kernel files; return the launch error).
 cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st);
+cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st);
 cudaError_t launch_anchor(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh, const float* qbar,
                           int B, int N, int H, int D, int nqb, int prefix, float* anchor, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st);

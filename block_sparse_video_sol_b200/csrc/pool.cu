@@ -116,6 +116,113 @@ __global__ void __launch_bounds__(HPB * (D / 8)) pool_kernel(const PoolArgs a) {
   }
 }
 
+// Anchor-weighted key/value summaries (Spark-H3 news page, Spark-Reweight
+// bullet: the compressed branch's mean-pooled summaries become weighted ones,
+// scored against one anchor per head).  Within key block j the weights are the
+// anchor's softmax over the block's rows, w_t = exp(s a.k_t) / sum_u exp(s a.k_u);
+// the centroid key and value the attention sees are ktil_j = sum_t w_t k_t and
+// vtil_j = sum_t w_t v_t (bf16), and the centroid-logit offset is
+// log n_j + bias_j = logsumexp_t(s a.k_t) - s a.ktil_j, so a query equal to the
+// anchor receives the block's exact contribution.  The fp32 mean of K is still
+// written: routing scores the mean-pooled centroids.
+//
+// One pass reads each K and V element once (the same HBM bytes as the mean
+// pooling of K and V): a thread owns 8 dims of one head of both tensors, keeps
+// 8 K rows and 8 V rows (16 x 16 B) in flight, and folds each group of 8 rows
+// into an online softmax (one rescale per group).  The dot a.k_t is reduced
+// over the head's TPH lanes with an xor butterfly, which leaves the bitwise
+// same value in every lane, so the online state is uniform over a head.
+template <int D, int HPB>
+__global__ void __launch_bounds__(HPB * (D / 8)) pool_kv_reweight_kernel(const PoolArgs a) {
+  constexpr int TPH = D / 8;  // threads per head
+  const int j = blockIdx.x;
+  const int h = blockIdx.y * HPB + threadIdx.x / TPH;
+  const int c = threadIdx.x % TPH;
+  const int b = blockIdx.z;
+  const bool active = h < a.H;
+  const int r0 = j * kBlock, r1 = min(a.N, r0 + kBlock), n = r1 - r0;
+  const int64_t off = (int64_t)b * a.sb + (int64_t)h * a.sh + c * 8;
+  const __nv_bfloat16* kb = a.src[1] + off;
+  const __nv_bfloat16* vb = a.src[2] + off;
+
+  float an[8], mean[8], wk[8], wv[8], m = -INFINITY, l = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    an[i] = active ? a.anchor[((int64_t)b * a.H + h) * D + c * 8 + i] : 0.f;
+    mean[i] = wk[i] = wv[i] = 0.f;
+  }
+
+  for (int r = r0; r < r1; r += 8) {
+    uint4 uk[8], uv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uk[k] = uv[k] = make_uint4(0, 0, 0, 0);
+      if (active && r + k < r1) {
+        uk[k] = __ldg(reinterpret_cast<const uint4*>(kb + (int64_t)(r + k) * a.sn));
+        uv[k] = __ldg(reinterpret_cast<const uint4*>(vb + (int64_t)(r + k) * a.sn));
+      }
+    }
+    float x[8], gmax = m;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float f[8], dot = 0.f;
+      bf16x8_to_f32(uk[k], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        mean[i] += f[i];
+        dot = fmaf(an[i], f[i], dot);
+      }
+#pragma unroll
+      for (int o = TPH / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      x[k] = (r + k < r1) ? a.scale * dot : -INFINITY;  // uniform over the CTA
+      gmax = fmaxf(gmax, x[k]);
+    }
+    // gmax is finite: row r is valid.  expf(-inf) = 0 covers the first group.
+    const float corr = expf(m - gmax);
+    m = gmax;
+    l *= corr;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { wk[i] *= corr; wv[i] *= corr; }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float e = expf(x[k] - m);
+      float fk[8], fv[8];
+      bf16x8_to_f32(uk[k], fk);
+      bf16x8_to_f32(uv[k], fv);
+      l += e;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        wk[i] = fmaf(e, fk[i], wk[i]);
+        wv[i] = fmaf(e, fv[i], wv[i]);
+      }
+    }
+  }
+  if (n <= 0) return;  // uniform over the CTA
+  const float inv_n = 1.f / (float)n, inv_l = 1.f / l;
+  float pooled = 0.f;  // s * a.ktil, reduced over the head's lanes (every lane takes part)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    mean[i] *= inv_n;
+    wk[i] *= inv_l;
+    wv[i] *= inv_l;
+    pooled = fmaf(an[i], wk[i], pooled);
+  }
+#pragma unroll
+  for (int o = TPH / 2; o > 0; o >>= 1) pooled += __shfl_xor_sync(0xffffffffu, pooled, o);
+  if (!active) return;
+  const int64_t row = ((int64_t)b * a.H + h) * a.nb + j;
+  float* dst = a.kbar + row * D + c * 8;
+  reinterpret_cast<float4*>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+  reinterpret_cast<uint4*>(a.kbar16 + row * D + c * 8)[0] =
+      make_uint4(pack_bf16x2(wk[0], wk[1]), pack_bf16x2(wk[2], wk[3]), pack_bf16x2(wk[4], wk[5]),
+                 pack_bf16x2(wk[6], wk[7]));
+  reinterpret_cast<uint4*>(a.vbar16 + row * D + c * 8)[0] =
+      make_uint4(pack_bf16x2(wv[0], wv[1]), pack_bf16x2(wv[2], wv[3]), pack_bf16x2(wv[4], wv[5]),
+                 pack_bf16x2(wv[6], wv[7]));
+  if (c == 0) a.cbias[row] = m + logf(l) - a.scale * pooled;
+}
+
 // Anchor a = mean of the query rows >= prefix (all rows when prefix >= N),
 // from the pooled Q block means plus the rows of the block the prefix ends in.
 template <int D>
@@ -143,6 +250,19 @@ cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st) {
     constexpr int HPB = 16;
     dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B * nt);
     pool_kernel<64, HPB><<<grid, HPB * 8, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st) {
+  if (D == 128) {
+    constexpr int HPB = 8;
+    dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B);
+    pool_kv_reweight_kernel<128, HPB><<<grid, HPB * 16, 0, st>>>(a);
+  } else {
+    constexpr int HPB = 16;
+    dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B);
+    pool_kv_reweight_kernel<64, HPB><<<grid, HPB * 8, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -73,12 +73,16 @@ def _check(status: int, where: str):
 
 
 def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: int = 0,
-                log_mass_bias: bool = False, scale: float = 0.0, in_strides=None, out_strides=None,
+                log_mass_bias: int = 0, scale: float = 0.0, in_strides=None, out_strides=None,
                 q_block: int = 64, k_block: int = 64) -> sol_params:
-    """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D]."""
+    """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D].
+
+    ``log_mass_bias``: 0 (or False) mean-pooled centroids, 1 (or True) plus the
+    log-mass bias, 2 anchor-weighted key/value summaries with the bias.
+    """
     in_strides = in_strides or (N * H * D, H * D, D)
     out_strides = out_strides or (N * H * D, H * D, D)
-    return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(bool(log_mass_bias)),
+    return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(log_mass_bias),
                       *[int(s) for s in in_strides], *[int(s) for s in out_strides])
 
 
@@ -179,7 +183,7 @@ def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
-              log_mass_bias: bool = False, scale: float = 0.0, with_lse: bool = False):
+              log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False):
     """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
 
     Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.

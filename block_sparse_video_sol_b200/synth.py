@@ -53,7 +53,7 @@ class Workload:
     prefix: int = 0
     tau: float = 1.0
     seed: int = 1000
-    log_mass_bias: bool = False
+    log_mass_bias: int = 0     # centroid mode: 0 means, 1 + log-mass bias, 2 weighted summaries
     q_block: int = 64
     k_block: int = 64
 
@@ -75,10 +75,15 @@ def h56_n4096() -> Workload:
                     n_topics=64, seed=1001)
 
 
-def h56_sweep(N: int, tau: float = 1.0, log_mass_bias: bool = False) -> Workload:
+def mode_suffix(log_mass_bias: int) -> str:
+    """Workload-name suffix of a centroid mode."""
+    return ("", "_lmb", "_rw")[int(log_mass_bias)]
+
+
+def h56_sweep(N: int, tau: float = 1.0, log_mass_bias: int = 0) -> Workload:
     if N % 1024:
         raise ValueError("length sweep uses N = T*1024")
-    return Workload(f"h56_n{N}_d128_tau{tau:g}" + ("_lmb" if log_mass_bias else ""),
+    return Workload(f"h56_n{N}_d128_tau{tau:g}" + mode_suffix(log_mass_bias),
                     B=1, H=56, N=N, D=128, grid=(N // 1024, 32, 32), n_topics=128,
                     tau=tau, log_mass_bias=log_mass_bias, seed=1002)
 

@@ -71,9 +71,17 @@ typedef struct {
   int32_t prefix_len;        /* rows [0, prefix_len) are the packed text/audio prefix:
                                 key blocks holding any of them are always exact (KV sink),
                                 query blocks holding any of them attend densely */
-  int32_t log_mass_bias;     /* 0: centroid logit s*q.kbar_j + log n_j;
-                                1: plus bias_j = log mean_t exp(s*a.k_t) - s*a.kbar_j with
-                                   anchor a = mean of the query rows >= prefix_len */
+  int32_t log_mass_bias;     /* centroid terms of unselected key blocks (Spark-H3 news page,
+                                Spark-Reweight bullet); a = anchor = mean of the query rows
+                                >= prefix_len (all rows when prefix_len = N):
+                                0: logit s*q.kbar_j + log n_j, value vbar_j (block means);
+                                1: plus bias_j = log mean_t exp(s*a.k_t) - s*a.kbar_j;
+                                2: anchor-weighted summaries: with w_t = softmax over the
+                                   block's rows of s*a.k_t, key ktil_j = sum_t w_t k_t, value
+                                   vtil_j = sum_t w_t v_t, logit s*q.ktil_j + log n_j + bias_j,
+                                   bias_j = log mean_t exp(s*a.k_t) - s*a.ktil_j.
+                                Routing always scores the block means.  Other values:
+                                SOL_ERR_INVALID_ARG. */
   int64_t in_stride_b, in_stride_n, in_stride_h;    /* element strides of Q, K, V */
   int64_t out_stride_b, out_stride_n, out_stride_h; /* element strides of O */
 } sol_params;
@@ -87,8 +95,10 @@ size_t sol_workspace_bytes(const sol_params* p);
  * sol_pool / sol_route leave in the workspace, for inspection and tests:
  *   offsets[0] qbar   fp32 [B, H, nqb, D]     offsets[1] kbar   fp32 [B, H, nkb, D]
  *   offsets[2] kbar   bf16 [B, H, nkb, D]     offsets[3] vbar   bf16 [B, H, nkb, D]
+ *              (the centroid key/value the attention uses: ktil_j / vtil_j when
+ *              log_mass_bias = 2, the block means otherwise)
  *   offsets[4] centroid-logit offset fp32 [B, H, nkb] = log n_j (+ bias_j)
- *   offsets[5] anchor fp32 [B, H, D] (log_mass_bias only)
+ *   offsets[5] anchor fp32 [B, H, D] (log_mass_bias 1 or 2 only)
  *   offsets[6] exact-block bitmap uint32 [B*H*nqb, ceil(nkb/32)]
  *   offsets[7] row counts int32 [B*H*nqb]
  * with nqb = nkb = ceil(N/64).  Returns SOL_ERR_INVALID_ARG for a bad p or
@@ -105,7 +115,9 @@ int64_t sol_col_capacity(const sol_params* p);
  *            256-byte aligned.  Receives, per (b, h, block): qbar, kbar as
  *            fp32, kbar and vbar as bf16, the valid row count n_j, and the
  *            centroid-logit offset log n_j (+ bias_j when log_mass_bias).
- * Means are over each block's valid rows, accumulated in fp32. */
+ * Means are over each block's valid rows, accumulated in fp32.  With
+ * log_mass_bias = 2 the bf16 key/value centroids are the anchor-weighted
+ * summaries, computed in one pass over K and V after the anchor. */
 sol_status sol_pool(const sol_params* p, const void* q, const void* k, const void* v,
                     void* ws, size_t ws_bytes, void* stream);
 

@@ -3,7 +3,9 @@ and compare each stage with the fp64 oracle.
 
 Criteria (bf16 I/O, fp32 accumulate):
   * pooled centroids: fp32 means within 1e-5 relative (+1e-6 absolute) of the
-    oracle; bf16 copies within one bf16 rounding of the oracle's mean;
+    oracle; bf16 copies within one bf16 rounding of the oracle's mean (of the
+    anchor-weighted summary in mode 2, +1e-5 absolute for the fp32 weighted
+    sums with expf weights);
   * routing: the GPU mask equals the oracle's on every block whose score is
     more than 1e-4 from its row threshold, and the GPU CSR equals the
     oracle's CSR of the GPU mask bit for bit;
@@ -46,6 +48,11 @@ def gpu_mask(p, buf):
     return rp, ci, sol_ref.from_csr(rp, ci, (p.B, p.H, nb, nb))
 
 
+def oracle_modes(lmb):
+    """sol_forward flags for the centroid mode 0 / 1 (bias) / 2 (weighted summaries)."""
+    return dict(log_mass_bias_on=int(lmb) == 1, reweight_on=int(lmb) == 2)
+
+
 def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix):
     """Pooled quantities of the given head indices vs the oracle."""
     from block_sparse_video_sol_b200 import sol
@@ -55,10 +62,16 @@ def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix):
     g = {k: w[k][:, heads].float().cpu().numpy().astype(np.float64) for k in ("qbar", "kbar", "kbar16", "vbar16", "cbias")}
     np.testing.assert_allclose(g["qbar"], qbar, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(g["kbar"], kbar, rtol=1e-5, atol=1e-6)
-    np.testing.assert_allclose(g["kbar16"], kbar, rtol=2 ** -8, atol=1e-6)
-    np.testing.assert_allclose(g["vbar16"], vbar, rtol=2 ** -8, atol=1e-6)
     logn = np.log(sol_ref.block_rows(p.N, 64).astype(np.float64))
-    want = logn[None, None, :] + (sol_ref.log_mass_bias(Qd, Kd, kbar, prefix, s, 64) if lmb else 0.0)
+    if int(lmb) == 2:
+        kc, vc, bias = sol_ref.reweighted_summaries(Qd, Kd, Vd, prefix, s, 64)
+        np.testing.assert_allclose(g["kbar16"], kc, rtol=2 ** -8, atol=1e-5)
+        np.testing.assert_allclose(g["vbar16"], vc, rtol=2 ** -8, atol=1e-5)
+    else:
+        np.testing.assert_allclose(g["kbar16"], kbar, rtol=2 ** -8, atol=1e-6)
+        np.testing.assert_allclose(g["vbar16"], vbar, rtol=2 ** -8, atol=1e-6)
+        bias = sol_ref.log_mass_bias(Qd, Kd, kbar, prefix, s, 64) if lmb else 0.0
+    want = logn[None, None, :] + bias
     want = np.broadcast_to(want, g["cbias"].shape)
     np.testing.assert_allclose(g["cbias"], want, rtol=0, atol=2e-4)
     return qbar, kbar, vbar
@@ -84,8 +97,8 @@ def check_route(p, buf, qbar, kbar, heads, tau, prefix):
 
 def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None):
     """O (and lse) of the given heads vs the oracle run on the GPU mask."""
-    ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, log_mass_bias_on=lmb,
-                              mask_override=gm_heads, rows=rows)
+    ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, mask_override=gm_heads, rows=rows,
+                              **oracle_modes(lmb))
     O = buf.o[:, :, heads].float().cpu().numpy().astype(np.float64)
     Oref = ref["O"]
     keep = ~np.isnan(Oref)

@@ -69,6 +69,12 @@ def test_argument_validation_is_synchronous(sol):
     assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, prefix_len=1001)) == sol.SOL_ERR_INVALID_ARG
     assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, in_strides=(512000, 516, 128))) == sol.SOL_ERR_INVALID_ARG
     assert _call_pool(sol, sol.make_params(1, 70000, 4, 128)) == sol.SOL_ERR_UNSUPPORTED
+    for mode in (-1, 3):
+        assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, log_mass_bias=mode)) == sol.SOL_ERR_INVALID_ARG
+        assert "log_mass_bias" in sol.lib.sol_last_error_text().decode()
+    for mode in (1, 2):   # valid modes pass validation and reach the size check
+        assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, log_mass_bias=mode), ws_bytes=10) \
+            == sol.SOL_ERR_WORKSPACE
     assert _call_pool(sol, ok, ptr=4100) == sol.SOL_ERR_INVALID_ARG          # misaligned
     assert _call_pool(sol, ok, ws_bytes=10) == sol.SOL_ERR_WORKSPACE
     assert sol.lib.sol_pool(ctypes.byref(ok), None, 4096, 4096, 4096, 1 << 30, None) == sol.SOL_ERR_INVALID_ARG

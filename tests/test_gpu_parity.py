@@ -25,7 +25,7 @@ def test_tiny_workload_full():
     assert r["flips"] <= 2
 
 
-@pytest.mark.parametrize("lmb", [False, True])
+@pytest.mark.parametrize("lmb", [0, 1, 2])
 def test_ragged_prefix_batch2_d64(lmb):
     # N = 1000 (tail block of 40 rows), prefix 100 (mixed block 1), B = 2
     w = synth.Workload("ragged", B=2, H=3, N=1000, D=64, grid=(9, 10, 10), n_topics=8, prefix=100,
@@ -33,7 +33,7 @@ def test_ragged_prefix_batch2_d64(lmb):
     parity.full_check(w)
 
 
-@pytest.mark.parametrize("lmb", [False, True])
+@pytest.mark.parametrize("lmb", [0, 1, 2])
 def test_ragged_prefix_d128(lmb):
     w = synth.Workload("ragged128", B=1, H=4, N=777, D=128, grid=(4, 1, 191), n_topics=8, prefix=13,
                        tau=1.0, seed=8, log_mass_bias=lmb)
@@ -48,7 +48,7 @@ def test_h56_n4096_full():
 
 
 @pytest.mark.parametrize("tau", [0.5, 2.0])
-@pytest.mark.parametrize("lmb", [False, True])
+@pytest.mark.parametrize("lmb", [0, 1, 2])
 def test_tau_sweep_n8192(tau, lmb):
     # the density sweep of the length-sweep workload: tau sets how many blocks
     # each query block takes exactly, hence the mix of blocks one or both of a
@@ -96,9 +96,33 @@ def test_fused_qkv_strided_views():
 
 
 @pytest.mark.parametrize("N", [1, 5, 63, 64, 65])
-def test_small_and_single_block(N):
-    w = synth.Workload(f"small{N}", B=1, H=2, N=N, D=64, grid=(1, 1, N), n_topics=2, tau=0.0, seed=12 + N)
+@pytest.mark.parametrize("lmb", [0, 2])
+def test_small_and_single_block(N, lmb):
+    w = synth.Workload(f"small{N}", B=1, H=2, N=N, D=64, grid=(1, 1, N), n_topics=2, tau=0.0, seed=12 + N,
+                       log_mass_bias=lmb)
     parity.full_check(w)
+
+
+@pytest.mark.parametrize("N,D,prefix", [(8192, 128, 0), (5000, 64, 321)])
+def test_reweight_anchor_queries_match_dense(N, D, prefix):
+    """With every query row equal to the anchor, the weighted summaries give each
+    centroid block its exact contribution, so the sparse output equals dense
+    attention whatever the routing (fp32 SDPA on the same bf16 inputs)."""
+    w = synth.Workload("anchorq", B=1, H=4, N=N, D=D, grid=(1, 1, N - prefix), n_topics=16, prefix=prefix,
+                       tau=1.0, seed=14)
+    q, k, v = synth.generate(w)
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    Q = Q[:, :1].expand_as(Q).contiguous()
+    p, buf = parity.run_gpu(Q, K, V, 1.0, prefix, 2)
+    nb = -(-N // 64)
+    assert int(buf.row_ptr[-1]) < 0.5 * 4 * nb * nb          # most blocks are centroid terms
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.float().transpose(1, 2), K.float().transpose(1, 2), V.float().transpose(1, 2)).transpose(1, 2)
+    err = (buf.o.float() - ref).abs()
+    assert err.max().item() <= parity.MAX_ABS and err.mean().item() <= parity.MEAN_ABS
+    # the mean-pooled summaries with the bias do not have this property
+    p1, buf1 = parity.run_gpu(Q, K, V, 1.0, prefix, 1)
+    assert (buf1.o.float() - ref).abs().mean().item() > 2 * err.mean().item()
 
 
 def test_empty_problem_is_noop():
@@ -138,10 +162,11 @@ def test_h56_n32768_sampled():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("lmb", [False, True])
+@pytest.mark.parametrize("lmb", [0, 1, 2])
 def test_joint_sequence_sampled(lmb):
     w = synth.h56_joint()
     if lmb:
-        w = synth.Workload(w.name + "_lmb", w.B, w.H, w.N, w.D, w.grid, w.n_topics, w.prefix, w.tau, w.seed, True)
+        w = synth.Workload(w.name + synth.mode_suffix(lmb), w.B, w.H, w.N, w.D, w.grid, w.n_topics, w.prefix,
+                           w.tau, w.seed, lmb)
     r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=1)
     assert r["flips"] <= 20
