@@ -79,7 +79,9 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
             if log.strip():
                 print(f"== {os.path.basename(obj)}\n{log}", file=sys.stderr)
     tmp = out + ".tmp"
-    cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-cudart=static"]
+    # --no-undefined: a symbol missing from the sources fails the build, not the first dlopen
+    cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-cudart=static",
+           "-Xlinker", "--no-undefined"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -137,9 +137,11 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SOL_ERR_INVALID_ARG, "sol_pool: workspace not 256-byte aligned");
   const WsLayout L = ws_layout(*p);
   if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_pool: workspace %zu < %zu bytes", ws_bytes, L.total);
-  if ((s = check_arch()) != SOL_OK) return s;
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   PoolArgs a{};
+  a.status = status;
   a.src[0] = static_cast<const __nv_bfloat16*>(q);
   a.src[1] = static_cast<const __nv_bfloat16*>(k);
   a.src[2] = static_cast<const __nv_bfloat16*>(v);

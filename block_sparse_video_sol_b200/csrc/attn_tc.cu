@@ -40,6 +40,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace sol {
 namespace {
@@ -86,7 +87,6 @@ __device__ __forceinline__ unsigned int sol_gtime() {
 #else
 #define SOL_TRACE_AT(slot, step) do { } while (0)
 #endif
-constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr float kRescale = 8.0f;   // log2 units: rescale O when the max grows by more than 2^8
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -126,56 +126,6 @@ struct Extra {
   unsigned int trace[kTraceSlots * kTraceSteps];
 #endif
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t c) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(b)), "r"(c));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-               : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
-  return ok != 0;
-}
-// Bounded wait: false (and the CTA-wide abort flag set) on expiry or abort.
-__device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status) {
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if (*abort_flag) return false;
-    if (i >= kSpinLimit) {
-      *abort_flag = 1;
-      raise_status(status, SOL_ERR_TIMEOUT);
-      return false;
-    }
-    if (i > 2048) __nanosleep(64);
-  }
-}
-
-// Bounded wait that ignores the abort flag: used to drain issued copies / MMAs
-// before the CTA releases shared memory and TMEM.
-__device__ __forceinline__ void drain_bar(uint64_t* b, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try(b, parity)) return;
-    if (i > 32) __nanosleep(64);
-  }
-  raise_status(status, SOL_ERR_TIMEOUT);
-}
-
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, int c0, int c1, int c2, int c3, uint64_t* bar) {
-  asm volatile("cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
-               :: "r"(smem_u32(dst)), "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, int c0, int c1, int c2, uint64_t* bar) {
-  asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-               :: "r"(smem_u32(dst)), "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)) : "memory");
-}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (canonical SW128 layout:
 // 128-byte rows, 8-row groups 1024 bytes apart).
@@ -238,26 +188,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Packed fp32 pair arithmetic (sm_100a f32x2): halves the instruction count
-// of the softmax's elementwise work.
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -796,32 +726,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 }
 
 // ---- host side: tensor maps and launch ------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-              const cuuint32_t* box) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mkb, mvb;
@@ -832,9 +736,9 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   const cuuint64_t dims3[3] = {(cuuint64_t)D, (cuuint64_t)a.nkb, (cuuint64_t)a.B * a.H};
   const cuuint64_t str3[2] = {(cuuint64_t)D * 2, (cuuint64_t)a.nkb * D * 2};
   const cuuint32_t box3[3] = {64, 128, 1};
-  if (!make_map(&mq, a.q, 4, dims4, str4, box4) || !make_map(&mk, a.k, 4, dims4, str4, box4) ||
-      !make_map(&mv, a.v, 4, dims4, str4, box4) || !make_map(&mkb, a.kbar16, 3, dims3, str3, box3) ||
-      !make_map(&mvb, a.vbar16, 3, dims3, str3, box3))
+  if (!make_map(&mq, a.q, 4, dims4, str4, box4, kSw128) || !make_map(&mk, a.k, 4, dims4, str4, box4, kSw128) ||
+      !make_map(&mv, a.v, 4, dims4, str4, box4, kSw128) || !make_map(&mkb, a.kbar16, 3, dims3, str3, box3, kSw128) ||
+      !make_map(&mvb, a.vbar16, 3, dims3, str3, box3, kSw128))
     return cudaErrorInvalidValue;
   TcParams prm{a, (a.nkb + 31) / 32};
   const size_t smem = 1024 + Cfg<D>::kSmemTiles + sizeof(Extra);

@@ -71,6 +71,7 @@ struct PoolArgs {
   int with_bias;                 // K pass also computes the log-mass bias (mean summaries)
   float* qbar; float* kbar; __nv_bfloat16* kbar16; __nv_bfloat16* vbar16;
   float* cbias; const float* anchor;
+  int* status;                   // device status word (bounded waits)
 };
 
 struct RouteArgs {

@@ -14,6 +14,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "ptx.cuh"   // packed f32x2 arithmetic
 
 namespace sol {
 
@@ -126,18 +127,36 @@ __global__ void __launch_bounds__(HPB * (D / 8)) pool_kernel(const PoolArgs a) {
 // anchor receives the block's exact contribution.  The fp32 mean of K is still
 // written: routing scores the mean-pooled centroids.
 //
-// One pass reads each K and V element once (the same HBM bytes as the mean
-// pooling of K and V): a thread owns 8 dims of one head of both tensors, keeps
-// 8 K rows and 8 V rows (16 x 16 B) in flight, and folds each group of 8 rows
-// into an online softmax (one rescale per group).  The dot a.k_t is reduced
-// over the head's TPH lanes with an xor butterfly, which leaves the bitwise
-// same value in every lane, so the online state is uniform over a head.
-template <int D, int HPB>
-__global__ void __launch_bounds__(HPB * (D / 8)) pool_kv_reweight_kernel(const PoolArgs a) {
-  constexpr int TPH = D / 8;  // threads per head
+// One pass reads each K and V element once.  A CTA owns one key block of
+// kHeads heads; a thread owns 8 dims (one 16-byte chunk) of one head and
+// streams the block's rows in groups of 4 (8 loads in flight), folding each
+// group into an online softmax:
+//   - partial dots of the 4 rows with the anchor, reduced over the head's
+//     chunk lanes by a transposing butterfly that leaves each lane one row's
+//     full dot (5 shuffles for 4 rows instead of 16);
+//   - the group's max (2 shuffles), one rescale of the running sums per
+//     group, and the 4 rows' weights gathered back to every lane (4 shuffles);
+//   - key sum, weighted key and weighted value in packed f32x2 arithmetic.
+// No shared memory and no barrier: warps are independent and hide each
+// other's load latency (about 120 registers, four CTAs per SM).  Measured against
+// this form on B200: a TMA-staged one-tile CTA, and persistent TMA-ring CTAs
+// (with and without a producer warp) whose barrier-separated phases left
+// each tile's critical path too long; both were slower.
+template <int D>
+struct RwCfg {
+  static constexpr int kChunks = D / 8;            // lanes per head
+  static constexpr int kThreads = 128;
+  static constexpr int kHeads = kThreads / kChunks;   // heads per CTA: 8 (D = 128) or 16 (D = 64)
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 4) pool_kv_reweight_kernel(const PoolArgs a) {
+  using C = RwCfg<D>;
+  constexpr int CH = C::kChunks, B1 = CH / 2, B2 = CH / 4;
+  const int lane = threadIdx.x % 32;
   const int j = blockIdx.x;
-  const int h = blockIdx.y * HPB + threadIdx.x / TPH;
-  const int c = threadIdx.x % TPH;
+  const int h = blockIdx.y * C::kHeads + threadIdx.x / CH;
+  const int c = threadIdx.x % CH;
   const int b = blockIdx.z;
   const bool active = h < a.H;
   const int r0 = j * kBlock, r1 = min(a.N, r0 + kBlock), n = r1 - r0;
@@ -145,99 +164,175 @@ __global__ void __launch_bounds__(HPB * (D / 8)) pool_kv_reweight_kernel(const P
   const __nv_bfloat16* kb = a.src[1] + off;
   const __nv_bfloat16* vb = a.src[2] + off;
 
-  float an[8], mean[8], wk[8], wv[8], m = -INFINITY, l = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    an[i] = active ? a.anchor[((int64_t)b * a.H + h) * D + c * 8 + i] : 0.f;
-    mean[i] = wk[i] = wv[i] = 0.f;
+  uint64_t an2[4];   // this chunk of the anchor, as packed pairs
+  {
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    if (active) {
+      a0 = *reinterpret_cast<const float4*>(a.anchor + ((int64_t)b * a.H + h) * D + c * 8);
+      a1 = *reinterpret_cast<const float4*>(a.anchor + ((int64_t)b * a.H + h) * D + c * 8 + 4);
+    }
+    an2[0] = f2pack(a0.x, a0.y);
+    an2[1] = f2pack(a0.z, a0.w);
+    an2[2] = f2pack(a1.x, a1.y);
+    an2[3] = f2pack(a1.z, a1.w);
   }
+  // After the butterfly this lane holds the full dot of row `own` of a group;
+  // the lanes holding rows 0..3 differ from it only in bits B1 and B2.
+  const bool b1 = lane & B1, b2 = lane & B2;
+  const int own = (b1 ? 2 : 0) + (b2 ? 1 : 0);
+  const int base_lane = lane & ~(B1 | B2);
 
-  for (int r = r0; r < r1; r += 8) {
-    uint4 uk[8], uv[8];
+  auto load = [&](int r, uint4* kr, uint4* vr) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uk[k] = uv[k] = make_uint4(0, 0, 0, 0);
-      if (active && r + k < r1) {
-        uk[k] = __ldg(reinterpret_cast<const uint4*>(kb + (int64_t)(r + k) * a.sn));
-        uv[k] = __ldg(reinterpret_cast<const uint4*>(vb + (int64_t)(r + k) * a.sn));
+    for (int i = 0; i < 4; ++i) {
+      kr[i] = vr[i] = make_uint4(0, 0, 0, 0);
+      if (active && r + i < r1) {
+        kr[i] = __ldg(reinterpret_cast<const uint4*>(kb + (int64_t)(r + i) * a.sn));
+        vr[i] = __ldg(reinterpret_cast<const uint4*>(vb + (int64_t)(r + i) * a.sn));
       }
     }
-    float x[8], gmax = m;
+  };
+  auto pair = [](uint32_t w) { return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+  auto word = [](const uint4& u, int e) { return e == 0 ? u.x : e == 1 ? u.y : e == 2 ? u.z : u.w; };
+
+  uint64_t sk[4] = {0, 0, 0, 0}, wk[4] = {0, 0, 0, 0}, wv[4] = {0, 0, 0, 0};   // packed (0.f, 0.f)
+  float m = -INFINITY, l = 0.f;
+  // The next group's loads are issued at the end of each iteration (measured
+  // on B200: the same loop with the loads at its top ran 35% slower).
+  uint4 kr[4], vr[4];
+  load(r0, kr, vr);
+  for (int r = r0; r < r1; r += 4) {   // uniform over the CTA
+    uint64_t k2[4][4];
+    float p[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float f[8], dot = 0.f;
-      bf16x8_to_f32(uk[k], f);
+    for (int i = 0; i < 4; ++i) {
+      uint64_t acc = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        mean[i] += f[i];
-        dot = fmaf(an[i], f[i], dot);
+      for (int e = 0; e < 4; ++e) {
+        k2[i][e] = pair(word(kr[i], e));
+        acc = ffma2(an2[e], k2[i][e], acc);
+        sk[e] = fadd2(sk[e], k2[i][e]);
       }
-#pragma unroll
-      for (int o = TPH / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      x[k] = (r + k < r1) ? a.scale * dot : -INFINITY;  // uniform over the CTA
-      gmax = fmaxf(gmax, x[k]);
+      float lo, hi;
+      f2unpack(acc, lo, hi);
+      p[i] = lo + hi;
     }
-    // gmax is finite: row r is valid.  expf(-inf) = 0 covers the first group.
-    const float corr = expf(m - gmax);
-    m = gmax;
-    l *= corr;
+    // transposing butterfly: 4 partial rows over CH lanes -> one full row dot per lane
+    const float u0 = (b1 ? p[2] : p[0]) + __shfl_xor_sync(0xffffffffu, b1 ? p[0] : p[2], B1);
+    const float u1 = (b1 ? p[3] : p[1]) + __shfl_xor_sync(0xffffffffu, b1 ? p[1] : p[3], B1);
+    float x = (b2 ? u1 : u0) + __shfl_xor_sync(0xffffffffu, b2 ? u0 : u1, B2);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { wk[i] *= corr; wv[i] *= corr; }
+    for (int o = B2 / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    x = r + own < r1 ? a.scale * x : -INFINITY;
+    float mg = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, B1));
+    mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, B2));
+    const float mn = fmaxf(m, mg);     // finite: row r is valid
+    const float corr = expf(m - mn);   // 0 for the first group
+    const float e = expf(x - mn);      // 0 for rows past N
+    m = mn;
+    float w[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float e = expf(x[k] - m);
-      float fk[8], fv[8];
-      bf16x8_to_f32(uk[k], fk);
-      bf16x8_to_f32(uv[k], fv);
-      l += e;
+    for (int i = 0; i < 4; ++i)
+      w[i] = __shfl_sync(0xffffffffu, e, base_lane | ((i & 2) ? B1 : 0) | ((i & 1) ? B2 : 0));
+    l = fmaf(l, corr, (w[0] + w[1]) + (w[2] + w[3]));
+    const uint64_t c2 = f2pack(corr, corr);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        wk[i] = fmaf(e, fk[i], wk[i]);
-        wv[i] = fmaf(e, fv[i], wv[i]);
+    for (int q = 0; q < 4; ++q) {
+      wk[q] = ffma2(wk[q], c2, 0);
+      wv[q] = ffma2(wv[q], c2, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t w2 = f2pack(w[i], w[i]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        wk[q] = ffma2(w2, k2[i][q], wk[q]);
+        wv[q] = ffma2(w2, pair(word(vr[i], q)), wv[q]);
       }
     }
+    if (r + 4 < r1) load(r + 4, kr, vr);
   }
-  if (n <= 0) return;  // uniform over the CTA
+  // epilogue: normalise, s a.ktil over the head's lanes, write the centroid
   const float inv_n = 1.f / (float)n, inv_l = 1.f / l;
-  float pooled = 0.f;  // s * a.ktil, reduced over the head's lanes (every lane takes part)
+  float mk[8], tk[8], tv[8], pooled = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    f2unpack(sk[q], mk[2 * q], mk[2 * q + 1]);
+    f2unpack(wk[q], tk[2 * q], tk[2 * q + 1]);
+    f2unpack(wv[q], tv[2 * q], tv[2 * q + 1]);
+  }
+  float an[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) f2unpack(an2[q], an[2 * q], an[2 * q + 1]);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    mean[i] *= inv_n;
-    wk[i] *= inv_l;
-    wv[i] *= inv_l;
-    pooled = fmaf(an[i], wk[i], pooled);
+    mk[i] *= inv_n;
+    tk[i] *= inv_l;
+    tv[i] *= inv_l;
+    pooled = fmaf(an[i], tk[i], pooled);
   }
 #pragma unroll
-  for (int o = TPH / 2; o > 0; o >>= 1) pooled += __shfl_xor_sync(0xffffffffu, pooled, o);
+  for (int o = CH / 2; o > 0; o >>= 1) pooled += __shfl_xor_sync(0xffffffffu, pooled, o);
   if (!active) return;
   const int64_t row = ((int64_t)b * a.H + h) * a.nb + j;
   float* dst = a.kbar + row * D + c * 8;
-  reinterpret_cast<float4*>(dst)[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+  reinterpret_cast<float4*>(dst)[0] = make_float4(mk[0], mk[1], mk[2], mk[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(mk[4], mk[5], mk[6], mk[7]);
   reinterpret_cast<uint4*>(a.kbar16 + row * D + c * 8)[0] =
-      make_uint4(pack_bf16x2(wk[0], wk[1]), pack_bf16x2(wk[2], wk[3]), pack_bf16x2(wk[4], wk[5]),
-                 pack_bf16x2(wk[6], wk[7]));
+      make_uint4(pack_bf16x2(tk[0], tk[1]), pack_bf16x2(tk[2], tk[3]), pack_bf16x2(tk[4], tk[5]),
+                 pack_bf16x2(tk[6], tk[7]));
   reinterpret_cast<uint4*>(a.vbar16 + row * D + c * 8)[0] =
-      make_uint4(pack_bf16x2(wv[0], wv[1]), pack_bf16x2(wv[2], wv[3]), pack_bf16x2(wv[4], wv[5]),
-                 pack_bf16x2(wv[6], wv[7]));
+      make_uint4(pack_bf16x2(tv[0], tv[1]), pack_bf16x2(tv[2], tv[3]), pack_bf16x2(tv[4], tv[5]),
+                 pack_bf16x2(tv[6], tv[7]));
   if (c == 0) a.cbias[row] = m + logf(l) - a.scale * pooled;
 }
 
 // Anchor a = mean of the query rows >= prefix (all rows when prefix >= N),
-// from the pooled Q block means plus the rows of the block the prefix ends in.
+// from the pooled Q block means (weighted by their row counts) plus the rows
+// of the block the prefix ends in.  One CTA per (head, batch) with 1024
+// threads: a thread owns a float4 of dims and every G-th block, so the whole
+// 2-D sum is in flight in a few rounds; the G partial sums are then added in
+// a fixed order (deterministic).
 template <int D>
-__global__ void __launch_bounds__(D) anchor_kernel(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh,
-                                                   const float* qbar, int N, int H, int nqb, int prefix,
-                                                   float* anchor) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(1024) anchor_kernel(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh,
+                                                     const float* qbar, int N, int H, int nqb, int prefix,
+                                                     float* anchor) {
+  constexpr int C4 = D / 4;        // float4 columns of a row
+  constexpr int G = 1024 / C4;     // row groups: 32 (D = 128) or 64 (D = 64)
+  __shared__ float4 red[G][C4];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int c = threadIdx.x % C4, g = threadIdx.x / C4;
   const int P = prefix < N ? prefix : 0;
-  const int first = (P + kBlock - 1) / kBlock;
-  const float* qb = qbar + ((int64_t)b * H + h) * nqb * D + d;
-  float acc = 0.f;
-  for (int i = first; i < nqb; ++i) acc += qb[(int64_t)i * D] * (float)(min(N, (i + 1) * kBlock) - i * kBlock);
-  const __nv_bfloat16* qr = q + (int64_t)b * sb + (int64_t)h * sh + d;
-  for (int r = P; r < min(N, first * kBlock); ++r) acc += __bfloat162float(qr[(int64_t)r * sn]);
-  anchor[((int64_t)b * H + h) * D + d] = acc / (float)(N - P);
+  const int first = (P + kBlock - 1) / kBlock;   // first block lying wholly at or after P
+  const float4* qb = reinterpret_cast<const float4*>(qbar + ((int64_t)b * H + h) * nqb * D) + c;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int i = first + g; i < nqb; i += G) {
+    const float w = (float)(min(N, (i + 1) * kBlock) - i * kBlock);
+    const float4 x = qb[(int64_t)i * C4];
+    acc.x = fmaf(w, x.x, acc.x);
+    acc.y = fmaf(w, x.y, acc.y);
+    acc.z = fmaf(w, x.z, acc.z);
+    acc.w = fmaf(w, x.w, acc.w);
+  }
+  // rows [P, first*64) of the block the prefix ends in, read directly
+  const __nv_bfloat16* qr = q + (int64_t)b * sb + (int64_t)h * sh + c * 4;
+  for (int r = P + g; r < min(N, first * kBlock); r += G) {
+    const uint2 u = *reinterpret_cast<const uint2*>(qr + (int64_t)r * sn);
+    acc.x += __uint_as_float(u.x << 16);
+    acc.y += __uint_as_float(u.x & 0xffff0000u);
+    acc.z += __uint_as_float(u.y << 16);
+    acc.w += __uint_as_float(u.y & 0xffff0000u);
+  }
+  red[g][c] = acc;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int d = threadIdx.x;
+    const float* col = reinterpret_cast<const float*>(&red[0][0]) + d;
+    float t = 0.f;
+    for (int k = 0; k < G; ++k) t += col[k * D];
+    anchor[((int64_t)b * H + h) * D + d] = t / (float)(N - P);
+  }
 }
 
 cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st) {
@@ -256,13 +351,13 @@ cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st) {
 
 cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st) {
   if (D == 128) {
-    constexpr int HPB = 8;
-    dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B);
-    pool_kv_reweight_kernel<128, HPB><<<grid, HPB * 16, 0, st>>>(a);
+    using C = RwCfg<128>;
+    dim3 grid(a.nb, (a.H + C::kHeads - 1) / C::kHeads, a.B);
+    pool_kv_reweight_kernel<128><<<grid, C::kThreads, 0, st>>>(a);
   } else {
-    constexpr int HPB = 16;
-    dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B);
-    pool_kv_reweight_kernel<64, HPB><<<grid, HPB * 8, 0, st>>>(a);
+    using C = RwCfg<64>;
+    dim3 grid(a.nb, (a.H + C::kHeads - 1) / C::kHeads, a.B);
+    pool_kv_reweight_kernel<64><<<grid, C::kThreads, 0, st>>>(a);
   }
   return cudaGetLastError();
 }
@@ -270,8 +365,8 @@ cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st) {
 cudaError_t launch_anchor(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh, const float* qbar,
                           int B, int N, int H, int D, int nqb, int prefix, float* anchor, cudaStream_t st) {
   dim3 grid(H, B);
-  if (D == 128) anchor_kernel<128><<<grid, 128, 0, st>>>(q, sb, sn, sh, qbar, N, H, nqb, prefix, anchor);
-  else anchor_kernel<64><<<grid, 64, 0, st>>>(q, sb, sn, sh, qbar, N, H, nqb, prefix, anchor);
+  if (D == 128) anchor_kernel<128><<<grid, 1024, 0, st>>>(q, sb, sn, sh, qbar, N, H, nqb, prefix, anchor);
+  else anchor_kernel<64><<<grid, 1024, 0, st>>>(q, sb, sn, sh, qbar, N, H, nqb, prefix, anchor);
   return cudaGetLastError();
 }
 
