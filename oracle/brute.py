@@ -31,11 +31,14 @@ def _dot(x, y):
     return s
 
 
-def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=False):
+def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=False, topk=None):
     """Return (O[b][n][h][d], sel[b][h][i][j]) computed row by row.
 
     ``rw`` replaces the centroid key/value of every block by the anchor-softmax
     weighted summaries (and implies the log-mass bias, taken against them).
+    ``topk`` (an int k) routes each query block to its k highest-scoring key
+    blocks (equal scores: lower index first), keeps every key block for query
+    blocks holding prefix rows, and drops unselected blocks.
     """
     s = scale if scale else 1.0 / math.sqrt(D)
     nqb = (N + bq - 1) // bq
@@ -80,8 +83,19 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=
                 var = sum((x - mu) ** 2 for x in sc) / nkb
                 thr = -math.inf if tau == -math.inf else mu + tau * math.sqrt(var)
                 row = []
-                for j in range(nkb):
-                    row.append(i < n_dense or j < n_sink or sc[j] > thr)
+                if topk is None:
+                    for j in range(nkb):
+                        row.append(i < n_dense or j < n_sink or sc[j] > thr)
+                else:   # repeated selection of the best remaining block
+                    row = [i < n_dense] * nkb
+                    left = list(range(nkb))
+                    for _ in range(topk):
+                        best = left[0]
+                        for jj in left[1:]:
+                            if sc[jj] > sc[best]:
+                                best = jj
+                        row[best] = True
+                        left.remove(best)
                 sel_bh.append(row)
                 for r in range(qlo, qhi):
                     q = [float(x) for x in Q[b][r][h]]
@@ -91,7 +105,7 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=
                             for t in range(lo, hi):
                                 logits.append(s * _dot(q, [float(x) for x in K[b][t][h]]))
                                 vals.append([float(x) for x in V[b][t][h]])
-                        else:
+                        elif topk is None:
                             logits.append(s * _dot(q, kc[j]) + math.log(hi - lo) + bias[j])
                             vals.append(vc[j])
                     m = max(logits)

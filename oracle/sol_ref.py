@@ -40,6 +40,15 @@ What it computes, step by step, in the order the sources describe it:
                  against the weighted key.  A query equal to the anchor then
                  gets the block's exact contribution, mass and value alike.
                  Routing still scores the mean-pooled kbar.
+  7. Top-K routing (the SLA variant of the same kernels; Star7 README,
+                 section 工作原理 > SLA: Q=128 / K=64 dynamic Top-K block
+                 routing keeping about 15% of the key blocks, fp32 online
+                 softmax, full attention for the audio query range; Spark-H3
+                 news page, workflow paragraph: topk_ratio 0.2 / 0.1).  Each
+                 128-row query block keeps the k = ceil(ratio * n_kb) key
+                 blocks with the largest scores s * qbar_i . kbar_j; query
+                 blocks holding prefix rows keep every key block; unselected
+                 blocks contribute nothing (no centroid term).
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -48,7 +57,11 @@ one over all key blocks; the comparison is strict; a key block is a sink iff
 it holds a prefix row and a query block is dense iff it holds a prefix row;
 log n_j and the centroid use the block's valid row count; the bias is
 bias_j = logsumexp_t(s*a.k_t) - log n_j - s*a.kbar_j and does not change
-routing; tau = -inf selects every block.
+routing; tau = -inf selects every block.  Top-K: equal scores are ranked by
+the lower key-block index; ratio is the float32 the ABI carries and k =
+ceil(ratio * n_kb) is evaluated in double from it, at least 1; no key block
+is forced (the SLA passage names full attention for the prefix query rows
+only); the dense query blocks are the 128-row ones holding prefix rows.
 
 Layouts: Q, K, V, O are float64 arrays [B, N, H, D] (BTHD); per-head block
 quantities are [B, H, n_blocks, ...].
@@ -106,6 +119,20 @@ def route(S: np.ndarray, tau: float, prefix: int, bq: int, bk: int) -> np.ndarra
     n_dense = n_blocks(prefix, bq)
     sel[..., :, :n_sink] = True
     sel[..., :n_dense, :] = True
+    return sel
+
+
+def topk_count(ratio: float, nkb: int) -> int:
+    """Key blocks kept per query block by Top-K routing (step 7)."""
+    return max(1, min(nkb, math.ceil(float(np.float32(ratio)) * nkb)))
+
+
+def route_topk(S: np.ndarray, k: int, prefix: int, bq: int) -> np.ndarray:
+    """Top-K mask (step 7): the k largest scores of each row, ties to the lower index."""
+    order = np.argsort(-S, axis=-1, kind="stable")
+    sel = np.zeros(S.shape, bool)
+    np.put_along_axis(sel, order[..., :k], True, axis=-1)
+    sel[..., :n_blocks(prefix, bq), :] = True
     return sel
 
 
@@ -183,7 +210,7 @@ def reweighted_summaries(Q: np.ndarray, K: np.ndarray, V: np.ndarray, prefix: in
 
 
 def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
-              rows: Optional[dict] = None):
+              rows: Optional[dict] = None, centroids: bool = True):
     """Exact + centroid attention (step 4).
 
     For every query row r of block i (per b, h): logits are s*q_r.k_t for the
@@ -191,7 +218,8 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
     unselected key block j, with values v_t and vbar_j; the output is the
     softmax-weighted sum.  Returns (O [B, N, H, D], lse [B, H, N]) where lse is
     the natural-log normaliser.  ``rows`` optionally maps (b, h) to an array
-    of query rows to compute; other rows are left NaN.
+    of query rows to compute; other rows are left NaN.  With ``centroids``
+    False unselected blocks contribute nothing (Top-K routing, step 7).
     """
     B, N, H, D = Q.shape
     nqb, nkb = sel.shape[-2], sel.shape[-1]
@@ -214,7 +242,7 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
                 s_j = sel[b, h, i]
                 key_rows = np.concatenate([np.arange(j * bk, min((j + 1) * bk, N))
                                            for j in np.nonzero(s_j)[0]] or [np.zeros(0, int)])
-                cent = np.nonzero(~s_j)[0]
+                cent = np.nonzero(~s_j)[0] if centroids else np.zeros(0, int)
                 q = Q[b, r, h, :]
                 lg = np.concatenate([scale * q @ K[b, key_rows, h, :].T,
                                      scale * q @ kbar[b, h, cent, :].T
@@ -231,17 +259,27 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
 def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: int = 64,
                 scale: Optional[float] = None, log_mass_bias_on: bool = False,
                 mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None,
-                reweight_on: bool = False):
+                reweight_on: bool = False, topk_ratio: Optional[float] = None):
     """The whole forward pass; returns a dict of every intermediate.
 
     ``reweight_on`` (step 6) gives the centroid terms the anchor-weighted
     summaries ``kc``/``vc`` and their bias; otherwise ``kc``/``vc`` are the
-    mean-pooled kbar/vbar.
+    mean-pooled kbar/vbar.  ``topk_ratio`` selects Top-K routing (step 7)
+    with query blocks of ``bq`` rows (128 in the SLA contract) and no
+    centroid terms; tau and the bias options are then unused.
     """
     D = Q.shape[-1]
     s = (1.0 / math.sqrt(D)) if not scale else float(scale)
     qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
     S = scores(qbar, kbar, s)
+    if topk_ratio is not None:
+        k = topk_count(topk_ratio, kbar.shape[2])
+        sel = route_topk(S, k, prefix, bq)
+        bias = np.zeros(kbar.shape[:3])
+        used = sel if mask_override is None else mask_override
+        O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows, centroids=False)
+        return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kbar, vc=vbar, S=S, thr=None, sel=sel, k=k,
+                    bias=bias, O=O, lse=lse, scale=s)
     thr = thresholds(S, tau)
     sel = route(S, tau, prefix, bq, bk)
     kc, vc = kbar, vbar

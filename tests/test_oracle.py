@@ -439,3 +439,102 @@ def test_planted_reweight_mistakes_are_caught(monkeypatch):
                 failures += 1
         assert failures > 0, fn.__name__
         monkeypatch.undo()
+
+
+# ---------------------------------------------------------------- Top-K routing
+def test_topk_count_reading():
+    # k = ceil(ratio * n_kb) evaluated from the float32 ratio the ABI carries
+    assert sol_ref.topk_count(0.15, 512) == 77
+    assert sol_ref.topk_count(0.1, 10) == 2          # float32(0.1) * 10 is just above 1
+    assert sol_ref.topk_count(0.25, 512) == 128      # exact in float32
+    assert sol_ref.topk_count(1e-9, 100) == 1
+    assert sol_ref.topk_count(1.0, 100) == 100
+
+
+def test_topk_selection_invariants():
+    rng = np.random.default_rng(19)
+    S = rng.standard_normal((2, 3, 9, 40))
+    prev = None
+    for k in (1, 5, 12, 40):
+        sel = sol_ref.route_topk(S, k, prefix=0, bq=128)
+        assert (sel.sum(-1) == k).all()
+        # the selected scores dominate the unselected ones row by row
+        lo = np.where(sel, S, np.inf).min(-1)
+        hi = np.where(sel, -np.inf, S).max(-1)
+        assert (lo >= hi).all()
+        if prev is not None:
+            assert (sel | ~prev).all(), "top-k sets nest"
+        prev = sel
+    # ties rank the lower index first; prefix query blocks keep everything
+    T = np.zeros((1, 1, 3, 10))
+    T[..., 7] = 1.0
+    sel = sol_ref.route_topk(T, 3, prefix=130, bq=128)
+    assert sel[0, 0, :2].all()
+    assert np.nonzero(sel[0, 0, 2])[0].tolist() == [0, 1, 7]
+
+
+def _masked_dense(Q, K, V, sel, scale, bq, bk):
+    """Softmax attention of each query row over only the keys of its selected blocks."""
+    B, N, H, D = Q.shape
+    keep = np.repeat(np.repeat(sel, bq, axis=2)[:, :, :N], bk, axis=3)[..., :N]   # [B, H, N, N]
+    lg = scale * np.einsum("bnhd,bmhd->bhnm", Q, K)
+    lg = np.where(keep, lg, -np.inf)
+    lg -= lg.max(-1, keepdims=True)
+    p = np.exp(lg)
+    p /= p.sum(-1, keepdims=True)
+    return np.einsum("bhnm,bmhd->bnhd", p, V)
+
+
+@pytest.mark.parametrize("N,bq,bk,P,ratio", [(300, 128, 64, 0, 0.2), (257, 128, 64, 70, 0.1),
+                                             (90, 16, 8, 5, 0.3)])
+def test_topk_attention_is_masked_softmax(N, bq, bk, P, ratio):
+    """Unselected blocks are dropped: the output is softmax attention restricted to
+    the selected keys (no centroid term); ratio 1 gives dense attention."""
+    Q, K, V = rand_qkv(1, N, 2, 8, seed=20)
+    s = 1 / math.sqrt(8)
+    o = sol_ref.sol_forward(Q, K, V, prefix=P, bq=bq, bk=bk, topk_ratio=ratio)
+    nkb = -(-N // bk)
+    assert o["k"] == sol_ref.topk_count(ratio, nkb)
+    np.testing.assert_allclose(o["O"], _masked_dense(Q, K, V, o["sel"], s, bq, bk), rtol=1e-11, atol=1e-12)
+    full = sol_ref.sol_forward(Q, K, V, prefix=P, bq=bq, bk=bk, topk_ratio=1.0)
+    np.testing.assert_allclose(full["O"], dense_attention(Q, K, V, s), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_matches_brute_random(seed):
+    rng = np.random.default_rng(500 + seed)
+    N = int(rng.integers(17, 90))
+    bq, bk = int(rng.choice([8, 16, 32])), int(rng.choice([4, 8, 16]))
+    P = int(rng.integers(0, N // 2))
+    ratio = float(rng.choice([0.1, 0.25, 0.5]))
+    Q, K, V = rand_qkv(1, N, 2, 4, seed=600 + seed)
+    o = sol_ref.sol_forward(Q, K, V, prefix=P, bq=bq, bk=bk, topk_ratio=ratio)
+    bo, bsel = brute.forward(Q, K, V, 1, N, 2, 4, 0.0, P, bq, bk, topk=o["k"])
+    assert (o["sel"][0] == np.array(bsel[0])).all()
+    np.testing.assert_allclose(o["O"], np.array(bo), rtol=1e-11, atol=1e-12)
+
+
+def test_planted_topk_mistakes_are_caught(monkeypatch):
+    good_route, good_count, good_att = sol_ref.route_topk, sol_ref.topk_count, sol_ref.attention
+
+    def ties_high(S, k, prefix, bq):              # equal scores ranked by the higher index
+        return good_route(S[..., ::-1], k, prefix, bq)[..., ::-1]
+
+    def one_short(ratio, nkb):                    # floor instead of ceil
+        return max(1, int(float(np.float32(ratio)) * nkb))
+
+    def keeps_centroids(*args, centroids=True, **kw):
+        return good_att(*args, centroids=True, **kw)
+
+    for name, fn in [("route_topk", ties_high), ("topk_count", one_short), ("attention", keeps_centroids)]:
+        monkeypatch.setattr(sol_ref, name, fn)
+        failures = 0
+        for test in (test_topk_count_reading, test_topk_selection_invariants,
+                     lambda: test_topk_attention_is_masked_softmax(257, 128, 64, 70, 0.1),
+                     lambda: test_topk_matches_brute_random(0)):
+            try:
+                test()
+            except AssertionError:
+                failures += 1
+        assert failures > 0, name
+        monkeypatch.undo()
