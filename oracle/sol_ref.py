@@ -45,7 +45,7 @@ What it computes, step by step, in the order the sources describe it:
                  routing keeping about 15% of the key blocks, fp32 online
                  softmax, full attention for the audio query range; Spark-H3
                  news page, workflow paragraph: topk_ratio 0.2 / 0.1).  Each
-                 128-row query block keeps the k = ceil(ratio * n_kb) key
+                 128-row query block keeps the k = round(ratio * n_kb) key
                  blocks with the largest scores s * qbar_i . kbar_j; query
                  blocks holding prefix rows keep every key block; unselected
                  blocks contribute nothing (no centroid term).
@@ -59,7 +59,8 @@ log n_j and the centroid use the block's valid row count; the bias is
 bias_j = logsumexp_t(s*a.k_t) - log n_j - s*a.kbar_j and does not change
 routing; tau = -inf selects every block.  Top-K: equal scores are ranked by
 the lower key-block index; ratio is the float32 the ABI carries and k =
-ceil(ratio * n_kb) is evaluated in double from it, at least 1; no key block
+floor(ratio * n_kb + 0.5) (nearest, halves up) is evaluated in double from
+it, clamped to [1, n_kb]; no key block
 is forced (the SLA passage names full attention for the prefix query rows
 only); the dense query blocks are the 128-row ones holding prefix rows.
 
@@ -124,7 +125,7 @@ def route(S: np.ndarray, tau: float, prefix: int, bq: int, bk: int) -> np.ndarra
 
 def topk_count(ratio: float, nkb: int) -> int:
     """Key blocks kept per query block by Top-K routing (step 7)."""
-    return max(1, min(nkb, math.ceil(float(np.float32(ratio)) * nkb)))
+    return max(1, min(nkb, math.floor(float(np.float32(ratio)) * nkb + 0.5)))
 
 
 def route_topk(S: np.ndarray, k: int, prefix: int, bq: int) -> np.ndarray:

@@ -443,9 +443,11 @@ def test_planted_reweight_mistakes_are_caught(monkeypatch):
 
 # ---------------------------------------------------------------- Top-K routing
 def test_topk_count_reading():
-    # k = ceil(ratio * n_kb) evaluated from the float32 ratio the ABI carries
-    assert sol_ref.topk_count(0.15, 512) == 77
-    assert sol_ref.topk_count(0.1, 10) == 2          # float32(0.1) * 10 is just above 1
+    # k = nearest integer to ratio * n_kb (halves up), from the float32 ratio the ABI carries
+    assert sol_ref.topk_count(0.15, 512) == 77       # 76.8
+    assert sol_ref.topk_count(0.1, 10) == 1          # float32(0.1) * 10 is just above 1
+    assert sol_ref.topk_count(0.3, 10) == 3          # float32(0.3) * 10 is just above 3
+    assert sol_ref.topk_count(0.25, 10) == 3         # exactly 2.5: halves up
     assert sol_ref.topk_count(0.25, 512) == 128      # exact in float32
     assert sol_ref.topk_count(1e-9, 100) == 1
     assert sol_ref.topk_count(1.0, 100) == 100
@@ -520,7 +522,7 @@ def test_planted_topk_mistakes_are_caught(monkeypatch):
     def ties_high(S, k, prefix, bq):              # equal scores ranked by the higher index
         return good_route(S[..., ::-1], k, prefix, bq)[..., ::-1]
 
-    def one_short(ratio, nkb):                    # floor instead of ceil
+    def one_short(ratio, nkb):                    # floor instead of the nearest integer
         return max(1, int(float(np.float32(ratio)) * nkb))
 
     def keeps_centroids(*args, centroids=True, **kw):
