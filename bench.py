@@ -162,13 +162,23 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
     from oracle import sol_ref
     q, k, v = (synth.bf16_bits_to_f64(x) for x in synth.generate(w, heads=heads, b_offset=b_offset))
     t0 = time.perf_counter()
-    out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
-                              reweight_on=int(w.log_mass_bias) == 2)
+    if w.topk_ratio is not None:
+        out = sol_ref.sol_forward(q, k, v, prefix=w.prefix, bq=128, topk_ratio=w.topk_ratio)
+    else:
+        out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
+                                  reweight_on=int(w.log_mass_bias) == 2)
     dt = time.perf_counter() - t0
     nk = sol_ref.block_rows(w.N, 64)
-    work = int(sum(((nk[None, :] * out["sel"][b, h]).sum(1) * nk).sum()
+    nq = sol_ref.block_rows(w.N, 128 if w.topk_ratio is not None else 64)
+    work = int(sum(((nk[None, :] * out["sel"][b, h]).sum(1) * nq).sum()
                    for b in range(w.B) for h in range(len(heads))))
     return dt, work
+
+
+def routing_config(w: synth.Workload) -> dict:
+    if w.topk_ratio is None:
+        return {"routing": "threshold"}
+    return {"routing": "topk", "topk_ratio": w.topk_ratio, "q_block": 128}
 
 
 def cpu_threads():
@@ -200,7 +210,7 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
-                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias},
+                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, **routing_config(w)},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -224,7 +234,8 @@ def run_ours(args, w):
     synth.generate(w, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host),
                    b_offset=shard_b_offset(rank, w))
     q, k, v = (h.to(dev) for h in host)
-    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias)
+    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
+                        topk_ratio=w.topk_ratio)
     buf = sol.alloc_buffers(p, dev)
     stream = torch.cuda.current_stream()
     launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 1
@@ -296,12 +307,14 @@ def run_ours(args, w):
         attn_tf = flop / (attn_ms * 1e-3) / 1e12
         traffic, tnote = profiled_traffic("sol_attn_fwd")
         in_bytes = 3 * w.B * w.N * w.H * w.D * 2
+        pool_bytes = (2 if w.topk_ratio is not None else 3) * w.B * w.N * w.H * w.D * 2   # Top-K pools no V
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
-                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, "global_batch": w.B * world,
+                       "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, **routing_config(w),
+                       "global_batch": w.B * world,
                        "parallelism": f"dp{world} (one sequence per GPU)",
                        "l2": f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB), no flush"},
             "roofline": {"kernel": "sol_attn_fwd", "bound": "tensor", "achieved": attn_tf,
@@ -309,8 +322,8 @@ def run_ours(args, w):
                          "peak_source": f"{peaks['source']} bf16 burst", "traffic": traffic,
                          "traffic_note": tnote},
             "kernels": {
-                "sol_pool": {"ms": pool_ms, "GB/s": in_bytes / (pool_ms * 1e-3) / 1e9,
-                             "frac_hbm": in_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm"]},
+                "sol_pool": {"ms": pool_ms, "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                             "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm"]},
                 "sol_route": {"ms": route_ms,
                               "TFLOP/s_fp32": 2.0 * w.B * w.H * nb * nb * w.D / (route_ms * 1e-3) / 1e12},
                 "sol_attn_fwd": {"ms": attn_ms, "TFLOP/s_effective": attn_tf,
@@ -343,6 +356,8 @@ def main():
     ap.add_argument("--log-mass-bias", action="store_true", help="centroid terms with the log-mass bias")
     ap.add_argument("--reweight", action="store_true",
                     help="anchor-weighted key/value summaries with the log-mass bias")
+    ap.add_argument("--topk-ratio", type=float, default=None,
+                    help="Top-K routing (the SLA variant: 128-row query blocks, no centroid terms)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
@@ -355,11 +370,15 @@ def main():
     if args.log_mass_bias and args.reweight:
         ap.error("--log-mass-bias and --reweight are exclusive")
     mode = 2 if args.reweight else int(args.log_mass_bias)
-    if args.tau is not None or mode:
+    if args.topk_ratio is not None and (mode or args.tau is not None):
+        ap.error("--topk-ratio takes neither tau nor centroid options")
+    if args.tau is not None or mode or args.topk_ratio is not None:
         import dataclasses
         w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau, log_mass_bias=mode,
+                                topk_ratio=args.topk_ratio,
                                 name=w.name + (f"_tau{args.tau:g}" if args.tau is not None else "")
-                                     + synth.mode_suffix(mode))
+                                     + synth.mode_suffix(mode)
+                                     + (f"_topk{args.topk_ratio:g}" if args.topk_ratio is not None else ""))
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -12,6 +12,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -80,9 +81,18 @@ sol_status validate(const sol_params* p) {
   if (!p) return fail(SOL_ERR_INVALID_ARG, "params is NULL");
   if (p->B < 0 || p->N < 0 || p->H <= 0) return fail(SOL_ERR_INVALID_ARG, "bad shape B=%d N=%d H=%d", p->B, p->N, p->H);
   if (p->D != 64 && p->D != 128) return fail(SOL_ERR_UNSUPPORTED, "head dim %d unsupported (64 or 128)", p->D);
-  if (p->q_block != kBlock || p->k_block != kBlock)
-    return fail(SOL_ERR_UNSUPPORTED, "block sizes %d/%d unsupported (the GPU path takes 64/64)", p->q_block, p->k_block);
-  if (isnan(p->tau) || p->tau == INFINITY) return fail(SOL_ERR_INVALID_ARG, "tau must be finite or -inf");
+  if (p->routing != 0 && p->routing != 1) return fail(SOL_ERR_INVALID_ARG, "routing must be 0 (threshold) or 1 (top-k)");
+  const int want_q = p->routing == 1 ? 2 * kBlock : kBlock;
+  if (p->q_block != want_q || p->k_block != kBlock)
+    return fail(SOL_ERR_UNSUPPORTED, "block sizes %d/%d unsupported (routing %d takes %d/%d)", p->q_block, p->k_block,
+                p->routing, want_q, kBlock);
+  if (p->routing == 1) {
+    if (!(p->topk_ratio > 0.f && p->topk_ratio <= 1.f))
+      return fail(SOL_ERR_INVALID_ARG, "topk_ratio must lie in (0, 1]");
+    if (p->log_mass_bias != 0) return fail(SOL_ERR_INVALID_ARG, "top-k routing has no centroid terms: log_mass_bias must be 0");
+  }
+  if (p->routing == 0 && (isnan(p->tau) || p->tau == INFINITY))
+    return fail(SOL_ERR_INVALID_ARG, "tau must be finite or -inf");
   if (!(p->scale >= 0.f) || isinf(p->scale)) return fail(SOL_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->prefix_len < 0 || p->prefix_len > p->N) return fail(SOL_ERR_INVALID_ARG, "prefix_len %d outside [0, N]", p->prefix_len);
   if (p->log_mass_bias < 0 || p->log_mass_bias > 2) return fail(SOL_ERR_INVALID_ARG, "log_mass_bias must be 0, 1 or 2");
@@ -97,6 +107,26 @@ sol_status validate(const sol_params* p) {
 }
 
 float eff_scale(const sol_params* p) { return p->scale > 0.f ? p->scale : 1.f / sqrtf((float)p->D); }
+
+// Routing kernel arguments shared by sol_route and sol_route_static (the
+// caller sets mask and counts).
+RouteArgs route_args(const sol_params* p, const WsLayout& L, const void* ws) {
+  RouteArgs a{};
+  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
+  a.B = p->B; a.H = p->H; a.N = p->N; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
+  a.scale = eff_scale(p); a.tau = p->tau;
+  if (p->routing == 1) {   // 128-row query rows, no KV sink
+    const double kk = floor((double)p->topk_ratio * (double)L.nkb + 0.5);   // nearest, halves up
+    a.topk = (int)std::max(1.0, std::min((double)L.nkb, kk));
+    a.n_sink = 0;
+    a.n_dense = (p->prefix_len + 2 * kBlock - 1) / (2 * kBlock);
+  } else {
+    a.topk = 0;
+    a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
+    a.n_dense = a.n_sink;
+  }
+  return a;
+}
 bool empty(const sol_params* p) { return p->B == 0 || p->N == 0; }
 
 }  // namespace
@@ -152,7 +182,10 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
   a.kbar16 = at<__nv_bfloat16>(ws, L.kbar16); a.vbar16 = at<__nv_bfloat16>(ws, L.vbar16);
   a.cbias = at<float>(ws, L.cbias); a.anchor = at<float>(ws, L.anchor);
   cudaError_t e;
-  if (!p->log_mass_bias) {
+  if (p->routing == 1) {   // Top-K routing needs no V centroids
+    a.tensor_mask = 3; a.with_bias = 0;
+    if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch");
+  } else if (!p->log_mass_bias) {
     a.tensor_mask = 7; a.with_bias = 0;
     if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch");
   } else if (p->log_mass_bias == 2) {
@@ -186,12 +219,7 @@ sol_status sol_route(const sol_params* p, void* ws, size_t ws_bytes, int32_t* ro
   if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_route: workspace %zu < %zu bytes", ws_bytes, L.total);
   if ((s = check_arch()) != SOL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  RouteArgs a{};
-  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
-  a.B = p->B; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
-  a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
-  a.n_dense = a.n_sink;
-  a.scale = eff_scale(p); a.tau = p->tau;
+  RouteArgs a = route_args(p, L, ws);
   a.mask = at<uint32_t>(ws, L.mask); a.counts = at<int32_t>(ws, L.counts);
   cudaError_t e = launch_route(a, p->D, st);
   if (e != cudaSuccess) return cuda_fail(e, "sol_route launch");
@@ -228,6 +256,7 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
   a.row_ptr = row_ptr; a.col_idx = col_idx;
   a.B = p->B; a.N = p->N; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb;
   a.scale = eff_scale(p);
+  a.centroids = p->routing == 0 ? 1 : 0;
   cudaError_t e = launch_attn(a, p->D, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sol_attn_fwd launch");
   return SOL_OK;
@@ -337,12 +366,7 @@ extern "C" sol_status sol_route_static(const sol_params* p, const void* ws, size
   unsigned char* scratch = nullptr;
   if ((s = route_scratch(&scratch)) != SOL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  RouteArgs a{};
-  a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
-  a.B = p->B; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
-  a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
-  a.n_dense = a.n_sink;
-  a.scale = eff_scale(p); a.tau = p->tau;
+  RouteArgs a = route_args(p, L, ws);
   a.mask = reinterpret_cast<uint32_t*>(scratch);
   a.counts = reinterpret_cast<int32_t*>(scratch + mask_bytes);
   cudaError_t e = launch_route(a, p->D, st);

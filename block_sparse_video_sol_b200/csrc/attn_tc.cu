@@ -345,7 +345,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       int n = 0;
       for (int ct = 0; ct < 8; ++ct)
         if ((wb >> (4 * ct)) & 0xFu) x.cent[n++] = ct;
-      x.n_cent = n;
+      x.n_cent = a.centroids ? n : 0;   // Top-K routing drops unselected blocks
     }
   }
   cta_sync();

@@ -76,8 +76,9 @@ struct PoolArgs {
 
 struct RouteArgs {
   const float* qbar; const float* kbar;
-  int B, H, nqb, nkb, mask_words, n_sink, n_dense;
+  int B, H, N, nqb, nkb, mask_words, n_sink, n_dense;   // n_dense counts the kernel's query rows
   float scale, tau;
+  int topk;                      // > 0: Top-K routing of 128-row query blocks keeping topk key blocks
   uint32_t* mask; int32_t* counts;
 };
 
@@ -91,6 +92,7 @@ struct AttnArgs {
   const int32_t* row_ptr; const int32_t* col_idx;
   int B, N, H, nqb, nkb;
   float scale;
+  int centroids;                 // 1: a centroid term per unselected key block; 0: unselected blocks dropped
   int* status;
 };
 

@@ -13,6 +13,15 @@
 // One CTA owns 32 query blocks of one (b, h) and all key blocks; it keeps
 // its 32 x nkb score rows in shared memory so that the mean, the population
 // std and the mask come from one evaluation of S.
+//
+// The same kernel does Top-K routing (the SLA variant: Star7 README, section
+// 工作原理 > SLA, Q=128 / K=64 dynamic Top-K): its query rows are then 128-row
+// blocks, whose centroid is the row-weighted mean of their two 64-row block
+// means, and a warp finds each row's k-th largest score exactly by a
+// bitwise binary search over order-preserving integer keys (32 counting
+// rounds over the row held in registers), then marks the scores above it
+// and, in index order, as many equal to it as k still needs.  Both 64-row
+// halves of a 128-row block get the same list.
 #include <math.h>
 
 #include "common.cuh"
@@ -30,6 +39,60 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// Top-K selection for one 128-row query block i (one warp; see the file
+// comment).  Column j = lane + 32 e lives in key[e]; columns past nkb get
+// key 0, below every real score (order-preserving keys of floats are >= 1).
+__device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, int i, int bh, int lane) {
+  const int nkb = a.nkb, k = a.topk;
+  const bool dense = i < a.n_dense;
+  uint32_t key[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int j = lane + 32 * e;
+    const uint32_t u = j < nkb ? __float_as_uint(Sr[j]) : 0u;
+    key[e] = j < nkb ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
+  }
+  uint32_t p = 0u;   // the k-th largest key: the largest v with #{key >= v} >= k
+  int need = 0;      // how many keys equal to p are still to be taken
+  if (!dense) {      // uniform over the warp
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = p | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) c += key[e] >= cand ? 1 : 0;
+      if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) p = cand;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) gt += key[e] > p ? 1 : 0;
+    need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+  }
+  const int64_t row0 = (int64_t)bh * a.nqb + 2 * i;
+  const bool second = 2 * i + 1 < a.nqb;
+  int cnt = 0;
+#pragma unroll
+  for (int w = 0; w < 32; ++w) {
+    if (w < a.mask_words) {   // uniform
+      const bool valid = lane + 32 * w < nkb;
+      const bool eq = valid && key[w] == p;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const int before = __popc(eqb & ((1u << lane) - 1u));
+      const bool sel = valid && (dense || key[w] > p || (eq && before < need));
+      need -= __popc(eqb);
+      const uint32_t bits = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) {
+        a.mask[row0 * a.mask_words + w] = bits;
+        if (second) a.mask[(row0 + 1) * a.mask_words + w] = bits;
+      }
+      cnt += __popc(bits);
+    }
+  }
+  if (lane == 0) {
+    a.counts[row0] = cnt;
+    if (second) a.counts[row0 + 1] = cnt;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) {
   extern __shared__ __align__(16) float sm[];
@@ -40,10 +103,22 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   const int bh = blockIdx.y, i0 = blockIdx.x * kRouteTQ;
   const float* qbar = a.qbar + (int64_t)bh * a.nqb * D;
   const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
+  const int nrows = a.topk ? (a.nqb + 1) / 2 : a.nqb;   // the kernel's query rows
 
   for (int idx = tid; idx < kRouteTQ * D; idx += 256) {
-    const int r = idx % kRouteTQ, d = idx / kRouteTQ;
-    qT[d * kRouteTQ + r] = (i0 + r < a.nqb) ? qbar[(int64_t)(i0 + r) * D + d] : 0.f;
+    const int r = idx % kRouteTQ, d = idx / kRouteTQ, i = i0 + r;
+    float v = 0.f;
+    if (i < nrows) {
+      if (a.topk) {   // 128-row block: row-weighted mean of its 64-row block means
+        const float n0 = (float)(min(a.N, 128 * i + 64) - 128 * i);
+        const float n1 = 2 * i + 1 < a.nqb ? (float)(min(a.N, 128 * i + 128) - (128 * i + 64)) : 0.f;
+        const float q1 = n1 > 0.f ? qbar[(int64_t)(2 * i + 1) * D + d] : 0.f;
+        v = (n0 * qbar[(int64_t)(2 * i) * D + d] + n1 * q1) / (n0 + n1);
+      } else {
+        v = qbar[(int64_t)i * D + d];
+      }
+    }
+    qT[d * kRouteTQ + r] = v;
   }
   const int rg = warp & 3;   // rows 8*rg .. 8*rg+7
   const int chh = warp >> 2; // columns 128*chh .. +127 of the chunk
@@ -97,8 +172,12 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   const float inv_n = 1.f / (float)a.nkb;
   for (int rr = 0; rr < kRouteTQ / 8; ++rr) {
     const int r = warp * (kRouteTQ / 8) + rr, i = i0 + r;
-    if (i >= a.nqb) break;
+    if (i >= nrows) break;
     const float* Sr = S + r * ldS;
+    if (a.topk) {
+      topk_row(a, Sr, i, bh, lane);
+      continue;
+    }
     float s = 0.f;
     for (int j = lane; j < a.nkb; j += 32) s += Sr[j];
     const float mu = warp_sum(s) * inv_n;
@@ -175,7 +254,8 @@ static size_t route_smem_bytes(int D, int ldS) {
 cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
   const int ldS = ((a.nkb + 3) / 4) * 4;
   const size_t smem = route_smem_bytes(D, ldS);
-  dim3 grid((a.nqb + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
+  const int nrows = a.topk ? (a.nqb + 1) / 2 : a.nqb;
+  dim3 grid((nrows + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
   cudaError_t e;
   if (D == 128) {
     e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -33,7 +33,8 @@ class sol_params(ctypes.Structure):
                 ("tau", ctypes.c_float), ("scale", ctypes.c_float),
                 ("prefix_len", ctypes.c_int32), ("log_mass_bias", ctypes.c_int32),
                 ("in_stride_b", ctypes.c_int64), ("in_stride_n", ctypes.c_int64), ("in_stride_h", ctypes.c_int64),
-                ("out_stride_b", ctypes.c_int64), ("out_stride_n", ctypes.c_int64), ("out_stride_h", ctypes.c_int64)]
+                ("out_stride_b", ctypes.c_int64), ("out_stride_n", ctypes.c_int64), ("out_stride_h", ctypes.c_int64),
+                ("routing", ctypes.c_int32), ("topk_ratio", ctypes.c_float)]
 
 
 _P = ctypes.POINTER(sol_params)
@@ -74,16 +75,22 @@ def _check(status: int, where: str):
 
 def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: int = 0,
                 log_mass_bias: int = 0, scale: float = 0.0, in_strides=None, out_strides=None,
-                q_block: int = 64, k_block: int = 64) -> sol_params:
+                q_block: Optional[int] = None, k_block: int = 64, topk_ratio: Optional[float] = None) -> sol_params:
     """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D].
 
     ``log_mass_bias``: 0 (or False) mean-pooled centroids, 1 (or True) plus the
     log-mass bias, 2 anchor-weighted key/value summaries with the bias.
+    ``topk_ratio`` selects Top-K routing (128-row query blocks, unselected
+    blocks dropped); otherwise threshold routing with ``tau``.
     """
+    routing = 0 if topk_ratio is None else 1
+    if q_block is None:
+        q_block = 128 if routing else 64
     in_strides = in_strides or (N * H * D, H * D, D)
     out_strides = out_strides or (N * H * D, H * D, D)
     return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(log_mass_bias),
-                      *[int(s) for s in in_strides], *[int(s) for s in out_strides])
+                      *[int(s) for s in in_strides], *[int(s) for s in out_strides], routing,
+                      float(topk_ratio or 0.0))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -108,7 +115,7 @@ def sol_workspace_offsets(p: sol_params) -> list:
 def workspace_views(p: sol_params, ws: torch.Tensor) -> dict:
     """Typed views of the pooled quantities inside a workspace (see sol_workspace_offsets)."""
     off = sol_workspace_offsets(p)
-    nb = -(-p.N // p.q_block)
+    nb = -(-p.N // 64)   # the workspace holds 64-row blocks for Q and K whatever the routing
     mw = -(-nb // 32)
     B, H, D = p.B, p.H, p.D
 
@@ -165,7 +172,7 @@ class Buffers:
 
 
 def alloc_buffers(p: sol_params, device, with_lse: bool = False) -> Buffers:
-    nqb = -(-p.N // p.q_block)
+    nqb = -(-p.N // 64)   # CSR rows are 64-row query blocks whatever the routing
     ws = torch.empty(max(1, sol_workspace_bytes(p)), dtype=torch.uint8, device=device)
     row_ptr = torch.empty(p.B * p.H * nqb + 1, dtype=torch.int32, device=device)
     col_idx = torch.empty(max(1, sol_col_capacity(p)), dtype=torch.int32, device=device)
@@ -183,7 +190,8 @@ def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
-              log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False):
+              log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False,
+              topk_ratio: Optional[float] = None):
     """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
 
     Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.
@@ -193,7 +201,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.
         if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(3) != 1 or t.stride() != q.stride():
             raise ValueError("q, k, v must be bf16 CUDA tensors with identical strides and contiguous head dim")
     p = make_params(B, N, H, D, tau, prefix_len, log_mass_bias, scale,
-                    in_strides=(q.stride(0), q.stride(1), q.stride(2)))
+                    in_strides=(q.stride(0), q.stride(1), q.stride(2)), topk_ratio=topk_ratio)
     buf = alloc_buffers(p, q.device, with_lse)
     forward(p, q, k, v, buf)
     return buf.o, buf

@@ -84,6 +84,18 @@ typedef struct {
                                 SOL_ERR_INVALID_ARG. */
   int64_t in_stride_b, in_stride_n, in_stride_h;    /* element strides of Q, K, V */
   int64_t out_stride_b, out_stride_n, out_stride_h; /* element strides of O */
+  int32_t routing;           /* 0: Sol threshold routing (tau), q_block = 64, a centroid term per
+                                unselected key block (Star7 README 工作原理 > Sol);
+                                1: Top-K routing, the SLA variant (Star7 README 工作原理 > SLA):
+                                q_block = 128, each 128-row query block keeps the
+                                k = round(topk_ratio * ceil(N/64)) key blocks with the largest
+                                scores (equal scores: lower index first), query blocks holding
+                                prefix rows keep every key block, unselected blocks are
+                                dropped; tau is unused and log_mass_bias must be 0.
+                                Other values: SOL_ERR_INVALID_ARG. */
+  float topk_ratio;          /* routing 1: fraction of key blocks kept, in (0, 1];
+                                k = floor(topk_ratio * n_kb + 0.5) in double precision from this
+                                float (nearest, halves up), clamped to [1, n_kb]. */
 } sol_params;
 
 /* Bytes of device workspace that sol_pool / sol_route / sol_attn_fwd share for
@@ -105,7 +117,7 @@ size_t sol_workspace_bytes(const sol_params* p);
  * a NULL offsets array. */
 sol_status sol_workspace_offsets(const sol_params* p, int64_t offsets[8]);
 
-/* Worst-case number of CSR column entries: B*H*ceil(N/q_block)*ceil(N/k_block). */
+/* Worst-case number of CSR column entries: B*H*ceil(N/64)*ceil(N/64) (64-row query-block rows). */
 int64_t sol_col_capacity(const sol_params* p);
 
 /* sol_pool: block centroids (Star7 README 工作原理 > Sol; Spark-H3 news page,
@@ -122,15 +134,20 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
                     void* ws, size_t ws_bytes, void* stream);
 
 /* sol_route: block scores and CSR lists of exact key blocks (thakicloud blog,
- * 이 기술은 무엇인가; Star7 README 工作原理 > Sol).
+ * 이 기술은 무엇인가; Star7 README 工作原理 > Sol, and 工作原理 > SLA for
+ * routing 1).
  *   ws       workspace filled by sol_pool for the same p.
- *   row_ptr  int32 [B*H*ceil(N/q_block) + 1] device, written: exclusive scan
+ *   row_ptr  int32 [B*H*ceil(N/64) + 1] device, written: exclusive scan
  *            of the per-row counts in (b, h, i) order; row_ptr[last] = nnz.
+ *            Rows are 64-row query blocks for either routing (with routing 1
+ *            the two halves of a 128-row block carry the same list).
  *   col_idx  int32 device, capacity sol_col_capacity(p); row r's exact key
  *            blocks, ascending, at [row_ptr[r], row_ptr[r+1]).
- * S_ij = s * qbar_i . kbar_j in fp32; block j is exact for row i iff
- * S_ij > mean_j S_ij + tau * std_j S_ij (population std over all key
- * blocks), or j is a sink block, or i is a dense (prefix) query block. */
+ * Routing 0: S_ij = s * qbar_i . kbar_j in fp32; block j is exact for row i
+ * iff S_ij > mean_j S_ij + tau * std_j S_ij (population std over all key
+ * blocks), or j is a sink block, or i is a dense (prefix) query block.
+ * Routing 1: qbar_i over 128 rows; row i keeps its k largest S_ij (equal
+ * scores: lower j first), or every block if it holds prefix rows. */
 sol_status sol_route(const sol_params* p, void* ws, size_t ws_bytes,
                      int32_t* row_ptr, int32_t* col_idx, void* stream);
 

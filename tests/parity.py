@@ -7,7 +7,9 @@ Criteria (bf16 I/O, fp32 accumulate):
     anchor-weighted summary in mode 2, +1e-5 absolute for the fp32 weighted
     sums with expf weights);
   * routing: the GPU mask equals the oracle's on every block whose score is
-    more than 1e-4 from its row threshold, and the GPU CSR equals the
+    more than 1e-4 from its row threshold (Top-K: from the row's k-th
+    largest score, with exactly k blocks per row and both 64-row halves of a
+    128-row block carrying the same list), and the GPU CSR equals the
     oracle's CSR of the GPU mask bit for bit;
   * attention: with the oracle run on the GPU's mask, max |O_gpu - O_ref| <=
     2e-2 and mean |O_gpu - O_ref| <= 2e-3.
@@ -29,11 +31,12 @@ def to_dev(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None):
+def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None, topk_ratio=None):
     from block_sparse_video_sol_b200 import sol
     B, N, H, D = q.shape
     strides = in_strides or (q.stride(0), q.stride(1), q.stride(2))
-    p = sol.make_params(B, N, H, D, tau=tau, prefix_len=prefix, log_mass_bias=lmb, in_strides=strides)
+    p = sol.make_params(B, N, H, D, tau=tau, prefix_len=prefix, log_mass_bias=lmb, in_strides=strides,
+                        topk_ratio=topk_ratio)
     buf = sol.alloc_buffers(p, q.device, with_lse=with_lse)
     sol.forward(p, q, k, v, buf)
     sol.sol_last_device_status()
@@ -53,13 +56,14 @@ def oracle_modes(lmb):
     return dict(log_mass_bias_on=int(lmb) == 1, reweight_on=int(lmb) == 2)
 
 
-def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix):
-    """Pooled quantities of the given head indices vs the oracle."""
+def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix, topk=False):
+    """Pooled quantities of the given head indices vs the oracle (Top-K routing pools no V)."""
     from block_sparse_video_sol_b200 import sol
     w = sol.workspace_views(p, buf.ws)
     s = 1.0 / math.sqrt(p.D)
     qbar, kbar, vbar = sol_ref.pool(Qd, 64), sol_ref.pool(Kd, 64), sol_ref.pool(Vd, 64)
-    g = {k: w[k][:, heads].float().cpu().numpy().astype(np.float64) for k in ("qbar", "kbar", "kbar16", "vbar16", "cbias")}
+    names = ("qbar", "kbar", "kbar16", "cbias") + (() if topk else ("vbar16",))   # Top-K pools no V
+    g = {k: w[k][:, heads].float().cpu().numpy().astype(np.float64) for k in names}
     np.testing.assert_allclose(g["qbar"], qbar, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(g["kbar"], kbar, rtol=1e-5, atol=1e-6)
     logn = np.log(sol_ref.block_rows(p.N, 64).astype(np.float64))
@@ -69,7 +73,8 @@ def check_pool(p, buf, Qd, Kd, Vd, heads, lmb, prefix):
         np.testing.assert_allclose(g["vbar16"], vc, rtol=2 ** -8, atol=1e-5)
     else:
         np.testing.assert_allclose(g["kbar16"], kbar, rtol=2 ** -8, atol=1e-6)
-        np.testing.assert_allclose(g["vbar16"], vbar, rtol=2 ** -8, atol=1e-6)
+        if not topk:
+            np.testing.assert_allclose(g["vbar16"], vbar, rtol=2 ** -8, atol=1e-6)
         bias = sol_ref.log_mass_bias(Qd, Kd, kbar, prefix, s, 64) if lmb else 0.0
     want = logn[None, None, :] + bias
     want = np.broadcast_to(want, g["cbias"].shape)
@@ -95,10 +100,40 @@ def check_route(p, buf, qbar, kbar, heads, tau, prefix):
     return gm, int(((g != sel) & ~far).sum())
 
 
-def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None):
+def check_route_topk(p, buf, Qd, Kd, heads, ratio, prefix):
+    """Top-K mask parity outside the tie band, k per row, equal halves, CSR bit-exactness.
+
+    Returns the GPU mask of the given heads at 128-row query-block granularity."""
+    s = 1.0 / math.sqrt(p.D)
+    S = sol_ref.scores(sol_ref.pool(Qd, 128), sol_ref.pool(Kd, 64), s)
+    nkb = S.shape[-1]
+    k = sol_ref.topk_count(ratio, nkb)
+    sel = sol_ref.route_topk(S, k, prefix, 128)
+    rp, ci, gm = gpu_mask(p, buf)
+    rp_ref, ci_ref = sol_ref.to_csr(gm)
+    assert np.array_equal(rp, rp_ref) and np.array_equal(ci, ci_ref)
+    nqb = gm.shape[2]
+    assert (gm[:, :, 1::2] == gm[:, :, 0:nqb - nqb % 2:2]).all(), "both halves of a 128-row block share a list"
+    g = gm[:, :, ::2][:, heads]
+    n_dense = sol_ref.n_blocks(prefix, 128)
+    cnt = g.sum(-1)
+    assert (cnt[:, :, n_dense:] == k).all() and (cnt[:, :, :n_dense] == nkb).all()
+    kth = -np.sort(-S, axis=-1)[..., k - 1]
+    far = np.abs(S - kth[..., None]) > BAND
+    far[:, :, :n_dense] = True
+    bad = (g != sel) & far
+    assert not bad.any(), f"{int(bad.sum())} top-k mismatches outside the {BAND} band"
+    return gm, g, int(((g != sel) & ~far).sum())
+
+
+def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None, topk_ratio=None):
     """O (and lse) of the given heads vs the oracle run on the GPU mask."""
-    ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, mask_override=gm_heads, rows=rows,
-                              **oracle_modes(lmb))
+    if topk_ratio is not None:
+        ref = sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, bq=128, mask_override=gm_heads, rows=rows,
+                                  topk_ratio=topk_ratio)
+    else:
+        ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, mask_override=gm_heads, rows=rows,
+                                  **oracle_modes(lmb))
     O = buf.o[:, :, heads].float().cpu().numpy().astype(np.float64)
     Oref = ref["O"]
     keep = ~np.isnan(Oref)
@@ -117,15 +152,20 @@ def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
     """Generate a workload, run it on the GPU, check pool/route/attention on `heads`."""
     q, k, v = synth.generate(w)
     Q, K, V = to_dev(q), to_dev(k), to_dev(v)
-    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias)
+    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias, topk_ratio=w.topk_ratio)
     heads = list(range(w.H)) if heads is None else list(heads)
     Qd, Kd, Vd = (synth.bf16_bits_to_f64(x[:, :, heads]) for x in (q, k, v))
-    qbar, kbar, _ = check_pool(p, buf, Qd, Kd, Vd, heads, w.log_mass_bias, w.prefix)
-    gm, flips = check_route(p, buf, qbar, kbar, heads, w.tau, w.prefix)
+    qbar, kbar, _ = check_pool(p, buf, Qd, Kd, Vd, heads, w.log_mass_bias, w.prefix, topk=w.topk_ratio is not None)
+    if w.topk_ratio is not None:
+        _, g128, flips = check_route_topk(p, buf, Qd, Kd, heads, w.topk_ratio, w.prefix)
+    else:
+        gm, flips = check_route(p, buf, qbar, kbar, heads, w.tau, w.prefix)
     rows = None
     if rows_per_head:
         rng = np.random.default_rng(seed_rows)
         rows = {(b, hh): np.sort(rng.choice(w.N, size=min(rows_per_head, w.N), replace=False))
                 for b in range(w.B) for hh in range(len(heads))}
-    errs = check_attention(p, buf, Qd, Kd, Vd, gm[:, heads], heads, w.tau, w.prefix, w.log_mass_bias, rows)
+    mask = g128 if w.topk_ratio is not None else gm[:, heads]
+    errs = check_attention(p, buf, Qd, Kd, Vd, mask, heads, w.tau, w.prefix, w.log_mass_bias, rows,
+                           topk_ratio=w.topk_ratio)
     return dict(flips=flips, errs=errs, nnz=int(buf.row_ptr[-1].item()), p=p, buf=buf)

@@ -72,6 +72,14 @@ def test_argument_validation_is_synchronous(sol):
     for mode in (-1, 3):
         assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, log_mass_bias=mode)) == sol.SOL_ERR_INVALID_ARG
         assert "log_mass_bias" in sol.lib.sol_last_error_text().decode()
+    bad = sol.make_params(1, 1000, 4, 128, topk_ratio=0.2)
+    bad.routing = 2
+    assert _call_pool(sol, bad) == sol.SOL_ERR_INVALID_ARG
+    for r in (0.0, 1.5, float("nan")):
+        assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=r)) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=0.2, q_block=64)) == sol.SOL_ERR_UNSUPPORTED
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=0.2, log_mass_bias=1)) == sol.SOL_ERR_INVALID_ARG
+    assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=0.2), ws_bytes=10) == sol.SOL_ERR_WORKSPACE
     for mode in (1, 2):   # valid modes pass validation and reach the size check
         assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, log_mass_bias=mode), ws_bytes=10) \
             == sol.SOL_ERR_WORKSPACE

@@ -1,4 +1,5 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle."""
+import dataclasses
 import math
 
 import numpy as np
@@ -169,4 +170,71 @@ def test_joint_sequence_sampled(lmb):
         w = synth.Workload(w.name + synth.mode_suffix(lmb), w.B, w.H, w.N, w.D, w.grid, w.n_topics, w.prefix,
                            w.tau, w.seed, lmb)
     r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=1)
+    assert r["flips"] <= 20
+
+
+# ---------------------------------------------------------------- Top-K routing (SLA variant)
+@pytest.mark.parametrize("ratio", [0.2, 0.5])
+def test_topk_ragged_prefix_batch2_d64(ratio):
+    w = synth.Workload("topk_ragged", B=2, H=3, N=1000, D=64, grid=(9, 10, 10), n_topics=8, prefix=100,
+                       seed=21, topk_ratio=ratio)
+    parity.full_check(w)
+
+
+def test_topk_odd_blocks_d128():
+    # 13 query blocks of 64 rows: the last 128-row block has one half
+    w = synth.Workload("topk_odd", B=1, H=4, N=777, D=128, grid=(4, 1, 191), n_topics=8, prefix=13,
+                       seed=22, topk_ratio=0.15)
+    parity.full_check(w)
+
+
+@pytest.mark.parametrize("N", [1, 5, 63, 64, 65, 129])
+def test_topk_small(N):
+    w = synth.Workload(f"topk_small{N}", B=1, H=2, N=N, D=64, grid=(1, 1, N), n_topics=2, seed=23 + N,
+                       topk_ratio=0.3)
+    parity.full_check(w)
+
+
+def test_topk_h56_n8192():
+    w = dataclasses.replace(synth.h56_sweep(8192), name="h56_n8192_sla15", topk_ratio=0.15)
+    r = parity.full_check(w, heads=[0, 23, 55])
+    nb = 8192 // 64
+    assert r["nnz"] == 56 * nb * sol_ref.topk_count(0.15, nb)
+
+
+def test_topk_ties_take_lower_index():
+    # identical key rows give every key block the same score: the first k blocks are kept
+    from block_sparse_video_sol_b200 import sol
+    w = synth.Workload("ties", B=1, H=2, N=640, D=64, grid=(1, 1, 640), n_topics=4, seed=24)
+    q, k, v = synth.generate(w)
+    k[:] = k[:, :1]
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    p, buf = parity.run_gpu(Q, K, V, 1.0, 0, 0, topk_ratio=0.3)
+    rp, ci, gm = parity.gpu_mask(p, buf)
+    kk = sol_ref.topk_count(0.3, 10)
+    assert kk == 3 and gm[..., :kk].all() and not gm[..., kk:].any()
+
+
+def test_topk_ratio_one_is_dense_sdpa():
+    w = synth.Workload("topk_dense", B=1, H=2, N=700, D=128, grid=(67, 10, 1), n_topics=4, prefix=30, seed=25)
+    q, k, v = synth.generate(w)
+    Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
+    p, buf = parity.run_gpu(Q, K, V, 1.0, 30, 0, topk_ratio=1.0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.float().transpose(1, 2), K.float().transpose(1, 2), V.float().transpose(1, 2)).transpose(1, 2)
+    err = (buf.o.float() - ref).abs()
+    assert err.max().item() <= parity.MAX_ABS and err.mean().item() <= parity.MEAN_ABS
+
+
+@pytest.mark.slow
+def test_topk_h56_n32768_sampled():
+    w = dataclasses.replace(synth.h56_sweep(32768), name="h56_n32768_sla15", topk_ratio=0.15)
+    r = parity.full_check(w, heads=[0, 41], rows_per_head=256)
+    assert r["flips"] <= 20
+
+
+@pytest.mark.slow
+def test_topk_joint_sequence_sampled():
+    w = dataclasses.replace(synth.h56_joint(), name="h56_joint_sla15", topk_ratio=0.15)
+    r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=2)
     assert r["flips"] <= 20
