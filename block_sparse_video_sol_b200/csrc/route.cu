@@ -40,14 +40,16 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // Top-K selection for one 128-row query block i (one warp; see the file
-// comment).  Column j = lane + 32 e lives in key[e]; columns past nkb get
-// key 0, below every real score (order-preserving keys of floats are >= 1).
+// comment).  Column j = lane + 32 e lives in key[e] (E slots per lane, E*32 >=
+// nkb); columns past nkb get key 0, below every real score (order-preserving
+// keys of floats are >= 1).
+template <int E>
 __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, int i, int bh, int lane) {
   const int nkb = a.nkb, k = a.topk;
   const bool dense = i < a.n_dense;
-  uint32_t key[32];
+  uint32_t key[E];
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
+  for (int e = 0; e < E; ++e) {
     const int j = lane + 32 * e;
     const uint32_t u = j < nkb ? __float_as_uint(Sr[j]) : 0u;
     key[e] = j < nkb ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
@@ -59,19 +61,19 @@ __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, in
       const uint32_t cand = p | (1u << bit);
       int c = 0;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) c += key[e] >= cand ? 1 : 0;
+      for (int e = 0; e < E; ++e) c += key[e] >= cand ? 1 : 0;
       if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) p = cand;
     }
     int gt = 0;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) gt += key[e] > p ? 1 : 0;
+    for (int e = 0; e < E; ++e) gt += key[e] > p ? 1 : 0;
     need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
   }
   const int64_t row0 = (int64_t)bh * a.nqb + 2 * i;
   const bool second = 2 * i + 1 < a.nqb;
   int cnt = 0;
 #pragma unroll
-  for (int w = 0; w < 32; ++w) {
+  for (int w = 0; w < E; ++w) {
     if (w < a.mask_words) {   // uniform
       const bool valid = lane + 32 * w < nkb;
       const bool eq = valid && key[w] == p;
@@ -174,8 +176,11 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
     const int r = warp * (kRouteTQ / 8) + rr, i = i0 + r;
     if (i >= nrows) break;
     const float* Sr = S + r * ldS;
-    if (a.topk) {
-      topk_row(a, Sr, i, bh, lane);
+    if (a.topk) {   // the row's scores in as few register slots per lane as cover nkb
+      if (a.nkb <= 128) topk_row<4>(a, Sr, i, bh, lane);
+      else if (a.nkb <= 256) topk_row<8>(a, Sr, i, bh, lane);
+      else if (a.nkb <= 512) topk_row<16>(a, Sr, i, bh, lane);
+      else topk_row<32>(a, Sr, i, bh, lane);
       continue;
     }
     float s = 0.f;
