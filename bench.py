@@ -282,22 +282,23 @@ def run_ours(args, w):
     per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
     pool_ms, route_ms, attn_ms = per.mean(axis=0)
 
-    # e2e through the C ABI with host buffers: H2D of q, k, v + forward + D2H of o, every step
+    # e2e through the C ABI's host-buffer entry point: every step copies q, k, v from pinned host
+    # memory, runs the forward pass and copies o back (pipelined over head chunks inside the call)
     o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    staging = torch.empty(sol.sol_host_staging_bytes(p), dtype=torch.uint8, device=dev)
     h2d = 3 * q.numel() * q.element_size()
     d2h = o_host.numel() * o_host.element_size()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    sol.sol_forward_host(p, host[0], host[1], host[2], o_host, staging)   # warm-up (creates the copy streams)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
-        for dst, src in zip((q, k, v), host):
-            dst.copy_(src, non_blocking=True)
-        step()
-        o_host.copy_(buf.o, non_blocking=True)
+        sol.sol_forward_host(p, host[0], host[1], host[2], o_host, staging)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    del staging
 
     total_ms, e2e_ms, flop_all = job_reduce((total_ms, e2e_ms, flop), dev, world)
     if rank == 0:
@@ -331,7 +332,8 @@ def run_ours(args, w):
             },
             "density": float(density), "exact_flop_per_step": flop, "clocks": clocks.summary(),
             "e2e": {"value": flop_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "api": "sol_forward_host, pinned host buffers, 8-head chunks"},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:

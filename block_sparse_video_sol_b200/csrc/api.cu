@@ -375,3 +375,176 @@ extern "C" sol_status sol_route_static(const sol_params* p, const void* ws, size
   if (e != cudaSuccess) return cuda_fail(e, "sol_route_static scan/compact launch");
   return SOL_OK;
 }
+
+// ---------------------------------------------------------------------------
+// sol_forward_host: the whole forward pass on host buffers.
+//
+// Heads are independent in every stage, so the call splits them into chunks
+// of heads_per_chunk heads and pipelines them through two staging slots in
+// the caller's device buffer: the copy of chunk c+1's Q/K/V into one slot
+// (a copy-in stream) overlaps chunk c's pool/route/attention on the caller's
+// stream, which overlaps chunk c-1's O copy back to the host (a copy-out
+// stream).  Host->device and device->host copies run on different copy
+// engines, so the call takes about the time of its host->device bytes plus
+// one chunk's compute and copy-out.  Host rows are gathered with strided 2-D
+// copies (one per batch element, or per head when heads are not adjacent).
+// Results are those of sol_pool + sol_route + sol_attn_fwd on the whole
+// problem, bit for bit (every stage is per head).
+namespace sol {
+namespace {
+
+struct HostLayout {
+  sol_params cp;   // a full chunk: hc heads, compact [B, N, hc, D] strides
+  size_t q, k, v, o, ws, row_ptr, col_idx, slot;
+};
+constexpr int kHostSlots = 2;
+constexpr int kDefaultHeadsPerChunk = 8;
+
+HostLayout host_layout(const sol_params* p, int hc) {
+  HostLayout L{};
+  L.cp = *p;
+  L.cp.H = hc;
+  const int64_t rowe = (int64_t)hc * p->D;
+  L.cp.in_stride_b = L.cp.out_stride_b = (int64_t)p->N * rowe;
+  L.cp.in_stride_n = L.cp.out_stride_n = rowe;
+  L.cp.in_stride_h = L.cp.out_stride_h = p->D;
+  const size_t tb = (size_t)p->B * p->N * rowe * 2;
+  const size_t nb = (size_t)(p->N + kBlock - 1) / kBlock;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  L.q = take(tb); L.k = take(tb); L.v = take(tb); L.o = take(tb);
+  L.ws = take(ws_layout(L.cp).total);
+  L.row_ptr = take(((size_t)p->B * hc * nb + 1) * 4);
+  L.col_idx = take((size_t)p->B * hc * nb * nb * 4);
+  L.slot = off;
+  return L;
+}
+
+int heads_per_chunk(const sol_params* p, int32_t hc) {
+  return std::min(p->H, hc > 0 ? hc : kDefaultHeadsPerChunk);
+}
+
+// Per-device copy streams and events, created on first use and kept until
+// exit.  The enqueue phase of a call holds the mutex, so calls from several
+// host threads use the events one after the other.
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t entry = nullptr, ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;
+
+sol_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SOL_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  HostPipe& P = g_pipe[dev];
+  if (!P.in) {
+    const unsigned ef = cudaEventDisableTiming;
+    e = cudaStreamCreateWithFlags(&P.in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P.entry, ef);
+    for (int s = 0; s < kHostSlots && e == cudaSuccess; ++s) {
+      e = cudaEventCreateWithFlags(&P.ev_in[s], ef);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P.ev_comp[s], ef);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P.ev_out[s], ef);
+    }
+    if (e != cudaSuccess) { P.in = nullptr; return cuda_fail(e, "sol_forward_host: stream/event creation"); }
+  }
+  *out = &P;
+  return SOL_OK;
+}
+
+// Strided 2-D copy of nh heads x D of every row of B x N rows between a
+// host tensor (strides sb, sn, sh in elements) and a compact device chunk.
+cudaError_t copy_chunk(void* dev, void* host, int64_t sb, int64_t sn, int64_t sh, int B, int N, int nh, int D,
+                       int64_t rowe, bool to_dev, cudaStream_t st) {
+  const cudaMemcpyKind kind = to_dev ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost;
+  const size_t hpitch = (size_t)sn * 2, dpitch = (size_t)rowe * 2;
+  const int groups = sh == D ? 1 : nh;   // adjacent heads go in one copy
+  const size_t width = (size_t)(sh == D ? nh : 1) * D * 2;
+  for (int b = 0; b < B; ++b)
+    for (int g = 0; g < groups; ++g) {
+      char* h = static_cast<char*>(host) + ((int64_t)b * sb + (int64_t)g * sh) * 2;
+      char* d = static_cast<char*>(dev) + ((int64_t)b * N * rowe + (int64_t)g * D) * 2;
+      const cudaError_t e = to_dev ? cudaMemcpy2DAsync(d, dpitch, h, hpitch, width, N, kind, st)
+                                   : cudaMemcpy2DAsync(h, hpitch, d, dpitch, width, N, kind, st);
+      if (e != cudaSuccess) return e;
+    }
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace sol
+
+extern "C" size_t sol_host_staging_bytes(const sol_params* p, int32_t hc) {
+  if (validate(p) != SOL_OK || empty(p) || hc < 0) return 0;
+  return kHostSlots * host_layout(p, heads_per_chunk(p, hc)).slot;
+}
+
+extern "C" sol_status sol_forward_host(const sol_params* p, const void* q, const void* k, const void* v, void* o,
+                                       int32_t hc_req, void* staging, size_t staging_bytes, void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (hc_req < 0) return fail(SOL_ERR_INVALID_ARG, "sol_forward_host: heads_per_chunk must be >= 0");
+  if (!q || !k || !v || !o || !staging) return fail(SOL_ERR_INVALID_ARG, "sol_forward_host: NULL pointer");
+  if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0)
+    return fail(SOL_ERR_INVALID_ARG, "sol_forward_host: staging not 256-byte aligned");
+  const int hc = heads_per_chunk(p, hc_req);
+  const HostLayout L = host_layout(p, hc);
+  if (staging_bytes < kHostSlots * L.slot)
+    return fail(SOL_ERR_WORKSPACE, "sol_forward_host: staging %zu < %zu bytes", staging_bytes, kHostSlots * L.slot);
+  if ((s = check_arch()) != SOL_OK) return s;
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  HostPipe* P = nullptr;
+  if ((s = host_pipe(&P)) != SOL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rowe = (int64_t)hc * p->D;
+  const int chunks = (p->H + hc - 1) / hc;
+  cudaError_t e;
+  // earlier work on the caller's stream (a previous call on this staging) comes first
+  if ((e = cudaEventRecord(P->entry, st)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: event record");
+  if ((e = cudaStreamWaitEvent(P->in, P->entry, 0)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: wait");
+  for (int c = 0; c < chunks; ++c) {
+    const int slot = c % kHostSlots, h0 = c * hc, nh = std::min(hc, p->H - h0);
+    char* base = static_cast<char*>(staging) + (size_t)slot * L.slot;
+    sol_params cp = L.cp;
+    cp.H = nh;
+    // copy in (after the compute that last read this slot)
+    if (c >= kHostSlots && (e = cudaStreamWaitEvent(P->in, P->ev_comp[slot], 0)) != cudaSuccess)
+      return cuda_fail(e, "sol_forward_host: wait");
+    const void* src[3] = {q, k, v};
+    const size_t dst[3] = {L.q, L.k, L.v};
+    for (int t = 0; t < 3; ++t) {
+      e = copy_chunk(base + dst[t], const_cast<char*>(static_cast<const char*>(src[t])) + (int64_t)h0 * p->in_stride_h * 2,
+                     p->in_stride_b, p->in_stride_n, p->in_stride_h, p->B, p->N, nh, p->D, rowe, true, P->in);
+      if (e != cudaSuccess) return cuda_fail(e, "sol_forward_host: host-to-device copy");
+    }
+    if ((e = cudaEventRecord(P->ev_in[slot], P->in)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: event record");
+    // compute on the caller's stream (after the copy-out that last read this slot's O)
+    if ((e = cudaStreamWaitEvent(st, P->ev_in[slot], 0)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: wait");
+    if (c >= kHostSlots && (e = cudaStreamWaitEvent(st, P->ev_out[slot], 0)) != cudaSuccess)
+      return cuda_fail(e, "sol_forward_host: wait");
+    const size_t wsb = ws_layout(cp).total;
+    int32_t* rp = reinterpret_cast<int32_t*>(base + L.row_ptr);
+    int32_t* ci = reinterpret_cast<int32_t*>(base + L.col_idx);
+    if ((s = sol_pool(&cp, base + L.q, base + L.k, base + L.v, base + L.ws, wsb, stream)) != SOL_OK) return s;
+    if ((s = sol_route(&cp, base + L.ws, wsb, rp, ci, stream)) != SOL_OK) return s;
+    if ((s = sol_attn_fwd(&cp, base + L.q, base + L.k, base + L.v, base + L.ws, wsb, rp, ci, base + L.o, nullptr,
+                          stream)) != SOL_OK)
+      return s;
+    if ((e = cudaEventRecord(P->ev_comp[slot], st)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: event record");
+    // copy out
+    if ((e = cudaStreamWaitEvent(P->out, P->ev_comp[slot], 0)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: wait");
+    e = copy_chunk(base + L.o, static_cast<char*>(o) + (int64_t)h0 * p->out_stride_h * 2, p->out_stride_b,
+                   p->out_stride_n, p->out_stride_h, p->B, p->N, nh, p->D, rowe, false, P->out);
+    if (e != cudaSuccess) return cuda_fail(e, "sol_forward_host: device-to-host copy");
+    if ((e = cudaEventRecord(P->ev_out[slot], P->out)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: event record");
+  }
+  // the caller's stream completes only after every chunk's O is on the host
+  for (int slot = 0; slot < std::min(chunks, kHostSlots); ++slot)
+    if ((e = cudaStreamWaitEvent(st, P->ev_out[slot], 0)) != cudaSuccess) return cuda_fail(e, "sol_forward_host: wait");
+  return SOL_OK;
+}

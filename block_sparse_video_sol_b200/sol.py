@@ -24,7 +24,8 @@ SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUD
 
 # Every entry point declared in include/sol.h.
 EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
-           "sol_attn_fwd", "sol_last_device_status", "sol_status_string", "sol_last_error_text")
+           "sol_attn_fwd", "sol_forward_host", "sol_host_staging_bytes", "sol_last_device_status",
+           "sol_status_string", "sol_last_error_text")
 
 
 class sol_params(ctypes.Structure):
@@ -53,6 +54,10 @@ lib.sol_route_static.argtypes = [_P, _vp, ctypes.c_size_t, _vp, _vp, _vp]
 lib.sol_route_static.restype = ctypes.c_int
 lib.sol_attn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]
 lib.sol_attn_fwd.restype = ctypes.c_int
+lib.sol_forward_host.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp, ctypes.c_size_t, _vp]
+lib.sol_forward_host.restype = ctypes.c_int
+lib.sol_host_staging_bytes.argtypes = [_P, ctypes.c_int32]
+lib.sol_host_staging_bytes.restype = ctypes.c_size_t
 lib.sol_last_device_status.argtypes = [_vp]
 lib.sol_last_device_status.restype = ctypes.c_int
 lib.sol_status_string.argtypes = [ctypes.c_int]
@@ -149,6 +154,24 @@ def sol_route_static(p: sol_params, ws: torch.Tensor, row_ptr: torch.Tensor, col
     """Routing without caller scratch (see include/sol.h); ws may hold only the pooled part."""
     _check(lib.sol_route_static(ctypes.byref(p), _ptr(ws), ws.numel() * ws.element_size(), _ptr(row_ptr),
                                 _ptr(col_idx), _stream(stream)), "sol_route_static")
+
+
+def sol_host_staging_bytes(p: sol_params, heads_per_chunk: int = 0) -> int:
+    return lib.sol_host_staging_bytes(ctypes.byref(p), heads_per_chunk)
+
+
+def sol_forward_host(p: sol_params, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                     staging: torch.Tensor, heads_per_chunk: int = 0, stream=None):
+    """Whole forward pass on host (CPU) tensors, pipelined over head chunks (see include/sol.h).
+
+    q, k, v, o are CPU bf16 tensors (pinned for copy/compute overlap); staging is a
+    CUDA uint8 tensor of at least sol_host_staging_bytes(p, heads_per_chunk) bytes.
+    Asynchronous: synchronise the stream before reading o."""
+    for t in (q, k, v, o):
+        if t.is_cuda:
+            raise ValueError("sol_forward_host takes host tensors")
+    _check(lib.sol_forward_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), heads_per_chunk, _ptr(staging),
+                                staging.numel() * staging.element_size(), _stream(stream)), "sol_forward_host")
 
 
 def sol_attn_fwd(p: sol_params, q, k, v, ws: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,

@@ -186,6 +186,34 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
 sol_status sol_route_static(const sol_params* p, const void* ws, size_t ws_bytes,
                             int32_t* row_ptr, int32_t* col_idx, void* stream);
 
+/* sol_forward_host: pool + route + attention on HOST buffers, pipelined.
+ *   q, k, v  host pointers [B, N, H, D] bf16 with p's in_stride_*; o a host
+ *            pointer with p's out_stride_* (written: every row < N of every
+ *            head).  Pinned (page-locked) memory lets the copies overlap the
+ *            kernels; pageable memory works but the copies then serialise.
+ *   heads_per_chunk  heads per pipeline chunk; 0 picks 8 (a chunk is also
+ *            capped at H).  Must be >= 0.
+ *   staging  device buffer of staging_bytes >= sol_host_staging_bytes(p,
+ *            heads_per_chunk), 256-byte aligned, owned by the caller; two
+ *            chunk slots of compact Q, K, V, O plus each chunk's workspace
+ *            and CSR.
+ * Heads are split into chunks; chunk c+1's host-to-device copy (an internal
+ * copy-in stream), chunk c's kernels (on `stream`) and chunk c-1's O copy
+ * back (an internal copy-out stream) overlap.  The output equals that of
+ * sol_pool + sol_route + sol_attn_fwd on the whole problem bit for bit.
+ * `stream` is ordered after all of it: synchronise it (or wait on an event
+ * recorded on it) before reading o or reusing staging.  On first use per
+ * device the library creates two non-blocking streams and seven events,
+ * kept until exit; calls from several host threads enqueue one at a time.
+ * The pages describe no such entry point: it serves the end-to-end path of
+ * a caller whose tensors live in host memory. */
+sol_status sol_forward_host(const sol_params* p, const void* q, const void* k, const void* v, void* o,
+                            int32_t heads_per_chunk, void* staging, size_t staging_bytes, void* stream);
+
+/* Bytes of device staging sol_forward_host needs for p and heads_per_chunk
+ * (0 for an invalid or empty problem or a negative heads_per_chunk). */
+size_t sol_host_staging_bytes(const sol_params* p, int32_t heads_per_chunk);
+
 /* Synchronises `stream`, then reports and clears the device-side status word
  * that kernels set when a bounded wait expires (SOL_ERR_TIMEOUT) or a CSR
  * entry is out of range (SOL_ERR_INVALID_ARG). */

@@ -101,3 +101,21 @@ def test_no_gpu_reports_cuda_error(sol):
         pytest.skip("a GPU is present")
     st = _call_pool(sol, sol.make_params(1, 1000, 4, 128))
     assert st in (sol.SOL_ERR_CUDA, sol.SOL_ERR_UNSUPPORTED)
+
+
+def test_host_entry_validation(sol):
+    p = sol.make_params(1, 1000, 4, 128)
+    one = sol.lib.sol_host_staging_bytes(ctypes.byref(p), 1)
+    four = sol.lib.sol_host_staging_bytes(ctypes.byref(p), 4)
+    assert 0 < one < four
+    # a full 4-head chunk holds Q, K, V, O of the whole problem in each of two slots
+    assert four >= 2 * 4 * 1000 * 4 * 128 * 2
+    assert sol.lib.sol_host_staging_bytes(ctypes.byref(p), 0) == sol.lib.sol_host_staging_bytes(ctypes.byref(p), 8)
+    assert sol.lib.sol_host_staging_bytes(ctypes.byref(p), -1) == 0
+    h = 4096
+    assert sol.lib.sol_forward_host(ctypes.byref(p), h, h, h, h, -1, h, 1 << 40, None) == sol.SOL_ERR_INVALID_ARG
+    assert sol.lib.sol_forward_host(ctypes.byref(p), None, h, h, h, 0, h, 1 << 40, None) == sol.SOL_ERR_INVALID_ARG
+    assert sol.lib.sol_forward_host(ctypes.byref(p), h, h, h, h, 0, h + 16, 1 << 40, None) == sol.SOL_ERR_INVALID_ARG
+    assert sol.lib.sol_forward_host(ctypes.byref(p), h, h, h, h, 2, h, one, None) == sol.SOL_ERR_WORKSPACE
+    assert sol.lib.sol_forward_host(ctypes.byref(sol.make_params(0, 1000, 4, 128)), None, None, None, None, 0,
+                                    None, 0, None) == sol.SOL_OK

@@ -238,3 +238,49 @@ def test_topk_joint_sequence_sampled():
     w = dataclasses.replace(synth.h56_joint(), name="h56_joint_sla15", topk_ratio=0.15)
     r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=2)
     assert r["flips"] <= 20
+
+
+# ---------------------------------------------------------------- host-buffer entry point
+def _host_vs_device(w, heads_per_chunk, pin=True, host_view=None):
+    from block_sparse_video_sol_b200 import sol
+    q, k, v = synth.generate(w)
+    to_host = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    Qh, Kh, Vh = (to_host(x) for x in (q, k, v))
+    if host_view is not None:
+        Qh, Kh, Vh = host_view(Qh), host_view(Kh), host_view(Vh)
+    if pin:
+        Qh, Kh, Vh = (x.pin_memory() for x in (Qh, Kh, Vh))
+    B, N, H, D = Qh.shape
+    p = sol.make_params(B, N, H, D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
+                        topk_ratio=w.topk_ratio, in_strides=(Qh.stride(0), Qh.stride(1), Qh.stride(2)))
+    Oh = torch.full((B, N, H, D), float("nan"), dtype=torch.bfloat16)
+    Oh = Oh.pin_memory() if pin else Oh
+    staging = torch.empty(sol.sol_host_staging_bytes(p, heads_per_chunk), dtype=torch.uint8, device="cuda")
+    sol.sol_forward_host(p, Qh, Kh, Vh, Oh, staging, heads_per_chunk)
+    torch.cuda.synchronize()
+    sol.sol_last_device_status()
+    pd = sol.make_params(B, N, H, D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
+                         topk_ratio=w.topk_ratio)
+    buf = sol.alloc_buffers(pd, "cuda")
+    sol.forward(pd, Qh.contiguous().cuda(), Kh.contiguous().cuda(), Vh.contiguous().cuda(), buf)
+    torch.cuda.synchronize()
+    assert torch.equal(Oh, buf.o.cpu()), "host pipeline differs from the device path"
+
+
+@pytest.mark.parametrize("hc", [0, 3, 56])
+def test_host_entry_matches_device_h56(hc):
+    _host_vs_device(synth.h56_n4096(), hc)
+
+
+@pytest.mark.parametrize("mode", ["lmb", "rw", "topk"])
+def test_host_entry_modes(mode):
+    kw = dict(lmb=dict(log_mass_bias=1), rw=dict(log_mass_bias=2), topk=dict(topk_ratio=0.2))[mode]
+    w = synth.Workload("host_" + mode, B=2, H=5, N=1000, D=64, grid=(9, 10, 10), n_topics=8, prefix=100, seed=26, **kw)
+    _host_vs_device(w, 2)
+
+
+def test_host_entry_strided_and_pageable():
+    w = synth.Workload("host_strided", B=1, H=6, N=640, D=128, grid=(4, 10, 16), n_topics=8, seed=27)
+    # every other head of a 12-head host tensor: heads are not adjacent (per-head copies)
+    wide = lambda x: torch.stack([x, torch.zeros_like(x)], dim=3).reshape(1, 640, 12, 128)[:, :, 0::2]
+    _host_vs_device(w, 4, pin=False, host_view=wide)
