@@ -31,14 +31,17 @@ def _dot(x, y):
     return s
 
 
-def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=False, topk=None):
+def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=False, topk=None,
+            compressed=False):
     """Return (O[b][n][h][d], sel[b][h][i][j]) computed row by row.
 
     ``rw`` replaces the centroid key/value of every block by the anchor-softmax
     weighted summaries (and implies the log-mass bias, taken against them).
     ``topk`` (an int k) routes each query block to its k highest-scoring key
     blocks (equal scores: lower index first), keeps every key block for query
-    blocks holding prefix rows, and drops unselected blocks.
+    blocks holding prefix rows, and drops unselected blocks; with
+    ``compressed`` it also keeps the sink blocks and gives unselected blocks
+    their centroid terms (the bias options apply).
     """
     s = scale if scale else 1.0 / math.sqrt(D)
     nqb = (N + bq - 1) // bq
@@ -87,7 +90,7 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=
                     for j in range(nkb):
                         row.append(i < n_dense or j < n_sink or sc[j] > thr)
                 else:   # repeated selection of the best remaining block
-                    row = [i < n_dense] * nkb
+                    row = [i < n_dense or (compressed and j < n_sink) for j in range(nkb)]
                     left = list(range(nkb))
                     for _ in range(topk):
                         best = left[0]
@@ -105,7 +108,7 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=
                             for t in range(lo, hi):
                                 logits.append(s * _dot(q, [float(x) for x in K[b][t][h]]))
                                 vals.append([float(x) for x in V[b][t][h]])
-                        elif topk is None:
+                        elif topk is None or compressed:
                             logits.append(s * _dot(q, kc[j]) + math.log(hi - lo) + bias[j])
                             vals.append(vc[j])
                     m = max(logits)

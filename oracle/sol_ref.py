@@ -49,6 +49,13 @@ What it computes, step by step, in the order the sources describe it:
                  blocks with the largest scores s * qbar_i . kbar_j; query
                  blocks holding prefix rows keep every key block; unselected
                  blocks contribute nothing (no centroid term).
+  8. Top-K with the compressed branch (the Spark-H3 configuration:
+                 topk_mode=topk_ratio, the exact branch on the top-ranked
+                 blocks and the compressed branch on the rest; Spark-H3 news
+                 page, "Spark-Attn이 바꾸는 것" and the workflow paragraph):
+                 steps 1-6 with the threshold test of step 3 replaced by
+                 membership in the row's k highest scores; 64-row query
+                 blocks, the KV sink and the dense prefix rows as in step 3.
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -128,11 +135,14 @@ def topk_count(ratio: float, nkb: int) -> int:
     return max(1, min(nkb, math.floor(float(np.float32(ratio)) * nkb + 0.5)))
 
 
-def route_topk(S: np.ndarray, k: int, prefix: int, bq: int) -> np.ndarray:
-    """Top-K mask (step 7): the k largest scores of each row, ties to the lower index."""
+def route_topk(S: np.ndarray, k: int, prefix: int, bq: int, bk: Optional[int] = None) -> np.ndarray:
+    """Top-K mask (steps 7, 8): the k largest scores of each row, ties to the lower index;
+    with ``bk`` the key blocks holding prefix rows are kept too (the KV sink of step 8)."""
     order = np.argsort(-S, axis=-1, kind="stable")
     sel = np.zeros(S.shape, bool)
     np.put_along_axis(sel, order[..., :k], True, axis=-1)
+    if bk is not None:
+        sel[..., :, :n_blocks(prefix, bk)] = True
     sel[..., :n_blocks(prefix, bq), :] = True
     return sel
 
@@ -260,20 +270,22 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
 def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: int = 64,
                 scale: Optional[float] = None, log_mass_bias_on: bool = False,
                 mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None,
-                reweight_on: bool = False, topk_ratio: Optional[float] = None):
+                reweight_on: bool = False, topk_ratio: Optional[float] = None, compressed: bool = False):
     """The whole forward pass; returns a dict of every intermediate.
 
     ``reweight_on`` (step 6) gives the centroid terms the anchor-weighted
     summaries ``kc``/``vc`` and their bias; otherwise ``kc``/``vc`` are the
     mean-pooled kbar/vbar.  ``topk_ratio`` selects Top-K routing (step 7)
     with query blocks of ``bq`` rows (128 in the SLA contract) and no
-    centroid terms; tau and the bias options are then unused.
+    centroid terms; tau and the bias options are then unused.  With
+    ``compressed`` Top-K keeps the compressed branch (step 8): the sink, the
+    centroid terms and the bias options work as under threshold routing.
     """
     D = Q.shape[-1]
     s = (1.0 / math.sqrt(D)) if not scale else float(scale)
     qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
     S = scores(qbar, kbar, s)
-    if topk_ratio is not None:
+    if topk_ratio is not None and not compressed:
         k = topk_count(topk_ratio, kbar.shape[2])
         sel = route_topk(S, k, prefix, bq)
         bias = np.zeros(kbar.shape[:3])
@@ -281,8 +293,14 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
         O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows, centroids=False)
         return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kbar, vc=vbar, S=S, thr=None, sel=sel, k=k,
                     bias=bias, O=O, lse=lse, scale=s)
-    thr = thresholds(S, tau)
-    sel = route(S, tau, prefix, bq, bk)
+    k = None
+    if topk_ratio is not None:   # step 8
+        thr = None
+        k = topk_count(topk_ratio, kbar.shape[2])
+        sel = route_topk(S, k, prefix, bq, bk)
+    else:
+        thr = thresholds(S, tau)
+        sel = route(S, tau, prefix, bq, bk)
     kc, vc = kbar, vbar
     if reweight_on:
         kc, vc, bias = reweighted_summaries(Q, K, V, prefix, s, bk)
@@ -292,5 +310,5 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
         bias = np.zeros(kbar.shape[:3])
     used = sel if mask_override is None else mask_override
     O, lse = attention(Q, K, V, used, kc, vc, bias, s, bq, bk, rows=rows)
-    return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kc, vc=vc, S=S, thr=thr, sel=sel,
+    return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kc, vc=vc, S=S, thr=thr, sel=sel, k=k,
                 bias=bias, O=O, lse=lse, scale=s)

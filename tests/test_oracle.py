@@ -540,3 +540,63 @@ def test_planted_topk_mistakes_are_caught(monkeypatch):
                 failures += 1
         assert failures > 0, name
         monkeypatch.undo()
+
+
+# ---------------------------------------------------------------- Top-K with the compressed branch
+@pytest.mark.parametrize("seed", range(4))
+def test_topk_compressed_matches_brute_random(seed):
+    rng = np.random.default_rng(700 + seed)
+    N = int(rng.integers(17, 90))
+    bq, bk = int(rng.choice([4, 8, 16])), int(rng.choice([4, 8, 16]))
+    P = int(rng.integers(0, N // 2))
+    ratio = float(rng.choice([0.1, 0.25, 0.5]))
+    lmb, rw = [(False, False), (True, False), (False, True), (False, False)][seed]
+    Q, K, V = rand_qkv(1, N, 2, 4, seed=800 + seed)
+    o = sol_ref.sol_forward(Q, K, V, prefix=P, bq=bq, bk=bk, topk_ratio=ratio, compressed=True,
+                            log_mass_bias_on=lmb, reweight_on=rw)
+    bo, bsel = brute.forward(Q, K, V, 1, N, 2, 4, 0.0, P, bq, bk, topk=o["k"], compressed=True, lmb=lmb, rw=rw)
+    assert (o["sel"][0] == np.array(bsel[0])).all()
+    np.testing.assert_allclose(o["O"], np.array(bo), rtol=1e-11, atol=1e-12)
+
+
+def test_topk_compressed_selection_and_reductions():
+    Q, K, V = rand_qkv(1, 200, 2, 8, seed=28)
+    P, bk = 40, 16
+    nkb = -(-200 // bk)
+    o = sol_ref.sol_forward(Q, K, V, prefix=P, bq=16, bk=bk, topk_ratio=0.3, compressed=True)
+    k, n_sink, n_dense = o["k"], sol_ref.n_blocks(P, bk), sol_ref.n_blocks(P, 16)
+    cnt = o["sel"].sum(-1)[:, :, n_dense:]
+    assert (cnt >= k).all() and (cnt <= k + n_sink).all()
+    assert o["sel"][..., :n_sink].all() and o["sel"][:, :, :n_dense].all()
+    plain = sol_ref.route_topk(o["S"], k, P, 16)
+    assert (o["sel"] == (plain | (np.arange(nkb) < n_sink))).all()
+    # every block kept: dense attention; blockwise-constant K/V: dense for any k
+    full = sol_ref.sol_forward(Q, K, V, prefix=P, bq=16, bk=bk, topk_ratio=1.0, compressed=True, reweight_on=True)
+    np.testing.assert_allclose(full["O"], dense_attention(Q, K, V, 1 / math.sqrt(8)), rtol=1e-11, atol=1e-12)
+    kb = np.random.default_rng(29).standard_normal((1, nkb, 2, 8))
+    vb = np.random.default_rng(30).standard_normal((1, nkb, 2, 8))
+    Kc, Vc = np.repeat(kb, bk, axis=1)[:, :200], np.repeat(vb, bk, axis=1)[:, :200]
+    oc = sol_ref.sol_forward(Q, Kc, Vc, prefix=P, bq=16, bk=bk, topk_ratio=0.2, compressed=True)
+    np.testing.assert_allclose(oc["O"], dense_attention(Q, Kc, Vc, 1 / math.sqrt(8)), rtol=1e-11, atol=1e-12)
+
+
+def test_planted_topk_compressed_mistakes_are_caught(monkeypatch):
+    good_route, good_att = sol_ref.route_topk, sol_ref.attention
+
+    def no_sink(S, k, prefix, bq, bk=None):
+        return good_route(S, k, prefix, bq)
+
+    def drops_centroids(*args, centroids=True, **kw):
+        return good_att(*args, centroids=False, **kw)
+
+    for name, fn in [("route_topk", no_sink), ("attention", drops_centroids)]:
+        monkeypatch.setattr(sol_ref, name, fn)
+        failures = 0
+        for test in (test_topk_compressed_selection_and_reductions,
+                     lambda: test_topk_compressed_matches_brute_random(1)):
+            try:
+                test()
+            except AssertionError:
+                failures += 1
+        assert failures > 0, name
+        monkeypatch.undo()
