@@ -163,13 +163,15 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
     q, k, v = (synth.bf16_bits_to_f64(x) for x in synth.generate(w, heads=heads, b_offset=b_offset))
     t0 = time.perf_counter()
     if w.topk_ratio is not None:
-        out = sol_ref.sol_forward(q, k, v, prefix=w.prefix, bq=128, topk_ratio=w.topk_ratio)
+        out = sol_ref.sol_forward(q, k, v, prefix=w.prefix, bq=64 if w.compressed else 128,
+                                  topk_ratio=w.topk_ratio, compressed=w.compressed,
+                                  log_mass_bias_on=int(w.log_mass_bias) == 1, reweight_on=int(w.log_mass_bias) == 2)
     else:
         out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
                                   reweight_on=int(w.log_mass_bias) == 2)
     dt = time.perf_counter() - t0
     nk = sol_ref.block_rows(w.N, 64)
-    nq = sol_ref.block_rows(w.N, 128 if w.topk_ratio is not None else 64)
+    nq = sol_ref.block_rows(w.N, 128 if (w.topk_ratio is not None and not w.compressed) else 64)
     work = int(sum(((nk[None, :] * out["sel"][b, h]).sum(1) * nq).sum()
                    for b in range(w.B) for h in range(len(heads))))
     return dt, work
@@ -178,6 +180,8 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
 def routing_config(w: synth.Workload) -> dict:
     if w.topk_ratio is None:
         return {"routing": "threshold"}
+    if w.compressed:
+        return {"routing": "topk+compressed", "topk_ratio": w.topk_ratio, "q_block": 64}
     return {"routing": "topk", "topk_ratio": w.topk_ratio, "q_block": 128}
 
 
@@ -235,7 +239,7 @@ def run_ours(args, w):
                    b_offset=shard_b_offset(rank, w))
     q, k, v = (h.to(dev) for h in host)
     p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
-                        topk_ratio=w.topk_ratio)
+                        topk_ratio=w.topk_ratio, compressed=w.compressed)
     buf = sol.alloc_buffers(p, dev)
     stream = torch.cuda.current_stream()
     launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 1
@@ -308,7 +312,8 @@ def run_ours(args, w):
         attn_tf = flop / (attn_ms * 1e-3) / 1e12
         traffic, tnote = profiled_traffic("sol_attn_fwd")
         in_bytes = 3 * w.B * w.N * w.H * w.D * 2
-        pool_bytes = (2 if w.topk_ratio is not None else 3) * w.B * w.N * w.H * w.D * 2   # Top-K pools no V
+        sla = w.topk_ratio is not None and not w.compressed
+        pool_bytes = (2 if sla else 3) * w.B * w.N * w.H * w.D * 2   # the SLA variant pools no V
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -360,6 +365,8 @@ def main():
                     help="anchor-weighted key/value summaries with the log-mass bias")
     ap.add_argument("--topk-ratio", type=float, default=None,
                     help="Top-K routing (the SLA variant: 128-row query blocks, no centroid terms)")
+    ap.add_argument("--compressed", action="store_true",
+                    help="with --topk-ratio: keep the compressed branch (64-row blocks, sink, centroid terms)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
@@ -372,15 +379,18 @@ def main():
     if args.log_mass_bias and args.reweight:
         ap.error("--log-mass-bias and --reweight are exclusive")
     mode = 2 if args.reweight else int(args.log_mass_bias)
-    if args.topk_ratio is not None and (mode or args.tau is not None):
-        ap.error("--topk-ratio takes neither tau nor centroid options")
+    if args.topk_ratio is not None and (args.tau is not None or (mode and not args.compressed)):
+        ap.error("--topk-ratio takes no tau, and centroid options only with --compressed")
+    if args.compressed and args.topk_ratio is None:
+        ap.error("--compressed needs --topk-ratio")
     if args.tau is not None or mode or args.topk_ratio is not None:
         import dataclasses
         w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau, log_mass_bias=mode,
-                                topk_ratio=args.topk_ratio,
+                                topk_ratio=args.topk_ratio, compressed=args.compressed,
                                 name=w.name + (f"_tau{args.tau:g}" if args.tau is not None else "")
                                      + synth.mode_suffix(mode)
-                                     + (f"_topk{args.topk_ratio:g}" if args.topk_ratio is not None else ""))
+                                     + (f"_topk{args.topk_ratio:g}" if args.topk_ratio is not None else "")
+                                     + ("_compressed" if args.compressed else ""))
     if args.impl == "reference":
         run_reference(args, w)
     else:

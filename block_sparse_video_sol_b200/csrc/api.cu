@@ -81,16 +81,16 @@ sol_status validate(const sol_params* p) {
   if (!p) return fail(SOL_ERR_INVALID_ARG, "params is NULL");
   if (p->B < 0 || p->N < 0 || p->H <= 0) return fail(SOL_ERR_INVALID_ARG, "bad shape B=%d N=%d H=%d", p->B, p->N, p->H);
   if (p->D != 64 && p->D != 128) return fail(SOL_ERR_UNSUPPORTED, "head dim %d unsupported (64 or 128)", p->D);
-  if (p->routing != 0 && p->routing != 1) return fail(SOL_ERR_INVALID_ARG, "routing must be 0 (threshold) or 1 (top-k)");
+  if (p->routing < 0 || p->routing > 2)
+    return fail(SOL_ERR_INVALID_ARG, "routing must be 0 (threshold), 1 (top-k, SLA) or 2 (top-k, compressed branch)");
   const int want_q = p->routing == 1 ? 2 * kBlock : kBlock;
   if (p->q_block != want_q || p->k_block != kBlock)
     return fail(SOL_ERR_UNSUPPORTED, "block sizes %d/%d unsupported (routing %d takes %d/%d)", p->q_block, p->k_block,
                 p->routing, want_q, kBlock);
-  if (p->routing == 1) {
-    if (!(p->topk_ratio > 0.f && p->topk_ratio <= 1.f))
-      return fail(SOL_ERR_INVALID_ARG, "topk_ratio must lie in (0, 1]");
-    if (p->log_mass_bias != 0) return fail(SOL_ERR_INVALID_ARG, "top-k routing has no centroid terms: log_mass_bias must be 0");
-  }
+  if (p->routing != 0 && !(p->topk_ratio > 0.f && p->topk_ratio <= 1.f))
+    return fail(SOL_ERR_INVALID_ARG, "topk_ratio must lie in (0, 1]");
+  if (p->routing == 1 && p->log_mass_bias != 0)
+    return fail(SOL_ERR_INVALID_ARG, "top-k routing without the compressed branch has no centroid terms: log_mass_bias must be 0");
   if (p->routing == 0 && (isnan(p->tau) || p->tau == INFINITY))
     return fail(SOL_ERR_INVALID_ARG, "tau must be finite or -inf");
   if (!(p->scale >= 0.f) || isinf(p->scale)) return fail(SOL_ERR_INVALID_ARG, "scale must be finite and >= 0");
@@ -115,13 +115,17 @@ RouteArgs route_args(const sol_params* p, const WsLayout& L, const void* ws) {
   a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
   a.B = p->B; a.H = p->H; a.N = p->N; a.nqb = L.nqb; a.nkb = L.nkb; a.mask_words = L.mask_words;
   a.scale = eff_scale(p); a.tau = p->tau;
-  if (p->routing == 1) {   // 128-row query rows, no KV sink
+  a.topk = 0;
+  if (p->routing != 0) {
     const double kk = floor((double)p->topk_ratio * (double)L.nkb + 0.5);   // nearest, halves up
     a.topk = (int)std::max(1.0, std::min((double)L.nkb, kk));
+  }
+  if (p->routing == 1) {   // SLA: 128-row query rows, no KV sink
+    a.q128 = 1;
     a.n_sink = 0;
     a.n_dense = (p->prefix_len + 2 * kBlock - 1) / (2 * kBlock);
-  } else {
-    a.topk = 0;
+  } else {                 // threshold, or top-k with the compressed branch
+    a.q128 = 0;
     a.n_sink = (p->prefix_len + kBlock - 1) / kBlock;
     a.n_dense = a.n_sink;
   }
@@ -256,7 +260,7 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
   a.row_ptr = row_ptr; a.col_idx = col_idx;
   a.B = p->B; a.N = p->N; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb;
   a.scale = eff_scale(p);
-  a.centroids = p->routing == 0 ? 1 : 0;
+  a.centroids = p->routing == 1 ? 0 : 1;
   cudaError_t e = launch_attn(a, p->D, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sol_attn_fwd launch");
   return SOL_OK;

@@ -78,7 +78,8 @@ struct RouteArgs {
   const float* qbar; const float* kbar;
   int B, H, N, nqb, nkb, mask_words, n_sink, n_dense;   // n_dense counts the kernel's query rows
   float scale, tau;
-  int topk;                      // > 0: Top-K routing of 128-row query blocks keeping topk key blocks
+  int topk;                      // > 0: Top-K routing keeping topk key blocks (0: threshold)
+  int q128;                      // Top-K query rows are 128-row blocks (both 64-row halves share a list)
   uint32_t* mask; int32_t* counts;
 };
 

@@ -14,14 +14,15 @@
 // its 32 x nkb score rows in shared memory so that the mean, the population
 // std and the mask come from one evaluation of S.
 //
-// The same kernel does Top-K routing (the SLA variant: Star7 README, section
-// 工作原理 > SLA, Q=128 / K=64 dynamic Top-K): its query rows are then 128-row
-// blocks, whose centroid is the row-weighted mean of their two 64-row block
-// means, and a warp finds each row's k-th largest score exactly by a
-// bitwise binary search over order-preserving integer keys (32 counting
-// rounds over the row held in registers), then marks the scores above it
-// and, in index order, as many equal to it as k still needs.  Both 64-row
-// halves of a 128-row block get the same list.
+// The same kernel does Top-K routing: a warp finds each row's k-th largest
+// score exactly by a bitwise binary search over order-preserving integer
+// keys (32 counting rounds over the row held in registers), then marks the
+// scores above it and, in index order, as many equal to it as k still
+// needs.  In the SLA variant (Star7 README, section 工作原理 > SLA, Q=128 /
+// K=64 dynamic Top-K) its query rows are 128-row blocks, whose centroid is
+// the row-weighted mean of their two 64-row block means, and both 64-row
+// halves get the same list; with the compressed branch (the Spark-H3
+// configuration) rows are 64-row blocks and the KV sink is kept.
 #include <math.h>
 
 #include "common.cuh"
@@ -39,8 +40,9 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// Top-K selection for one 128-row query block i (one warp; see the file
-// comment).  Column j = lane + 32 e lives in key[e] (E slots per lane, E*32 >=
+// Top-K selection for one query row i of the kernel (a 128-row block when
+// a.q128, else a 64-row block; one warp; see the file comment); key blocks
+// below a.n_sink are kept as well.  Column j = lane + 32 e lives in key[e] (E slots per lane, E*32 >=
 // nkb); columns past nkb get key 0, below every real score (order-preserving
 // keys of floats are >= 1).
 template <int E>
@@ -69,8 +71,8 @@ __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, in
     for (int e = 0; e < E; ++e) gt += key[e] > p ? 1 : 0;
     need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
   }
-  const int64_t row0 = (int64_t)bh * a.nqb + 2 * i;
-  const bool second = 2 * i + 1 < a.nqb;
+  const int64_t row0 = (int64_t)bh * a.nqb + (a.q128 ? 2 * i : i);
+  const bool second = a.q128 && 2 * i + 1 < a.nqb;
   int cnt = 0;
 #pragma unroll
   for (int w = 0; w < E; ++w) {
@@ -79,7 +81,7 @@ __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, in
       const bool eq = valid && key[w] == p;
       const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
       const int before = __popc(eqb & ((1u << lane) - 1u));
-      const bool sel = valid && (dense || key[w] > p || (eq && before < need));
+      const bool sel = valid && (dense || lane + 32 * w < a.n_sink || key[w] > p || (eq && before < need));
       need -= __popc(eqb);
       const uint32_t bits = __ballot_sync(0xffffffffu, sel);
       if (lane == 0) {
@@ -105,13 +107,13 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   const int bh = blockIdx.y, i0 = blockIdx.x * kRouteTQ;
   const float* qbar = a.qbar + (int64_t)bh * a.nqb * D;
   const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
-  const int nrows = a.topk ? (a.nqb + 1) / 2 : a.nqb;   // the kernel's query rows
+  const int nrows = a.q128 ? (a.nqb + 1) / 2 : a.nqb;   // the kernel's query rows
 
   for (int idx = tid; idx < kRouteTQ * D; idx += 256) {
     const int r = idx % kRouteTQ, d = idx / kRouteTQ, i = i0 + r;
     float v = 0.f;
     if (i < nrows) {
-      if (a.topk) {   // 128-row block: row-weighted mean of its 64-row block means
+      if (a.q128) {   // 128-row block: row-weighted mean of its 64-row block means
         const float n0 = (float)(min(a.N, 128 * i + 64) - 128 * i);
         const float n1 = 2 * i + 1 < a.nqb ? (float)(min(a.N, 128 * i + 128) - (128 * i + 64)) : 0.f;
         const float q1 = n1 > 0.f ? qbar[(int64_t)(2 * i + 1) * D + d] : 0.f;
@@ -259,7 +261,7 @@ static size_t route_smem_bytes(int D, int ldS) {
 cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
   const int ldS = ((a.nkb + 3) / 4) * 4;
   const size_t smem = route_smem_bytes(D, ldS);
-  const int nrows = a.topk ? (a.nqb + 1) / 2 : a.nqb;
+  const int nrows = a.q128 ? (a.nqb + 1) / 2 : a.nqb;
   dim3 grid((nrows + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
   cudaError_t e;
   if (D == 128) {

@@ -80,17 +80,20 @@ def _check(status: int, where: str):
 
 def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: int = 0,
                 log_mass_bias: int = 0, scale: float = 0.0, in_strides=None, out_strides=None,
-                q_block: Optional[int] = None, k_block: int = 64, topk_ratio: Optional[float] = None) -> sol_params:
+                q_block: Optional[int] = None, k_block: int = 64, topk_ratio: Optional[float] = None,
+                compressed: bool = False) -> sol_params:
     """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D].
 
     ``log_mass_bias``: 0 (or False) mean-pooled centroids, 1 (or True) plus the
     log-mass bias, 2 anchor-weighted key/value summaries with the bias.
-    ``topk_ratio`` selects Top-K routing (128-row query blocks, unselected
-    blocks dropped); otherwise threshold routing with ``tau``.
+    ``topk_ratio`` selects Top-K routing: the SLA variant (128-row query
+    blocks, unselected blocks dropped), or with ``compressed`` the Spark-H3
+    configuration (64-row blocks, sink and centroid terms as under threshold
+    routing); otherwise threshold routing with ``tau``.
     """
-    routing = 0 if topk_ratio is None else 1
+    routing = 0 if topk_ratio is None else (2 if compressed else 1)
     if q_block is None:
-        q_block = 128 if routing else 64
+        q_block = 128 if routing == 1 else 64
     in_strides = in_strides or (N * H * D, H * D, D)
     out_strides = out_strides or (N * H * D, H * D, D)
     return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(log_mass_bias),
@@ -214,7 +217,7 @@ def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
               log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False,
-              topk_ratio: Optional[float] = None):
+              topk_ratio: Optional[float] = None, compressed: bool = False):
     """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
 
     Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.
@@ -224,7 +227,8 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.
         if t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(3) != 1 or t.stride() != q.stride():
             raise ValueError("q, k, v must be bf16 CUDA tensors with identical strides and contiguous head dim")
     p = make_params(B, N, H, D, tau, prefix_len, log_mass_bias, scale,
-                    in_strides=(q.stride(0), q.stride(1), q.stride(2)), topk_ratio=topk_ratio)
+                    in_strides=(q.stride(0), q.stride(1), q.stride(2)), topk_ratio=topk_ratio,
+                    compressed=compressed)
     buf = alloc_buffers(p, q.device, with_lse)
     forward(p, q, k, v, buf)
     return buf.o, buf

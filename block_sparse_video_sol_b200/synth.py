@@ -54,7 +54,8 @@ class Workload:
     tau: float = 1.0
     seed: int = 1000
     log_mass_bias: int = 0     # centroid mode: 0 means, 1 + log-mass bias, 2 weighted summaries
-    topk_ratio: Optional[float] = None   # Top-K routing (128-row query blocks) instead of tau
+    topk_ratio: Optional[float] = None   # Top-K routing instead of tau
+    compressed: bool = False             # Top-K keeps the compressed branch (64-row blocks, centroids)
     q_block: int = 64
     k_block: int = 64
 

@@ -91,9 +91,14 @@ typedef struct {
                                 k = round(topk_ratio * ceil(N/64)) key blocks with the largest
                                 scores (equal scores: lower index first), query blocks holding
                                 prefix rows keep every key block, unselected blocks are
-                                dropped; tau is unused and log_mass_bias must be 0.
+                                dropped; tau is unused and log_mass_bias must be 0;
+                                2: Top-K with the compressed branch (the Spark-H3
+                                configuration): as 0 with the threshold test replaced by
+                                membership in the row's k highest scores (q_block = 64, sink
+                                and dense prefix rows kept, centroid terms and every
+                                log_mass_bias mode apply; tau is unused).
                                 Other values: SOL_ERR_INVALID_ARG. */
-  float topk_ratio;          /* routing 1: fraction of key blocks kept, in (0, 1];
+  float topk_ratio;          /* routing 1, 2: fraction of key blocks kept, in (0, 1];
                                 k = floor(topk_ratio * n_kb + 0.5) in double precision from this
                                 float (nearest, halves up), clamped to [1, n_kb]. */
 } sol_params;

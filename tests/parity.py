@@ -31,12 +31,12 @@ def to_dev(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None, topk_ratio=None):
+def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None, topk_ratio=None, compressed=False):
     from block_sparse_video_sol_b200 import sol
     B, N, H, D = q.shape
     strides = in_strides or (q.stride(0), q.stride(1), q.stride(2))
     p = sol.make_params(B, N, H, D, tau=tau, prefix_len=prefix, log_mass_bias=lmb, in_strides=strides,
-                        topk_ratio=topk_ratio)
+                        topk_ratio=topk_ratio, compressed=compressed)
     buf = sol.alloc_buffers(p, q.device, with_lse=with_lse)
     sol.forward(p, q, k, v, buf)
     sol.sol_last_device_status()
@@ -100,24 +100,31 @@ def check_route(p, buf, qbar, kbar, heads, tau, prefix):
     return gm, int(((g != sel) & ~far).sum())
 
 
-def check_route_topk(p, buf, Qd, Kd, heads, ratio, prefix):
-    """Top-K mask parity outside the tie band, k per row, equal halves, CSR bit-exactness.
+def check_route_topk(p, buf, Qd, Kd, heads, ratio, prefix, compressed=False):
+    """Top-K mask parity outside the tie band, k per row (plus sinks with the
+    compressed branch), equal halves of a 128-row block (SLA), CSR bit-exactness.
 
-    Returns the GPU mask of the given heads at 128-row query-block granularity."""
+    Returns the GPU mask of the given heads at the routing's query-block granularity."""
     s = 1.0 / math.sqrt(p.D)
-    S = sol_ref.scores(sol_ref.pool(Qd, 128), sol_ref.pool(Kd, 64), s)
+    bq = 64 if compressed else 128
+    S = sol_ref.scores(sol_ref.pool(Qd, bq), sol_ref.pool(Kd, 64), s)
     nkb = S.shape[-1]
     k = sol_ref.topk_count(ratio, nkb)
-    sel = sol_ref.route_topk(S, k, prefix, 128)
+    sel = sol_ref.route_topk(S, k, prefix, bq, 64 if compressed else None)
     rp, ci, gm = gpu_mask(p, buf)
     rp_ref, ci_ref = sol_ref.to_csr(gm)
     assert np.array_equal(rp, rp_ref) and np.array_equal(ci, ci_ref)
     nqb = gm.shape[2]
-    assert (gm[:, :, 1::2] == gm[:, :, 0:nqb - nqb % 2:2]).all(), "both halves of a 128-row block share a list"
-    g = gm[:, :, ::2][:, heads]
-    n_dense = sol_ref.n_blocks(prefix, 128)
+    if compressed:
+        g = gm[:, heads]
+    else:
+        assert (gm[:, :, 1::2] == gm[:, :, 0:nqb - nqb % 2:2]).all(), "both halves of a 128-row block share a list"
+        g = gm[:, :, ::2][:, heads]
+    n_dense = sol_ref.n_blocks(prefix, bq)
+    n_sink = sol_ref.n_blocks(prefix, 64) if compressed else 0
     cnt = g.sum(-1)
-    assert (cnt[:, :, n_dense:] == k).all() and (cnt[:, :, :n_dense] == nkb).all()
+    assert (cnt[:, :, n_dense:] >= k).all() and (cnt[:, :, n_dense:] <= k + n_sink).all()
+    assert (cnt[:, :, :n_dense] == nkb).all() and g[..., :n_sink].all()
     kth = -np.sort(-S, axis=-1)[..., k - 1]
     far = np.abs(S - kth[..., None]) > BAND
     far[:, :, :n_dense] = True
@@ -126,9 +133,13 @@ def check_route_topk(p, buf, Qd, Kd, heads, ratio, prefix):
     return gm, g, int(((g != sel) & ~far).sum())
 
 
-def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None, topk_ratio=None):
+def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None, topk_ratio=None,
+                    compressed=False):
     """O (and lse) of the given heads vs the oracle run on the GPU mask."""
-    if topk_ratio is not None:
+    if topk_ratio is not None and compressed:
+        ref = sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, mask_override=gm_heads, rows=rows,
+                                  topk_ratio=topk_ratio, compressed=True, **oracle_modes(lmb))
+    elif topk_ratio is not None:
         ref = sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, bq=128, mask_override=gm_heads, rows=rows,
                                   topk_ratio=topk_ratio)
     else:
@@ -152,12 +163,13 @@ def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
     """Generate a workload, run it on the GPU, check pool/route/attention on `heads`."""
     q, k, v = synth.generate(w)
     Q, K, V = to_dev(q), to_dev(k), to_dev(v)
-    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias, topk_ratio=w.topk_ratio)
+    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias, topk_ratio=w.topk_ratio, compressed=w.compressed)
     heads = list(range(w.H)) if heads is None else list(heads)
     Qd, Kd, Vd = (synth.bf16_bits_to_f64(x[:, :, heads]) for x in (q, k, v))
-    qbar, kbar, _ = check_pool(p, buf, Qd, Kd, Vd, heads, w.log_mass_bias, w.prefix, topk=w.topk_ratio is not None)
+    sla = w.topk_ratio is not None and not w.compressed
+    qbar, kbar, _ = check_pool(p, buf, Qd, Kd, Vd, heads, w.log_mass_bias, w.prefix, topk=sla)
     if w.topk_ratio is not None:
-        _, g128, flips = check_route_topk(p, buf, Qd, Kd, heads, w.topk_ratio, w.prefix)
+        _, g128, flips = check_route_topk(p, buf, Qd, Kd, heads, w.topk_ratio, w.prefix, w.compressed)
     else:
         gm, flips = check_route(p, buf, qbar, kbar, heads, w.tau, w.prefix)
     rows = None
@@ -167,5 +179,5 @@ def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
                 for b in range(w.B) for hh in range(len(heads))}
     mask = g128 if w.topk_ratio is not None else gm[:, heads]
     errs = check_attention(p, buf, Qd, Kd, Vd, mask, heads, w.tau, w.prefix, w.log_mass_bias, rows,
-                           topk_ratio=w.topk_ratio)
+                           topk_ratio=w.topk_ratio, compressed=w.compressed)
     return dict(flips=flips, errs=errs, nnz=int(buf.row_ptr[-1].item()), p=p, buf=buf)

@@ -73,8 +73,13 @@ def test_argument_validation_is_synchronous(sol):
         assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, log_mass_bias=mode)) == sol.SOL_ERR_INVALID_ARG
         assert "log_mass_bias" in sol.lib.sol_last_error_text().decode()
     bad = sol.make_params(1, 1000, 4, 128, topk_ratio=0.2)
-    bad.routing = 2
+    bad.routing = 3
     assert _call_pool(sol, bad) == sol.SOL_ERR_INVALID_ARG
+    # top-k with the compressed branch: 64-row query blocks, every centroid mode
+    spark = lambda **kw: sol.make_params(1, 1000, 4, 128, topk_ratio=0.2, compressed=True, **kw)
+    assert spark().routing == 2 and spark().q_block == 64
+    assert _call_pool(sol, spark(q_block=128)) == sol.SOL_ERR_UNSUPPORTED
+    assert _call_pool(sol, spark(log_mass_bias=2), ws_bytes=10) == sol.SOL_ERR_WORKSPACE
     for r in (0.0, 1.5, float("nan")):
         assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=r)) == sol.SOL_ERR_INVALID_ARG
     assert _call_pool(sol, sol.make_params(1, 1000, 4, 128, topk_ratio=0.2, q_block=64)) == sol.SOL_ERR_UNSUPPORTED

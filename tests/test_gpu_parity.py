@@ -284,3 +284,34 @@ def test_host_entry_strided_and_pageable():
     # every other head of a 12-head host tensor: heads are not adjacent (per-head copies)
     wide = lambda x: torch.stack([x, torch.zeros_like(x)], dim=3).reshape(1, 640, 12, 128)[:, :, 0::2]
     _host_vs_device(w, 4, pin=False, host_view=wide)
+
+
+# ---------------------------------------------------------------- Top-K with the compressed branch (routing 2)
+@pytest.mark.parametrize("lmb", [0, 1, 2])
+def test_spark_ragged_prefix_batch2_d64(lmb):
+    w = synth.Workload("spark_ragged", B=2, H=3, N=1000, D=64, grid=(9, 10, 10), n_topics=8, prefix=100,
+                       seed=31, log_mass_bias=lmb, topk_ratio=0.2, compressed=True)
+    parity.full_check(w)
+
+
+def test_spark_d128_small_and_ties():
+    w = synth.Workload("spark_d128", B=1, H=4, N=777, D=128, grid=(4, 1, 191), n_topics=8, prefix=13,
+                       seed=32, log_mass_bias=2, topk_ratio=0.1, compressed=True)
+    parity.full_check(w)
+    for N in (1, 65):
+        parity.full_check(synth.Workload(f"spark_small{N}", B=1, H=2, N=N, D=64, grid=(1, 1, N), n_topics=2,
+                                         seed=33 + N, topk_ratio=0.5, compressed=True))
+
+
+def test_spark_h56_n8192():
+    w = dataclasses.replace(synth.h56_sweep(8192), name="h56_n8192_spark20", log_mass_bias=2, topk_ratio=0.2,
+                            compressed=True)
+    parity.full_check(w, heads=[0, 23, 55])
+
+
+@pytest.mark.slow
+def test_spark_joint_sequence_sampled():
+    w = dataclasses.replace(synth.h56_joint(), name="h56_joint_spark20", log_mass_bias=2, topk_ratio=0.2,
+                            compressed=True)
+    r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=3)
+    assert r["flips"] <= 20
