@@ -258,6 +258,7 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
   a.kbar16 = at<__nv_bfloat16>(ws, L.kbar16); a.vbar16 = at<__nv_bfloat16>(ws, L.vbar16);
   a.cbias = at<float>(ws, L.cbias);
   a.row_ptr = row_ptr; a.col_idx = col_idx;
+  a.plan = at<int>(const_cast<void*>(ws), L.plan);
   a.B = p->B; a.N = p->N; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb;
   a.scale = eff_scale(p);
   a.centroids = p->routing == 1 ? 0 : 1;

@@ -233,6 +233,87 @@ __device__ __forceinline__ void cta_sync() {
   __syncthreads();
 }
 
+// ---- plan kernel -------------------------------------------------------------------------------
+// Per query tile (two consecutive 64-row query blocks of one (b, h)): the
+// exact-block bitmaps of both blocks from their CSR lists, the union of the
+// lists with per-half tags, and the centroid tiles to visit, written to the
+// tile's plan (layout: plan_ints in common.cuh).  Building this inside the
+// attention kernel cost each CTA several microseconds at its start, with the
+// tensor cores idle (the set-up code runs once per CTA from a cold
+// instruction cache while HBM is saturated); here one warp per tile builds
+// it for all tiles at once.  Out-of-range CSR entries raise
+// SOL_ERR_INVALID_ARG and are skipped.
+constexpr int kPlanWarps = 8;
+
+__global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(const AttnArgs a, int mw) {
+  __shared__ uint32_t sel[kPlanWarps][2][kMaxWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntq = (a.nqb + 1) / 2;
+  const int64_t tile = (int64_t)blockIdx.x * kPlanWarps + warp;
+  if (tile >= (int64_t)a.B * a.H * ntq) return;   // whole warp
+  const int tq = (int)(tile % ntq);
+  const int64_t bh = tile / ntq;
+  const int i0 = 2 * tq;
+  for (int w = lane; w < 2 * kMaxWords; w += 32) (&sel[warp][0][0])[w] = 0u;
+  __syncwarp();
+  for (int hf = 0; hf < 2; ++hf) {
+    const int i = i0 + hf;
+    if (i >= a.nqb) continue;
+    const int64_t row = bh * a.nqb + i;
+    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
+    for (int e = beg + lane; e < end; e += 32) {
+      const int j = a.col_idx[e];
+      if (j >= 0 && j < a.nkb) atomicOr(&sel[warp][hf][j >> 5], 1u << (j & 31));
+      else raise_status(a.status, SOL_ERR_INVALID_ARG);
+    }
+  }
+  __syncwarp();
+  int* P = a.plan + tile * plan_ints(mw, a.nkb);
+  int* list = P + 16 + 2 * mw;
+  // Union list with per-half tags.  The S tiles take consecutive pairs of
+  // entries, and a half's exponentials are skipped for a block it does not
+  // need, so the order balances the two halves' warps: first pairs (block
+  // only A needs, block only B needs), then the blocks both need, then the
+  // leftover single-half blocks.  (The online softmax is order-free.)
+  const uint32_t ua = lane < mw ? sel[warp][0][lane] : 0u, ub = lane < mw ? sel[warp][1][lane] : 0u;
+  const uint32_t oa = ua & ~ub, ob = ub & ~ua, oc = ua & ub;
+  const int ca = __popc(oa), cb = __popc(ob), cc = __popc(oc);
+  int ia = ca, ib = cb, ic = cc;   // inclusive scans over the lanes' words
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o),
+              yc = __shfl_up_sync(0xffffffffu, ic, o);
+    if (lane >= o) { ia += ya; ib += yb; ic += yc; }
+  }
+  const int NA = __shfl_sync(0xffffffffu, ia, 31), NB = __shfl_sync(0xffffffffu, ib, 31),
+            NC = __shfl_sync(0xffffffffu, ic, 31);
+  const int npair = min(NA, NB), rest = 2 * npair + NC;   // leftovers of one kind start at rest
+  int ra = ia - ca, rb = ib - cb, rc = ic - cc;
+  for (uint32_t m = oa; m; m &= m - 1, ++ra)
+    list[ra < npair ? 2 * ra : rest + ra - npair] = (32 * lane + __ffs(m) - 1) | (1 << 16);
+  for (uint32_t m = ob; m; m &= m - 1, ++rb)
+    list[rb < npair ? 2 * rb + 1 : rest + rb - npair] = (32 * lane + __ffs(m) - 1) | (1 << 17);
+  for (uint32_t m = oc; m; m &= m - 1, ++rc)
+    list[2 * npair + rc] = (32 * lane + __ffs(m) - 1) | (3 << 16);
+  // centroid tiles (128 blocks = 4 bitmap words) holding at least one
+  // block unselected by a present half: lane w checks word w
+  const bool present1 = i0 + 1 < a.nqb;
+  const uint32_t vm = lane < mw ? (a.nkb - 32 * lane >= 32 ? 0xffffffffu : ((1u << (a.nkb - 32 * lane)) - 1u)) : 0u;
+  const uint32_t wb = __ballot_sync(0xffffffffu, ((~ua & vm) != 0u) || (present1 && (~ub & vm) != 0u));
+  if (lane < mw) {
+    P[16 + lane] = (int)ua;
+    P[16 + mw + lane] = (int)ub;
+  }
+  if (lane == 0) {
+    int n = 0;
+    for (int ct = 0; ct < 8; ++ct)
+      if ((wb >> (4 * ct)) & 0xFu) P[4 + n++] = ct;
+    P[0] = NA + NB + NC;
+    P[1] = a.centroids ? n : 0;   // Top-K routing without the compressed branch drops unselected blocks
+    P[2] = present1 ? 1 : 0;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
@@ -280,7 +361,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&x.tmem_base)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  for (int w = tid; w < 2 * kMaxWords; w += kThreads) (&x.sel[0][0])[w] = 0u;
   const int n_tail = a.N - 64 * (a.nkb - 1);   // valid rows of the last key block
   for (int c = tid; c < 64; c += kThreads) x.tail_add[c] = c < n_tail ? 0.f : -INFINITY;
   // this (b, h)'s centroid biases, needed once the lists are built: loaded now to overlap the CSR reads
@@ -292,63 +372,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 #ifdef SOL_TRACE
   if (tid == 0) SOL_GT_AT(8);
 #endif
-  for (int hf = 0; hf < 2; ++hf) {
-    const int i = i0 + hf;
-    if (i >= a.nqb) continue;
-    const int64_t row = bh * a.nqb + i;
-    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
-    for (int e = beg + tid; e < end; e += kThreads) {
-      const int j = a.col_idx[e];
-      if (j >= 0 && j < a.nkb) atomicOr(&x.sel[hf][j >> 5], 1u << (j & 31));
-      else raise_status(a.status, SOL_ERR_INVALID_ARG);
+  {   // this tile's plan (plan_kernel): header, both halves' bitmaps, the union list
+    const int* P = a.plan + ((int64_t)bh * ((a.nqb + 1) / 2) + tq) * plan_ints(mw, a.nkb);
+    const int n_plan = 16 + 2 * mw + a.nkb;
+    for (int e = tid; e < n_plan; e += kThreads) {
+      const int v = P[e];
+      if (e >= 16 + 2 * mw) x.list[e - 16 - 2 * mw] = v;
+      else if (e >= 16) x.sel[(e - 16) / mw][(e - 16) % mw] = (uint32_t)v;
+      else if (e == 0) x.n_union = v;
+      else if (e == 1) x.n_cent = v;
+      else if (e == 2) x.present[1] = v;
+      else if (e >= 4 && e < 12) x.cent[e - 4] = v;
     }
+    if (tid == 0) x.present[0] = 1;
   }
   cta_sync();
 #ifdef SOL_TRACE
   if (tid == 0) SOL_GT_AT(9);
 #endif
-  if (warp == 0) {
-    // Union list with per-half tags.  The S tiles take consecutive pairs of
-    // entries, and a half's exponentials are skipped for a block it does not
-    // need, so the order balances the two halves' warps: first pairs (block
-    // only A needs, block only B needs), then the blocks both need, then the
-    // leftover single-half blocks.  (The online softmax is order-free.)
-    const uint32_t ua = lane < mw ? x.sel[0][lane] : 0u, ub = lane < mw ? x.sel[1][lane] : 0u;
-    const uint32_t oa = ua & ~ub, ob = ub & ~ua, oc = ua & ub;
-    const int ca = __popc(oa), cb = __popc(ob), cc = __popc(oc);
-    int ia = ca, ib = cb, ic = cc;   // inclusive scans over the lanes' words
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o),
-                yc = __shfl_up_sync(0xffffffffu, ic, o);
-      if (lane >= o) { ia += ya; ib += yb; ic += yc; }
-    }
-    const int NA = __shfl_sync(0xffffffffu, ia, 31), NB = __shfl_sync(0xffffffffu, ib, 31),
-              NC = __shfl_sync(0xffffffffu, ic, 31);
-    const int npair = min(NA, NB), rest = 2 * npair + NC;   // leftovers of one kind start at rest
-    int ra = ia - ca, rb = ib - cb, rc = ic - cc;
-    for (uint32_t m = oa; m; m &= m - 1, ++ra)
-      x.list[ra < npair ? 2 * ra : rest + ra - npair] = (32 * lane + __ffs(m) - 1) | (1 << 16);
-    for (uint32_t m = ob; m; m &= m - 1, ++rb)
-      x.list[rb < npair ? 2 * rb + 1 : rest + rb - npair] = (32 * lane + __ffs(m) - 1) | (1 << 17);
-    for (uint32_t m = oc; m; m &= m - 1, ++rc)
-      x.list[2 * npair + rc] = (32 * lane + __ffs(m) - 1) | (3 << 16);
-    if (lane == 0) x.n_union = NA + NB + NC;
-    // centroid tiles (128 blocks = 4 bitmap words) holding at least one
-    // block unselected by a present half: lane w checks word w
-    const bool present1 = i0 + 1 < a.nqb;
-    const uint32_t vm = lane < mw ? (a.nkb - 32 * lane >= 32 ? 0xffffffffu : ((1u << (a.nkb - 32 * lane)) - 1u)) : 0u;
-    const uint32_t wb = __ballot_sync(0xffffffffu, ((~ua & vm) != 0u) || (present1 && (~ub & vm) != 0u));
-    if (lane == 0) {
-      x.present[0] = 1;
-      x.present[1] = present1 ? 1 : 0;
-      int n = 0;
-      for (int ct = 0; ct < 8; ++ct)
-        if ((wb >> (4 * ct)) & 0xFu) x.cent[n++] = ct;
-      x.n_cent = a.centroids ? n : 0;   // Top-K routing drops unselected blocks
-    }
-  }
-  cta_sync();
 #ifdef SOL_TRACE
   if (tid == 0) SOL_GT_AT(10);
 #endif
@@ -741,6 +782,10 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
       !make_map(&mvb, a.vbar16, 3, dims3, str3, box3, kSw128))
     return cudaErrorInvalidValue;
   TcParams prm{a, (a.nkb + 31) / 32};
+  const int64_t tiles = (int64_t)a.B * a.H * ((a.nqb + 1) / 2);
+  plan_kernel<<<(unsigned)((tiles + kPlanWarps - 1) / kPlanWarps), kPlanWarps * 32, 0, st>>>(a, prm.mask_words);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
   const size_t smem = 1024 + Cfg<D>::kSmemTiles + sizeof(Extra);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

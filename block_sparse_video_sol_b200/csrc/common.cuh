@@ -20,6 +20,12 @@ __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Ints of one query tile's attention plan (built from the CSR lists before the
+// attention kernel): a 16-int header (union length, centroid tile count,
+// whether the second query block exists, the centroid tiles), both halves'
+// exact-block bitmaps (mask_words each), then the union list (<= nkb entries).
+__host__ __device__ inline int plan_ints(int mask_words, int nkb) { return (16 + 2 * mask_words + nkb + 3) & ~3; }
+
 // Private workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
   int nqb, nkb, mask_words;
@@ -31,6 +37,7 @@ struct WsLayout {
   size_t anchor;    // fp32 [B,H,D]
   size_t mask;      // uint32 [B*H*nqb, mask_words] exact-block bitmap
   size_t counts;    // int32 [B*H*nqb]
+  size_t plan;      // int32 [B*H*ceil(nqb/2)][plan_ints]: per query tile, its attention plan
   size_t total;
 };
 
@@ -51,6 +58,7 @@ inline WsLayout ws_layout(const sol_params& p) {
   L.anchor = take(bh * p.D * 4);
   L.mask = take(bh * L.nqb * L.mask_words * 4);
   L.counts = take(bh * L.nqb * 4);
+  L.plan = take(bh * ((L.nqb + 1) / 2) * plan_ints(L.mask_words, L.nkb) * 4);
   L.total = off;
   return L;
 }
@@ -91,6 +99,7 @@ struct AttnArgs {
   float* lse;
   const __nv_bfloat16* kbar16; const __nv_bfloat16* vbar16; const float* cbias;
   const int32_t* row_ptr; const int32_t* col_idx;
+  int* plan;                     // workspace region for the per-tile plans
   int B, N, H, nqb, nkb;
   float scale;
   int centroids;                 // 1: a centroid term per unselected key block; 0: unselected blocks dropped
