@@ -242,7 +242,7 @@ def run_ours(args, w):
                         topk_ratio=w.topk_ratio, compressed=w.compressed)
     buf = sol.alloc_buffers(p, dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 1
+    launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 2   # pool (+ anchor, K/V), route + scan + compact, plan + attention
 
     def step(ev=None):
         if ev:
