@@ -787,14 +787,23 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
   const size_t smem = 1024 + Cfg<D>::kSmemTiles + sizeof(Extra);
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // Once per device (so that launches stay free of attribute calls, e.g.
+  // inside a stream capture): opt in to the shared memory, and check the
+  // register count.  The setmaxnreg split is sized for exactly kRegsLaunch
+  // registers per thread at launch; with any other count the softmax
+  // warpgroups' increase could not be granted, so refuse to launch.
+  static int prepared[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  // The setmaxnreg split is sized for exactly kRegsLaunch registers per
-  // thread at launch; with any other count the softmax warpgroups' increase
-  // could not be granted, so refuse to launch.
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>)) != cudaSuccess) return e;
-  if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+  if (dev < 0 || dev >= 64 || !prepared[dev]) {
+    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>)) != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) prepared[dev] = 1;
+  }
   dim3 grid((a.nqb + 1) / 2, a.H, a.B);
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkb, mvb, prm);
   return cudaGetLastError();

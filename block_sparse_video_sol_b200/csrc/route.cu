@@ -263,16 +263,21 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
   const size_t smem = route_smem_bytes(D, ldS);
   const int nrows = a.q128 ? (a.nqb + 1) / 2 : a.nqb;
   dim3 grid((nrows + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
-  cudaError_t e;
-  if (D == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
+  // Shared-memory opt-in once per device, for the largest problem (so that
+  // launches stay free of attribute calls, e.g. inside a stream capture).
+  static int prepared[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !prepared[dev]) {
+    const int max128 = (int)route_smem_bytes(128, kMaxKeyBlocks), max64 = (int)route_smem_bytes(64, kMaxKeyBlocks);
+    if ((e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, max128)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, max64)) != cudaSuccess)
+      return e;
+    if (dev >= 0 && dev < 64) prepared[dev] = 1;
   }
+  if (D == 128) route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
+  else route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
   return cudaGetLastError();
 }
 

@@ -315,3 +315,34 @@ def test_spark_joint_sequence_sampled():
                             compressed=True)
     r = parity.full_check(w, heads=[3, 55], rows_per_head=256, seed_rows=3)
     assert r["flips"] <= 20
+
+
+# ---------------------------------------------------------------- CUDA graphs
+@pytest.mark.parametrize("kw", [dict(), dict(log_mass_bias=2), dict(topk_ratio=0.2, compressed=True),
+                                dict(topk_ratio=0.15)])
+def test_forward_captures_into_a_cuda_graph(kw):
+    """The entry points allocate nothing and never synchronise, so one forward pass
+    captures into a CUDA graph; replays on new inputs equal eager calls bit for bit."""
+    from block_sparse_video_sol_b200 import sol
+    w = synth.Workload("graph", B=1, H=4, N=2048, D=128, grid=(2, 974, 1), n_topics=16, prefix=100, seed=34)
+    q, k, v = (parity.to_dev(x) for x in synth.generate(w))
+    p = sol.make_params(1, 2048, 4, 128, tau=1.0, prefix_len=100, **kw)
+    buf = sol.alloc_buffers(p, "cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        sol.forward(p, q, k, v, buf, stream=s)   # first call per device before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        sol.forward(p, q, k, v, buf, stream=s)
+    ref_buf = sol.alloc_buffers(p, "cuda")
+    for seed in (35, 36):
+        w2 = dataclasses.replace(w, seed=seed)
+        q2, k2, v2 = (parity.to_dev(x) for x in synth.generate(w2))
+        q.copy_(q2), k.copy_(k2), v.copy_(v2)
+        g.replay()
+        sol.forward(p, q2, k2, v2, ref_buf)
+        torch.cuda.synchronize()
+        assert torch.equal(buf.o, ref_buf.o)
+        assert torch.equal(buf.row_ptr, ref_buf.row_ptr)
+    sol.sol_last_device_status()

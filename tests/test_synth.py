@@ -51,3 +51,22 @@ def test_workload_shapes():
     assert j.N == 38247 and j.prefix == 2407 and j.N - j.prefix == 10 * 56 * 64
     assert synth.h56_sweep(32768).grid == (32, 32, 32)
     assert synth.h56_n4096().grid == (16, 16, 16)
+
+
+def test_literal_workloads_of_the_gpu_tests_are_valid():
+    """Every Workload(...) with literal arguments in the GPU tests builds (its grid covers
+    the video rows), so a mistyped case fails here rather than on a GPU."""
+    import ast
+    import os
+    src = open(os.path.join(os.path.dirname(__file__), "test_gpu_parity.py")).read()
+    n = 0
+    for node in ast.walk(ast.parse(src)):
+        if isinstance(node, ast.Call) and getattr(node.func, "attr", "") == "Workload":
+            try:
+                args = [ast.literal_eval(a) for a in node.args]
+                kw = {k.arg: ast.literal_eval(k.value) for k in node.keywords}
+            except ValueError:
+                continue   # arguments computed at run time
+            synth.Workload(*args, **kw)
+            n += 1
+    assert n >= 5
