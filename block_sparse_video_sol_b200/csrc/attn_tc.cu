@@ -17,21 +17,21 @@
 // p = 0 there (its exponentials are skipped, warp-uniformly).  Then come the
 // centroid tiles: 128 centroids each, the half's selected blocks masked.
 //
-// Roles (12 warps):
+// Roles (16 warps):
 //   warp 0     TMA producer: Q once, then the K tiles into a 3-stage ring.
 //   warp 1     MMA issuer (the whole warp; one elected lane issues):
 //              S_(t%3) = Q K^T into TMEM, then O += P V with P read from
 //              TMEM; QK runs three tiles ahead.
 //   warp 2     TMA producer: the V tiles into a 2-stage ring.
-//   warps 4-7  softmax warpgroup 0: the even S tiles t = 0, 2, 4, ...
-//   warps 8-11 softmax warpgroup 1: the odd S tiles.  One thread per row
-//              (TMEM lane), fp32 online softmax with lazy rescaling: the
-//              groups share each row's reference max (handed from step t-1
-//              to step t through an mbarrier per warp pair) and O is
-//              rescaled only when that reference grows by more than 2^8;
-//              bf16 P is written back over S.  The groups alternate, so one
-//              group's exponentials overlap the other's TMEM traffic and
-//              waits.  The epilogue normalises O and stores bf16 rows.
+//   warps 4-15 softmax warpgroups 0, 1, 2: group g takes the S tiles
+//              t = g, g+3, ... (S buffer g).  One thread per row (TMEM
+//              lane), fp32 online softmax with lazy rescaling: the groups
+//              share each row's reference max (handed from step t-1 to
+//              step t through an mbarrier per warp) and O is rescaled only
+//              when that reference grows by more than 2^8; bf16 P is
+//              written back over S.  The groups rotate, so one group's
+//              exponentials overlap the others' TMEM traffic and waits.
+//              The epilogue normalises O and stores bf16 rows.
 // TMEM: S_0, S_1, S_2 = columns [0,128), [128,256), [256,384) (P = bf16 pairs
 //       over the first 64 columns of its S), O = [384, 384+D).
 // Every mbarrier wait is bounded; on expiry the kernel raises
@@ -45,15 +45,16 @@
 namespace sol {
 namespace {
 
-constexpr int kThreads = 384;       // 12 warps: two softmax warpgroups + one control warpgroup
+constexpr int kSoftmaxGroups = 3;   // softmax warpgroups: one per S buffer
+constexpr int kThreads = 128 * (kSoftmaxGroups + 1);   // + one control warpgroup: 16 warps
 constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2;   // warp 3 idles; warps 4-11 softmax
 constexpr uint32_t kOCol = 384;     // TMEM column of O; S_0, S_1, S_2 at 0, 128, 256
 // Register split (setmaxnreg): the block launches with kRegsLaunch per
-// thread; the control warpgroup gives registers back so that the softmax
-// warpgroups can hold a whole 128-column S row.  2*128*kRegsSoftmax +
-// 128*kRegsControl must not exceed 384*kRegsLaunch.
-constexpr int kRegsLaunch = 168, kRegsSoftmax = 224, kRegsControl = 56;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch, "register split");
+// thread; the control warpgroup gives registers back to the softmax
+// warpgroups.  kSoftmaxGroups*128*kRegsSoftmax + 128*kRegsControl must not
+// exceed kThreads*kRegsLaunch.
+constexpr int kRegsLaunch = 128, kRegsSoftmax = 152, kRegsControl = 56;
+static_assert(kSoftmaxGroups * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch, "register split");
 constexpr int kKStages = 3;   // K tiles in flight (needed first, by QK)
 constexpr int kVStages = 2;   // V tiles in flight (needed a softmax later, by PV)
 // A K stage is released by the commit that signals its S buffer and a V stage
@@ -105,7 +106,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKStages], v_full[kVStages];
   uint64_t s_full[3], p_full[3], o_done[2], final_mma;
-  uint64_t ref_full[2][4];           // [group][warp]: the group's step published its reference max
+  uint64_t ref_full[kSoftmaxGroups][4];   // [group][warp]: the group's step published its reference max
 };
 
 struct Extra {
@@ -119,7 +120,7 @@ struct Extra {
   int cent_live[kMaxCentTiles][2][2];           // [slot][half][64-column half]: any live centroid
   alignas(16) float cent_add[kMaxCentTiles][2][128];        // log2-unit offset of each centroid column, -inf if masked
   alignas(16) float tail_add[64];                         // 0 for valid rows of the last key block, -inf beyond N
-  float2 ml[2][128];                            // per warpgroup and row: (reference, partial sum)
+  float2 ml[kSoftmaxGroups][128];               // per warpgroup and row: (reference, partial sum)
   float m_ref[128];                             // per row: reference max after the latest step (log2 units)
   float cbias[kMaxKeyBlocks];                   // this (b, h)'s centroid logit biases, prefetched
 #ifdef SOL_TRACE
@@ -346,7 +347,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     for (int s = 0; s < kVStages; ++s) mbar_init(&bar.v_full[s], 1);
     for (int s = 0; s < 3; ++s) { mbar_init(&bar.s_full[s], 1); mbar_init(&bar.p_full[s], 4); }
     for (int s = 0; s < 2; ++s) mbar_init(&bar.o_done[s], 1);
-    for (int g = 0; g < 2; ++g)
+    for (int g = 0; g < kSoftmaxGroups; ++g)
       for (int s = 0; s < 4; ++s) mbar_init(&bar.ref_full[g][s], 32);
     mbar_init(&bar.final_mma, 1);
     x.abort_flag = 0;
@@ -558,17 +559,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsSoftmax));
     // ---------------------------------------------------------------- softmax warpgroups
-    // Warpgroup w (warps 4w+4 .. 4w+7) takes the steps t = w, w+2, w+4, ...,
-    // one thread per row (TMEM lane), so one group exponentiates while the
-    // other waits on TMEM.  Both feed the one accumulator O, so they share
-    // each row's reference max m (log2 units): step t reads the reference
-    // left by step t-1 (the other group), raises it only when its tile's max
-    // exceeds it by more than 2^8 (lazy rescaling), publishes it at once and
-    // then exponentiates against it.  A raise rescales O after PV(t-1), the
-    // last product taken against the old reference.  Each group keeps its
-    // partial sum l_w relative to the reference of its latest step; the
-    // epilogue brings both to the final reference.
-    const int w = (warp >> 2) - 1;            // softmax warpgroup 0 or 1
+    // Warpgroup w (warps 4w+4 .. 4w+7) takes the steps t = w, w+3, w+6, ...,
+    // i.e. always S buffer w, one thread per row (TMEM lane), so the three
+    // groups' TMEM loads, exponentials and waits overlap.  All feed the one
+    // accumulator O, so they share each row's reference max m (log2 units):
+    // step t reads the reference left by step t-1 (the previous group),
+    // raises it only when its tile's max exceeds it by more than 2^8 (lazy
+    // rescaling), publishes it at once and then exponentiates against it.
+    // A raise rescales O after PV(t-1), the last product taken against the
+    // old reference.  Each group keeps its partial sum l_w relative to the
+    // reference of its latest step; the epilogue brings all to the final
+    // reference.  A thread holds half an S row at a time (the register
+    // budget of three groups), so the row max reads S once and the
+    // exponentials read it again.
+    const int w = (warp >> 2) - 1;            // softmax warpgroup 0 .. kSoftmaxGroups-1
     const int sub = warp & 3;                 // TMEM sub-partition = rows 32*sub .. 32*sub+31
     const int r = 32 * sub + lane;            // row of the tile
     const int hf = r >> 6;                    // query block half (warp-uniform)
@@ -583,8 +587,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     (void)tracer;
     float ref_w = -INFINITY, l = 0.f;         // this group's partial sum, relative to ref_w
     bool ok = true;
-    int bb = w;                               // S buffer of step t: t % 3
-    for (int t = w; t < T && ok; t += 2, bb = (bb + 2) % 3) {
+    const int bb = w;                         // S buffer of every step of this group: t % 3 = w
+    static_assert(kSoftmaxGroups == 3, "one softmax warpgroup per S buffer");
+    for (int t = w; t < T && ok; t += kSoftmaxGroups) {
 #ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(15, t);
 #endif
@@ -613,18 +618,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         add0 = x.cent_add[slot][hf];
         add1 = x.cent_add[slot][hf] + 64;
       }
-      float sv[128];
-      if (need0) { tmem_ld32(s_addr, sv); tmem_ld32(s_addr + 32, sv + 32); }
-      if (need1) { tmem_ld32(s_addr + 64, sv + 64); tmem_ld32(s_addr + 96, sv + 96); }
-      tmem_wait_ld();
-      // logits in log2 units (offset / masked) and the tile's row max; an
-      // ordinary block's scores are scaled inside the exponent instead
+      // pass 1: the tile's row max (log2 units), one 64-column half at a time;
+      // pass 2 below reloads each half for its exponentials (the register
+      // budget of three softmax warpgroups holds half a row, not a whole one)
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (!(hh ? need1 : need0)) continue;
         const float* ad = hh ? add1 : add0;
-        float* v = sv + 64 * hh;
+        float v[64];
+        tmem_ld32(s_addr + 64 * hh, v);
+        tmem_ld32(s_addr + 64 * hh + 32, v + 32);
+        tmem_wait_ld();
         if (ad) {
           const uint64_t sl22 = f2pack(sl2, sl2);
           const float4* ad4 = reinterpret_cast<const float4*>(ad);
@@ -651,7 +656,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       // the reference after step t-1, raised if this tile exceeds it by more than 2^8
       float m_prev = -INFINITY;
       if (t > 0) {
-        ok = __all_sync(0xffffffffu, wait_bar(&bar.ref_full[w ^ 1][sub], ((t - 1) >> 1) & 1, abort_flag, a.status));
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.ref_full[(w + kSoftmaxGroups - 1) % kSoftmaxGroups][sub],
+                                              ((t - 1) / kSoftmaxGroups) & 1, abort_flag, a.status));
         if (!ok) break;
         m_prev = x.m_ref[r];
       }
@@ -671,13 +677,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
         if (hh ? need1 : need0) {
-          const float mul = (hh ? add1 : add0) != nullptr ? 1.f : sl2;   // offset logits are in log2 units
+          const float* ad = hh ? add1 : add0;
+          float v[64];
+          tmem_ld32(s_addr + 64 * hh, v);
+          tmem_ld32(s_addr + 64 * hh + 32, v + 32);
+          tmem_wait_ld();
+          if (ad) {   // offset logits in log2 units, as in pass 1
+            const uint64_t sl22 = f2pack(sl2, sl2);
+            const float2* ad2 = reinterpret_cast<const float2*>(ad);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float2 o = ad2[c];
+              f2unpack(ffma2(f2pack(v[2 * c], v[2 * c + 1]), sl22, f2pack(o.x, o.y)), v[2 * c], v[2 * c + 1]);
+            }
+          }
+          const float mul = ad != nullptr ? 1.f : sl2;   // offset logits are in log2 units
           const uint64_t mul2 = f2pack(mul, mul), nb2 = f2pack(-base, -base);
           uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             float x0, x1;
-            f2unpack(ffma2(f2pack(sv[64 * hh + 2 * c], sv[64 * hh + 2 * c + 1]), mul2, nb2), x0, x1);
+            f2unpack(ffma2(f2pack(v[2 * c], v[2 * c + 1]), mul2, nb2), x0, x1);
             const float p0 = ex2(x0), p1 = ex2(x1);
             acc2[c & 1] = fadd2(acc2[c & 1], f2pack(p0, p1));
             pk[c] = pack_bf16(p0, p1);
@@ -716,23 +736,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     // epilogue: with M the final reference, O / (l_0 2^(ref_0 - M) + l_1 2^(ref_1 - M));
     // warpgroup w writes the columns [w D/2, (w+1) D/2)
 #ifdef SOL_TRACE
-    if (tracer) { SOL_TRACE_AT(12, w); SOL_GT_AT(2 + w); }
+    if (tracer && w < 2) { SOL_TRACE_AT(12, w); SOL_GT_AT(2 + w); }
 #endif
     x.ml[w][r] = make_float2(ref_w, l);
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bar.final_mma, 0, abort_flag, a.status));
-    named_bar_sync(1, 256);
+    named_bar_sync(1, 128 * kSoftmaxGroups);
     if (ok && !*abort_flag && T > 0) {
       fence_after();
       const float M = x.m_ref[r];            // written by step T-1
-      const float2 p0 = x.ml[0][r], p1 = x.ml[1][r];
-      const float L = (p0.x == -INFINITY ? 0.f : p0.y * ex2(p0.x - M)) + (p1.x == -INFINITY ? 0.f : p1.y * ex2(p1.x - M));
+      float L = 0.f;
+#pragma unroll
+      for (int g = 0; g < kSoftmaxGroups; ++g) {
+        const float2 pg = x.ml[g][r];
+        if (pg.x != -INFINITY) L += pg.y * ex2(pg.x - M);
+      }
       const float inv = L > 0.f ? 1.f / L : 0.f;
       const int grow = 64 * (i0 + hf) + (r & 63);
       const bool store = present && grow < a.N;
       __nv_bfloat16* orow = a.o + (int64_t)b * a.ob + (int64_t)h * a.oh + (int64_t)grow * a.on;
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = w * (D / 2) + 32 * c;
+      for (int c = w; c < D / 32; c += kSoftmaxGroups) {   // 32-column chunks, dealt round the groups
+        const int col = 32 * c;
         float ov[32];
         tmem_ld32(o_addr + col, ov);
         tmem_wait_ld();
@@ -749,7 +772,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     }
   }
 #ifdef SOL_TRACE
-  if (warp >= 4 && (warp & 3) == SOL_TRACE_WARP && lane == 0) { SOL_TRACE_AT(14, (warp >> 2) - 1); SOL_GT_AT(4 + (warp >> 2) - 1); }
+  if (warp >= 4 && warp < 12 && (warp & 3) == SOL_TRACE_WARP && lane == 0) { SOL_TRACE_AT(14, (warp >> 2) - 1); SOL_GT_AT(4 + (warp >> 2) - 1); }
 #endif
   fence_before();
   cta_sync();
