@@ -53,6 +53,31 @@ def exact_work(row_ptr: np.ndarray, col_idx: np.ndarray, B: int, H: int, N: int)
     return int((keys.reshape(B * H, nb) * nrows[None, :]).sum())
 
 
+def route_stats(row_ptr, col_idx, B, H, N, prefix, q128, centroids):
+    """Density over video query blocks, union waste of the attention's two-block tiles
+    (MMA work over needed work on exact tiles) and the exponentials per step."""
+    nb = -(-N // 64)
+    rows = B * H * nb
+    mask = np.zeros((rows, nb), bool)
+    cnt = np.diff(row_ptr)
+    mask[np.repeat(np.arange(rows), cnt), col_idx] = True
+    mask = mask.reshape(B * H, nb, nb)
+    n_dense = -(-prefix // (128 if q128 else 64))
+    first_video = min(nb, n_dense * (2 if q128 else 1))
+    video = mask[:, first_video:]
+    dens_video = float(video.mean()) if video.size else 0.0
+    a, b = mask[:, 0::2], mask[:, 1::2]
+    b = np.concatenate([b, np.zeros_like(a[:, :a.shape[1] - b.shape[1]])], axis=1)
+    union = (a | b).sum()
+    needed = a.sum() + b.sum()
+    nrows = np.minimum(np.arange(nb) * 64 + 64, N) - np.arange(nb) * 64   # valid rows of each block
+    exact_keys = (mask * nrows[None, None, :]).sum(-1)                    # [B*H, query block]
+    exps = int((exact_keys * nrows[None, :]).sum())
+    if centroids:   # one term per unselected key block
+        exps += int(((~mask).sum(-1) * nrows[None, :]).sum())
+    return dens_video, float(2 * union / max(needed, 1)), exps
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -257,6 +282,8 @@ def run_ours(args, w):
         if ev:
             ev[3].record()
 
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+
     for _ in range(args.warmup):
         step()
     sol.sol_last_device_status()
@@ -265,6 +292,8 @@ def run_ours(args, w):
     work = exact_work(rp, ci, w.B, w.H, w.N)
     nb = -(-w.N // 64)
     density = rp[-1] / (w.B * w.H * nb * nb)
+    sla = w.topk_ratio is not None and not w.compressed
+    dens_video, union_waste, exps = route_stats(rp, ci, w.B, w.H, w.N, w.prefix, sla, not sla)
     flop = 4.0 * w.D * work   # work is summed over every (b, h)
     cent_flop = 4.0 * w.D * w.B * w.H * w.N * nb
 
@@ -276,6 +305,8 @@ def run_ours(args, w):
     with ClockSampler(local) as clocks:
         t0.record()
         for s in range(args.steps):
+            if flush is not None:
+                flush.zero_()   # 256 MB through L2 before each step (outside the per-kernel events)
             step(evs[s])
         t1.record()
         torch.cuda.synchronize()
@@ -312,7 +343,8 @@ def run_ours(args, w):
         attn_tf = flop / (attn_ms * 1e-3) / 1e12
         traffic, tnote = profiled_traffic("sol_attn_fwd")
         in_bytes = 3 * w.B * w.N * w.H * w.D * 2
-        sla = w.topk_ratio is not None and not w.compressed
+        # route: fp32 centroids in, bitmap + counts + CSR out (not its bound: it is ALU work)
+        route_bytes = 2 * w.B * w.H * nb * w.D * 4 + w.B * w.H * nb * (4 * (-(-nb // 32)) + 8) + 4 * int(rp[-1])
         pool_bytes = (2 if sla else 3) * w.B * w.N * w.H * w.D * 2   # the SLA variant pools no V
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -322,7 +354,8 @@ def run_ours(args, w):
                        "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, **routing_config(w),
                        "global_batch": w.B * world,
                        "parallelism": f"dp{world} (one sequence per GPU)",
-                       "l2": f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB), no flush"},
+                       "l2": (f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB)"
+                              + (", 256 MB written before each step" if args.flush_l2 else ", no flush"))},
             "roofline": {"kernel": "sol_attn_fwd", "bound": "tensor", "achieved": attn_tf,
                          "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16"],
                          "peak_source": f"{peaks['source']} bf16 burst", "traffic": traffic,
@@ -331,11 +364,14 @@ def run_ours(args, w):
                 "sol_pool": {"ms": pool_ms, "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9,
                              "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm"]},
                 "sol_route": {"ms": route_ms,
-                              "TFLOP/s_fp32": 2.0 * w.B * w.H * nb * nb * w.D / (route_ms * 1e-3) / 1e12},
+                              "TFLOP/s_fp32": 2.0 * w.B * w.H * nb * nb * w.D / (route_ms * 1e-3) / 1e12,
+                              "GB/s": route_bytes / (route_ms * 1e-3) / 1e9},
                 "sol_attn_fwd": {"ms": attn_ms, "TFLOP/s_effective": attn_tf,
                                  "TFLOP/s_incl_centroids": (flop + cent_flop) / (attn_ms * 1e-3) / 1e12},
             },
-            "density": float(density), "exact_flop_per_step": flop, "clocks": clocks.summary(),
+            "density": float(density), "density_video_blocks": dens_video,
+            "union_waste": union_waste, "exponentials_per_step": exps,
+            "exact_flop_per_step": flop, "clocks": clocks.summary(),
             "e2e": {"value": flop_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "api": "sol_forward_host, pinned host buffers, 8-head chunks"},
@@ -372,6 +408,8 @@ def main():
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write 256 MB before each timed step (ms_per_step then includes it; the per-kernel times do not)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
