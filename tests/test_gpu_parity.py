@@ -139,6 +139,13 @@ def test_max_key_blocks():
     parity.full_check(w, rows_per_head=300)
 
 
+@pytest.mark.parametrize("kw", [dict(topk_ratio=0.1), dict(topk_ratio=0.1, compressed=True, log_mass_bias=2)])
+def test_max_key_blocks_topk(kw):
+    # 1024 key blocks: the Top-K selection's widest register layout (32 keys per lane)
+    w = synth.Workload("maxN_topk", B=1, H=2, N=65536, D=128, grid=(64, 32, 32), n_topics=128, seed=13, **kw)
+    parity.full_check(w, rows_per_head=300)
+
+
 def test_bad_csr_entry_is_reported_not_read():
     from block_sparse_video_sol_b200 import sol
     w = synth.tiny()

@@ -36,7 +36,12 @@ def test_rejects_problems_beyond_the_fixed_array():
 @pytest.mark.gpu
 @pytest.mark.parametrize("make", [synth.tiny, synth.h56_n4096,
                                   lambda: synth.Workload("ragged", B=2, H=3, N=1000, D=64, grid=(9, 10, 10),
-                                                         n_topics=8, prefix=100, tau=0.5, seed=7)])
+                                                         n_topics=8, prefix=100, tau=0.5, seed=7),
+                                  lambda: synth.Workload("ragged_topk", B=2, H=3, N=1000, D=64, grid=(9, 10, 10),
+                                                         n_topics=8, prefix=100, seed=7, topk_ratio=0.2),
+                                  lambda: synth.Workload("ragged_spark", B=2, H=3, N=1000, D=64, grid=(9, 10, 10),
+                                                         n_topics=8, prefix=100, seed=7, log_mass_bias=2,
+                                                         topk_ratio=0.2, compressed=True)])
 def test_static_route_matches_sol_route_twice(make):
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
@@ -44,7 +49,8 @@ def test_static_route_matches_sol_route_twice(make):
     w = make()
     q, k, v = synth.generate(w)
     Q, K, V = parity.to_dev(q), parity.to_dev(k), parity.to_dev(v)
-    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias)
+    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
+                        topk_ratio=w.topk_ratio, compressed=w.compressed)
     buf = sol.alloc_buffers(p, Q.device)
     sol.sol_pool(p, Q, K, V, buf.ws)
     sol.sol_route(p, buf.ws, buf.row_ptr, buf.col_idx)
