@@ -374,7 +374,7 @@ def run_ours(args, w):
             "exact_flop_per_step": flop, "clocks": clocks.summary(),
             "e2e": {"value": flop_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "api": "sol_forward_host, pinned host buffers, 8-head chunks"},
+                    "api": "sol_forward_host, pinned host buffers, 4-head chunks"},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -403,7 +403,7 @@ struct HostLayout {
   size_t q, k, v, o, ws, row_ptr, col_idx, slot;
 };
 constexpr int kHostSlots = 2;
-constexpr int kDefaultHeadsPerChunk = 8;
+constexpr int kDefaultHeadsPerChunk = 4;   // measured at H=56, N=32768: 27.5 ms per step against 27.8 (2), 28.5 (8), 31.6 (14)
 
 HostLayout host_layout(const sol_params* p, int hc) {
   HostLayout L{};

@@ -196,7 +196,7 @@ sol_status sol_route_static(const sol_params* p, const void* ws, size_t ws_bytes
  *            pointer with p's out_stride_* (written: every row < N of every
  *            head).  Pinned (page-locked) memory lets the copies overlap the
  *            kernels; pageable memory works but the copies then serialise.
- *   heads_per_chunk  heads per pipeline chunk; 0 picks 8 (a chunk is also
+ *   heads_per_chunk  heads per pipeline chunk; 0 picks 4 (a chunk is also
  *            capped at H).  Must be >= 0.
  *   staging  device buffer of staging_bytes >= sol_host_staging_bytes(p,
  *            heads_per_chunk), 256-byte aligned, owned by the caller; two

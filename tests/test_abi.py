@@ -117,7 +117,7 @@ def test_host_entry_validation(sol):
     assert 0 < one < four
     # a full 4-head chunk holds Q, K, V, O of the whole problem in each of two slots
     assert four >= 2 * 4 * 1000 * 4 * 128 * 2
-    assert sol.lib.sol_host_staging_bytes(ctypes.byref(p), 0) == sol.lib.sol_host_staging_bytes(ctypes.byref(p), 8)
+    assert sol.lib.sol_host_staging_bytes(ctypes.byref(p), 0) == sol.lib.sol_host_staging_bytes(ctypes.byref(p), 4)
     assert sol.lib.sol_host_staging_bytes(ctypes.byref(p), -1) == 0
     h = 4096
     assert sol.lib.sol_forward_host(ctypes.byref(p), h, h, h, h, -1, h, 1 << 40, None) == sol.SOL_ERR_INVALID_ARG
