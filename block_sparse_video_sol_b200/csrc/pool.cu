@@ -1,4 +1,5 @@
-// sol_pool kernels: block centroids of Q, K, V and the optional log-mass bias.
+// sol_pool kernels: block centroids of Q, K, V, the anchor, the optional
+// log-mass bias and the optional anchor-weighted key/value summaries.
 //
 // Block centroids ("K/V centroids") follow the Star7 README "MiniMax H3
 // Activation Chunk & Attention Acceleration", section 工作原理 > Sol; the
@@ -7,7 +8,7 @@
 // bias restores the missing mass, scored against one anchor per head (the
 // mean video query).
 //
-// The pass is HBM-bound: every input element is read exactly once.  A CTA
+// The mean pass is HBM-bound: every input element is read exactly once.  A CTA
 // owns one 64-row block of HPB heads; each thread owns one 16-byte chunk
 // (8 bf16) of one head and streams the block's rows with 8 independent
 // 16-byte loads in flight, accumulating in fp32.
