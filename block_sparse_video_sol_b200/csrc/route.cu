@@ -109,24 +109,57 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
   const int nrows = a.q128 ? (a.nqb + 1) / 2 : a.nqb;   // the kernel's query rows
 
-  for (int idx = tid; idx < kRouteTQ * D; idx += 256) {
-    const int r = idx % kRouteTQ, d = idx / kRouteTQ, i = i0 + r;
-    float v = 0.f;
-    if (i < nrows) {
-      if (a.q128) {   // 128-row block: row-weighted mean of its 64-row block means
-        const float n0 = (float)(min(a.N, 128 * i + 64) - 128 * i);
-        const float n1 = 2 * i + 1 < a.nqb ? (float)(min(a.N, 128 * i + 128) - (128 * i + 64)) : 0.f;
-        const float q1 = n1 > 0.f ? qbar[(int64_t)(2 * i + 1) * D + d] : 0.f;
-        v = (n0 * qbar[(int64_t)(2 * i) * D + d] + n1 * q1) / (n0 + n1);
-      } else {
-        v = qbar[(int64_t)i * D + d];
+  // Stage q transposed: lane = query row, one float4 of head dims per load;
+  // every thread issues all its loads before its first store.
+  constexpr int kQv = kRouteTQ * D / 4 / 256;
+  {
+    float4 qv[kQv];
+#pragma unroll
+    for (int u = 0; u < kQv; ++u) {
+      const int idx = tid + 256 * u, r = idx % kRouteTQ, d = 4 * (idx / kRouteTQ), i = i0 + r;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < nrows) {
+        if (a.q128) {   // 128-row block: row-weighted mean of its 64-row block means
+          const float n0 = (float)(min(a.N, 128 * i + 64) - 128 * i);
+          const float n1 = 2 * i + 1 < a.nqb ? (float)(min(a.N, 128 * i + 128) - (128 * i + 64)) : 0.f;
+          const float4 q0 = *reinterpret_cast<const float4*>(qbar + (int64_t)(2 * i) * D + d);
+          float4 q1 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (n1 > 0.f) q1 = *reinterpret_cast<const float4*>(qbar + (int64_t)(2 * i + 1) * D + d);
+          const float n = n0 + n1;
+          v = make_float4((n0 * q0.x + n1 * q1.x) / n, (n0 * q0.y + n1 * q1.y) / n,
+                          (n0 * q0.z + n1 * q1.z) / n, (n0 * q0.w + n1 * q1.w) / n);
+        } else {
+          v = *reinterpret_cast<const float4*>(qbar + (int64_t)i * D + d);
+        }
       }
+      qv[u] = v;
     }
-    qT[d * kRouteTQ + r] = v;
+#pragma unroll
+    for (int u = 0; u < kQv; ++u) {
+      const int idx = tid + 256 * u, r = idx % kRouteTQ, d = 4 * (idx / kRouteTQ);
+      qT[(d + 0) * kRouteTQ + r] = qv[u].x;
+      qT[(d + 1) * kRouteTQ + r] = qv[u].y;
+      qT[(d + 2) * kRouteTQ + r] = qv[u].z;
+      qT[(d + 3) * kRouteTQ + r] = qv[u].w;
+    }
   }
   const int rg = warp & 3;   // rows 8*rg .. 8*rg+7
   const int chh = warp >> 2; // columns 128*chh .. +127 of the chunk
 
+  // k slices (kRouteCH key blocks x kRouteDS head dims) are software-pipelined
+  // through registers: the next slice's loads are issued before the current
+  // slice's FMAs, so their latency hides behind the arithmetic.
+  constexpr int kKv = kRouteCH * kRouteDS / 4 / 256;
+  float4 kn[kKv];
+  auto load_slice = [&](int c0, int d0) {
+#pragma unroll
+    for (int u = 0; u < kKv; ++u) {
+      const int idx = tid + 256 * u, jj = idx / (kRouteDS / 4), dq = (idx % (kRouteDS / 4)) * 4;
+      kn[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + jj < a.nkb) kn[u] = *reinterpret_cast<const float4*>(kbar + (int64_t)(c0 + jj) * D + d0 + dq);
+    }
+  };
+  load_slice(0, 0);
   for (int c0 = 0; c0 < a.nkb; c0 += kRouteCH) {
     float acc[8][4];
 #pragma unroll
@@ -136,17 +169,21 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
     for (int d0 = 0; d0 < D; d0 += kRouteDS) {
       __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
       __syncthreads();
-      for (int idx = tid; idx < kRouteCH * (kRouteDS / 4); idx += 256) {
-        const int jj = idx / (kRouteDS / 4), dq = (idx % (kRouteDS / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c0 + jj < a.nkb) v = *reinterpret_cast<const float4*>(kbar + (int64_t)(c0 + jj) * D + d0 + dq);
-        kT[(dq + 0) * kRouteLdK + jj] = v.x;
-        kT[(dq + 1) * kRouteLdK + jj] = v.y;
-        kT[(dq + 2) * kRouteLdK + jj] = v.z;
-        kT[(dq + 3) * kRouteLdK + jj] = v.w;
+#pragma unroll
+      for (int u = 0; u < kKv; ++u) {
+        const int idx = tid + 256 * u, jj = idx / (kRouteDS / 4), dq = (idx % (kRouteDS / 4)) * 4;
+        kT[(dq + 0) * kRouteLdK + jj] = kn[u].x;
+        kT[(dq + 1) * kRouteLdK + jj] = kn[u].y;
+        kT[(dq + 2) * kRouteLdK + jj] = kn[u].z;
+        kT[(dq + 3) * kRouteLdK + jj] = kn[u].w;
       }
       __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
       __syncthreads();
+      {   // the next slice: next head-dim slice, else the next chunk's first
+        const int nd0 = d0 + kRouteDS < D ? d0 + kRouteDS : 0;
+        const int nc0 = d0 + kRouteDS < D ? c0 : c0 + kRouteCH;
+        if (nc0 < a.nkb) load_slice(nc0, nd0);
+      }
 #pragma unroll 4
       for (int dd = 0; dd < kRouteDS; ++dd) {
         const float4 qa = *reinterpret_cast<const float4*>(qT + (d0 + dd) * kRouteTQ + 8 * rg);
