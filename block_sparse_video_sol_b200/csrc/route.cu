@@ -26,6 +26,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace sol {
 
@@ -161,11 +162,13 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   };
   load_slice(0, 0);
   for (int c0 = 0; c0 < a.nkb; c0 += kRouteCH) {
-    float acc[8][4];
+    // acc[p][c]: rows 8*rg + 2p (low half) and 2p+1 (high half) of column c,
+    // updated by one packed f32x2 FMA (each half an ordinary fp32 FMA)
+    uint64_t acc[4][4];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int p = 0; p < 4; ++p)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+      for (int c = 0; c < 4; ++c) acc[p][c] = 0ull;
     for (int d0 = 0; d0 < D; d0 += kRouteDS) {
       __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
       __syncthreads();
@@ -184,26 +187,34 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
         const int nc0 = d0 + kRouteDS < D ? c0 : c0 + kRouteCH;
         if (nc0 < a.nkb) load_slice(nc0, nd0);
       }
-#pragma unroll 4
+#pragma unroll
       for (int dd = 0; dd < kRouteDS; ++dd) {
         const float4 qa = *reinterpret_cast<const float4*>(qT + (d0 + dd) * kRouteTQ + 8 * rg);
         const float4 qb = *reinterpret_cast<const float4*>(qT + (d0 + dd) * kRouteTQ + 8 * rg + 4);
-        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-        float kv[4];
+        const uint64_t q2[4] = {f2pack(qa.x, qa.y), f2pack(qa.z, qa.w), f2pack(qb.x, qb.y), f2pack(qb.z, qb.w)};
+        uint64_t k2[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) kv[c] = kT[dd * kRouteLdK + 128 * chh + lane + 32 * c];
+        for (int c = 0; c < 4; ++c) {
+          const float kv = kT[dd * kRouteLdK + 128 * chh + lane + 32 * c];
+          k2[c] = f2pack(kv, kv);
+        }
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int p = 0; p < 4; ++p)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(qv[r], kv[c], acc[r][c]);
+          for (int c = 0; c < 4; ++c) acc[p][c] = ffma2(q2[p], k2[c], acc[p][c]);
       }
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int p = 0; p < 4; ++p)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int col = c0 + 128 * chh + lane + 32 * c;
-        if (col < a.nkb) S[(8 * rg + r) * ldS + col] = a.scale * acc[r][c];
+        float lo, hi;
+        f2unpack(acc[p][c], lo, hi);
+        if (col < a.nkb) {
+          S[(8 * rg + 2 * p) * ldS + col] = a.scale * lo;
+          S[(8 * rg + 2 * p + 1) * ldS + col] = a.scale * hi;
+        }
       }
   }
   __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
