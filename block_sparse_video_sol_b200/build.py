@@ -40,22 +40,29 @@ def _deps():
         os.path.join(ROOT, "include", "sol.h"), os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(OUT):
+FAULT_OUT = os.path.join(PKG, "libsol_fault.so")
+
+
+def up_to_date(out: str = OUT) -> bool:
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, trace: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, trace: bool = False,
+          fault_test: bool = False) -> str:
     """Compile csrc/*.cu for sm_100a and link libsol.so; returns its path.
 
     ``trace`` builds a separate libsol_trace.so with the attention kernel's
     phase trace compiled in (for pipeline analysis; not used by the product).
+    ``fault_test`` builds libsol_fault.so (SOL_FAULT_TEST: short wait limits
+    and the withheld-arrive hook of sol_debug_drop_arrive), which the tests of
+    the device-side timeout path load in a child process.
     """
-    out = OUT if not trace else os.path.join(PKG, "libsol_trace.so")
-    if not force and not trace and up_to_date():
-        return OUT
+    out = os.path.join(PKG, "libsol_trace.so") if trace else FAULT_OUT if fault_test else OUT
+    if not force and not trace and up_to_date(out):
+        return out
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
@@ -63,9 +70,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
         extra.append("-DSOL_TRACE")
         if os.environ.get("SOL_TRACE_WARP"):
             extra.append("-DSOL_TRACE_WARP=" + os.environ["SOL_TRACE_WARP"])
+    if fault_test:
+        extra.append("-DSOL_FAULT_TEST")
+    suffix = ".trace.o" if trace else ".fault.o" if fault_test else ".o"
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + (".trace.o" if trace else ".o"))
+        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + suffix)
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -91,4 +101,4 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas" in sys.argv,
-                trace="--trace" in sys.argv))
+                trace="--trace" in sys.argv, fault_test="--fault-test" in sys.argv))

@@ -280,6 +280,20 @@ sol_status sol_last_device_status(void* stream) {
   return fail((sol_status)v, "device status: %s", sol_status_string((sol_status)v));
 }
 
+sol_status sol_debug_drop_arrive(int32_t step) {
+#ifdef SOL_FAULT_TEST
+  sol_status s = check_arch();
+  if (s != SOL_OK) return s;
+  if (step < -1) return fail(SOL_ERR_INVALID_ARG, "sol_debug_drop_arrive: step %d < -1", (int)step);
+  const cudaError_t e = sol::set_drop_p_arrive(step);
+  if (e != cudaSuccess) return cuda_fail(e, "sol_debug_drop_arrive");
+  return SOL_OK;
+#else
+  (void)step;
+  return fail(SOL_ERR_UNSUPPORTED, "sol_debug_drop_arrive: this library was built without SOL_FAULT_TEST");
+#endif
+}
+
 const char* sol_status_string(sol_status s) {
   switch (s) {
     case SOL_OK: return "SOL_OK";

@@ -45,6 +45,10 @@
 namespace sol {
 namespace {
 
+#ifdef SOL_FAULT_TEST
+__device__ int g_drop_p_arrive = -1;   // step whose "P ready" arrive is withheld (-1: none)
+#endif
+
 constexpr int kSoftmaxGroups = 3;   // softmax warpgroups: one per S buffer
 constexpr int kThreads = 128 * (kSoftmaxGroups + 1);   // + one control warpgroup: 16 warps
 constexpr int kKWarp = 0, kMmaWarp = 1, kVWarp = 2;   // warp 3 idles; warps 4-11 softmax
@@ -731,7 +735,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       if (tracer) SOL_TRACE_AT(3, t);
       if (lane == 0) SOL_TRACE_AT(16 + sub, t);
 #endif
+#ifdef SOL_FAULT_TEST
+      // fault-test build: the arrive of step g_drop_p_arrive is withheld, so the
+      // MMA warp's bounded wait for P(t) expires (sol_debug_drop_arrive)
+      if (lane == 0 && t != g_drop_p_arrive) mbar_arrive(&bar.p_full[bb]);
+#else
       if (lane == 0) mbar_arrive(&bar.p_full[bb]);
+#endif
     }
     // epilogue: with M the final reference, O / (l_0 2^(ref_0 - M) + l_1 2^(ref_1 - M));
     // warpgroup w writes the columns [w D/2, (w+1) D/2)
@@ -837,6 +847,12 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
 cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st) {
   return D == 128 ? launch_tc<128>(a, st) : launch_tc<64>(a, st);
 }
+
+#ifdef SOL_FAULT_TEST
+cudaError_t set_drop_p_arrive(int step) {
+  return cudaMemcpyToSymbol(g_drop_p_arrive, &step, sizeof(int));
+}
+#endif
 
 }  // namespace sol
 

@@ -115,5 +115,8 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st);
 cudaError_t launch_scan_compact(const uint32_t* mask, const int32_t* counts, int rows, int mask_words,
                                 int32_t* row_ptr, int32_t* col_idx, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st);
+#ifdef SOL_FAULT_TEST
+cudaError_t set_drop_p_arrive(int step);   // fault-test build only
+#endif
 
 }  // namespace sol

@@ -12,7 +12,13 @@
 
 namespace sol {
 
+#ifdef SOL_FAULT_TEST
+// The fault-test build (libsol_fault.so): a short limit, so that a withheld
+// arrive expires within milliseconds.
+constexpr uint32_t kSpinLimit = 1u << 16;
+#else
 constexpr uint32_t kSpinLimit = 1u << 22;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 

@@ -25,7 +25,7 @@ SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUD
 # Every entry point declared in include/sol.h.
 EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
            "sol_attn_fwd", "sol_forward_host", "sol_host_staging_bytes", "sol_last_device_status",
-           "sol_status_string", "sol_last_error_text")
+           "sol_status_string", "sol_last_error_text", "sol_debug_drop_arrive")
 
 
 class sol_params(ctypes.Structure):
@@ -64,6 +64,8 @@ lib.sol_status_string.argtypes = [ctypes.c_int]
 lib.sol_status_string.restype = ctypes.c_char_p
 lib.sol_last_error_text.argtypes = []
 lib.sol_last_error_text.restype = ctypes.c_char_p
+lib.sol_debug_drop_arrive.argtypes = [ctypes.c_int32]
+lib.sol_debug_drop_arrive.restype = ctypes.c_int
 
 
 class SolError(RuntimeError):
@@ -185,6 +187,12 @@ def sol_attn_fwd(p: sol_params, q, k, v, ws: torch.Tensor, row_ptr: torch.Tensor
 
 def sol_last_device_status(stream=None):
     _check(lib.sol_last_device_status(_stream(stream)), "device status")
+
+
+def sol_debug_drop_arrive(step: int):
+    """Fault-test library only: withhold the attention's "P ready" arrive of S
+    tile `step` in every CTA (-1: none), so that its bounded wait expires."""
+    _check(lib.sol_debug_drop_arrive(step), "sol_debug_drop_arrive")
 
 
 @dataclass

@@ -224,6 +224,19 @@ size_t sol_host_staging_bytes(const sol_params* p, int32_t heads_per_chunk);
  * entry is out of range (SOL_ERR_INVALID_ARG). */
 sol_status sol_last_device_status(void* stream);
 
+/* Fault injection for testing the bounded waits (the device-side failure
+ * path).  Only a library built with SOL_FAULT_TEST (libsol_fault.so, whose
+ * waits expire after 2^16 polls instead of 2^22) acts on it: from the next
+ * sol_attn_fwd on, every CTA's softmax withholds its "P ready" arrive of
+ * step `step` (0-based S tile; -1 restores normal operation), so the MMA
+ * warp's bounded wait expires.  That launch then stops issuing, drains its
+ * copies and MMAs, frees its tensor memory, writes no output and leaves
+ * SOL_ERR_TIMEOUT in the device status word; the context stays usable.
+ * Synchronous (a symbol copy), not for use while kernels run.  Returns
+ * SOL_ERR_INVALID_ARG for step < -1; the product library returns
+ * SOL_ERR_UNSUPPORTED and changes nothing. */
+sol_status sol_debug_drop_arrive(int32_t step);
+
 /* Static, human-readable name of a status code. */
 const char* sol_status_string(sol_status s);
 

@@ -36,6 +36,18 @@ def test_every_declared_symbol_is_exported(sol):
     assert declared == set(sol.EXPORTS)
 
 
+def test_fault_hook_is_inert_in_the_product_library(sol):
+    assert sol.lib.sol_debug_drop_arrive(0) == sol.SOL_ERR_UNSUPPORTED
+    assert "SOL_FAULT_TEST" in sol.lib.sol_last_error_text().decode()
+
+
+def test_fault_test_library_builds_and_exports_the_same_entry_points(sol):
+    from block_sparse_video_sol_b200 import build
+    fault = ctypes.CDLL(build.build(fault_test=True))
+    for name in sol.EXPORTS:
+        assert hasattr(fault, name), name
+
+
 def test_status_strings(sol):
     for code, name in enumerate(["SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_WORKSPACE",
                                  "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT"]):
