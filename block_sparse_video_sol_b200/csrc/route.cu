@@ -16,7 +16,8 @@
 //
 // The same kernel does Top-K routing: a warp finds each row's k-th largest
 // score exactly by a bitwise binary search over order-preserving integer
-// keys (32 counting rounds over the row held in registers), then marks the
+// keys (counting rounds over the row held in registers, at most 32: it stops
+// once exactly k keys lie at or above the candidate), then marks the
 // scores above it and, in index order, as many equal to it as k still
 // needs.  In the SLA variant (Star7 README, section 工作原理 > SLA, Q=128 /
 // K=64 dynamic Top-K) its query rows are 128-row blocks, whose centroid is
@@ -59,18 +60,27 @@ __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, in
   }
   uint32_t p = 0u;   // the k-th largest key: the largest v with #{key >= v} >= k
   int need = 0;      // how many keys equal to p are still to be taken
+  bool all_eq = false;   // every key equal to p is taken
   if (!dense) {      // uniform over the warp
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = p | (1u << bit);
       int c = 0;
 #pragma unroll
       for (int e = 0; e < E; ++e) c += key[e] >= cand ? 1 : 0;
-      if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) p = cand;
+      const int tot = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+      if (tot >= k) {
+        p = cand;
+        // exactly k keys >= cand: they are the k largest and the next one is
+        // smaller, so {key >= cand} is the selection and no tie is left to break
+        if (tot == k) { all_eq = true; break; }
+      }
     }
-    int gt = 0;
+    if (!all_eq) {
+      int gt = 0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) gt += key[e] > p ? 1 : 0;
-    need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+      for (int e = 0; e < E; ++e) gt += key[e] > p ? 1 : 0;
+      need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+    }
   }
   const int64_t row0 = (int64_t)bh * a.nqb + (a.q128 ? 2 * i : i);
   const bool second = a.q128 && 2 * i + 1 < a.nqb;
@@ -82,7 +92,7 @@ __device__ __forceinline__ void topk_row(const RouteArgs& a, const float* Sr, in
       const bool eq = valid && key[w] == p;
       const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
       const int before = __popc(eqb & ((1u << lane) - 1u));
-      const bool sel = valid && (dense || lane + 32 * w < a.n_sink || key[w] > p || (eq && before < need));
+      const bool sel = valid && (dense || lane + 32 * w < a.n_sink || key[w] > p || (eq && (all_eq || before < need)));
       need -= __popc(eqb);
       const uint32_t bits = __ballot_sync(0xffffffffu, sel);
       if (lane == 0) {
