@@ -39,6 +39,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -825,17 +827,17 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   // register count.  The setmaxnreg split is sized for exactly kRegsLaunch
   // registers per thread at launch; with any other count the softmax
   // warpgroups' increase could not be granted, so refuse to launch.
-  static int prepared[64];
+  static std::atomic<int> prepared[64];   // zero-initialised; set once per device (any thread)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !prepared[dev]) {
+  if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>)) != cudaSuccess) return e;
     if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-    if (dev >= 0 && dev < 64) prepared[dev] = 1;
+    if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
   dim3 grid((a.nqb + 1) / 2, a.H, a.B);
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkb, mvb, prm);

@@ -26,6 +26,8 @@
 // configuration) rows are 64-row blocks and the KV sink is kept.
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -323,16 +325,16 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
   dim3 grid((nrows + kRouteTQ - 1) / kRouteTQ, a.B * a.H);
   // Shared-memory opt-in once per device, for the largest problem (so that
   // launches stay free of attribute calls, e.g. inside a stream capture).
-  static int prepared[64];
+  static std::atomic<int> prepared[64];   // zero-initialised; set once per device (any thread)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !prepared[dev]) {
+  if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
     const int max128 = (int)route_smem_bytes(128, kMaxKeyBlocks), max64 = (int)route_smem_bytes(64, kMaxKeyBlocks);
     if ((e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, max128)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, max64)) != cudaSuccess)
       return e;
-    if (dev >= 0 && dev < 64) prepared[dev] = 1;
+    if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
   if (D == 128) route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
   else route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
