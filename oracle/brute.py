@@ -118,3 +118,85 @@ def forward(Q, K, V, B, N, H, D, tau, prefix, bq, bk, scale=None, lmb=False, rw=
                         O[b][r][h][c] = sum(wi * vi[c] for wi, vi in zip(w, vals)) / z
             SEL[b][h] = sel_bh
     return O, SEL
+
+
+# ---- adaptive partition (Spark-H3 news page, Spark-Reblock bullet), scalar form ----------------
+def _cholesky(M, D):
+    """Textbook Cholesky-Banachiewicz: lower L with L L^T = M."""
+    L = [[0.0] * D for _ in range(D)]
+    for i in range(D):
+        for j in range(i + 1):
+            s = M[i][j]
+            for c in range(j):
+                s -= L[i][c] * L[j][c]
+            L[i][j] = math.sqrt(s) if i == j else s / L[j][j]
+    return L
+
+
+def reblock_perm(Q, K, B, N, H, D, prefix, bs=64, iters=4):
+    """perm[b][h][pos] of the size-balanced principal-axis bisection of the keys
+    whitened by the video queries' second moment (ridge 1e-4 * trace / D).
+
+    Level by level over explicit group lists (the oracle recurses); the same
+    reading: split along the covariance's principal axis by ``iters`` power
+    steps from the group's first member minus its mean, the left part takes
+    bs * ceil(ceil(n / bs) / 2) lowest projections (ties to the lower row),
+    groups keep ascending row order, prefix blocks stay in place.
+    """
+    n_fix = min(N, bs * (-(-prefix // bs)))
+    perm = [[list(range(N)) for _ in range(H)] for _ in range(B)]
+    if n_fix == N:
+        return perm
+    lo = prefix if prefix < N else 0
+    for b in range(B):
+        for h in range(H):
+            M = [[0.0] * D for _ in range(D)]
+            for t in range(lo, N):
+                q = [float(Q[b][t][h][c]) for c in range(D)]
+                for i in range(D):
+                    for j in range(D):
+                        M[i][j] += q[i] * q[j]
+            n = N - lo
+            tr = 0.0
+            for i in range(D):
+                for j in range(D):
+                    M[i][j] /= n
+                tr += M[i][i]
+            ridge = 1e-4 * tr / D if tr > 0 else 1.0
+            for i in range(D):
+                M[i][i] += ridge
+            L = _cholesky(M, D)
+            Y = []
+            for t in range(n_fix, N):
+                k = [float(K[b][t][h][c]) for c in range(D)]
+                x = [sum(k[r] * L[r][c] for r in range(D)) for c in range(D)]   # row k times L
+                nx = math.sqrt(_dot(x, x))
+                Y.append([v / nx for v in x] if nx > 0 else [0.0] * D)
+            groups = [list(range(N - n_fix))]
+            while any(len(g) > bs for g in groups):
+                nxt = []
+                for g in groups:
+                    if len(g) <= bs:
+                        nxt.append(g)
+                        continue
+                    m = len(g)
+                    left = bs * (-(-(-(-m // bs)) // 2))
+                    mean = [sum(Y[t][c] for t in g) / m for c in range(D)]
+                    C = [[Y[t][c] - mean[c] for c in range(D)] for t in g]
+                    w = list(C[0])
+                    nw = math.sqrt(_dot(w, w))
+                    w = [v / nw for v in w] if nw > 0 else [1.0] + [0.0] * (D - 1)
+                    for _ in range(iters):
+                        proj = [_dot(c, w) for c in C]
+                        z = [sum(C[r][c] * proj[r] for r in range(m)) for c in range(D)]
+                        nz = math.sqrt(_dot(z, z))
+                        if nz == 0:
+                            break
+                        w = [v / nz for v in z]
+                    ranked = sorted(range(m), key=lambda r: (_dot(Y[g[r]], w), g[r]))
+                    in_left = set(ranked[:left])
+                    nxt.append([g[r] for r in range(m) if r in in_left])
+                    nxt.append([g[r] for r in range(m) if r not in in_left])
+                groups = nxt
+            perm[b][h] = list(range(n_fix)) + [n_fix + t for g in groups for t in g]
+    return perm

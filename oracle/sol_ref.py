@@ -56,6 +56,26 @@ What it computes, step by step, in the order the sources describe it:
                  steps 1-6 with the threshold test of step 3 replaced by
                  membership in the row's k highest scores; 64-row query
                  blocks, the KV sink and the dense prefix rows as in step 3.
+  9. adaptive partition (optional; Spark-H3 news page, Spark-Reblock
+                 bullet: fixed tiles replaced by an adaptive partition whose
+                 similarity is the cosine under the Mahalanobis metric of the
+                 opposite side's second moment, split hierarchically until
+                 every leaf has the block size, in O(N log N); workflow
+                 paragraph: reblock_layout=q_reuse_k, queries take the keys'
+                 partition).  Reading: per (b, h) the keys are whitened by the
+                 Cholesky factor of the video queries' second moment
+                 M = mean q q^T (plus a ridge of 1e-4 * trace(M) / D), so the
+                 plain cosine of the whitened unit vectors is the Mahalanobis
+                 cosine; a group splits along its principal axis (REBLOCK_ITERS
+                 power-iteration steps on its covariance, started from its
+                 first member minus its mean) at the size-balanced median:
+                 the left part takes 64 * ceil(ceil(n / 64) / 2) rows, the
+                 lowest projections, ties to the lower row index; every group
+                 keeps its rows in ascending original order, so the partial
+                 leaf is last and each leaf lists its rows ascending.  Blocks
+                 holding prefix rows keep their place.  Q, K and V are
+                 permuted per head, steps 1-8 run on the permuted rows, and O
+                 is permuted back.
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -267,10 +287,103 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
     return O, lse
 
 
+REBLOCK_ITERS = 4   # power-iteration steps per split (step 9)
+
+
+def second_moment_whitener(Q: np.ndarray, prefix: int) -> np.ndarray:
+    """Lower Cholesky factors L[b, h] of the video queries' second moment
+    M = mean q q^T + 1e-4 * trace(M) / D * I (step 9), so that
+    (k L) . (k' L) = k^T M k'."""
+    B, N, H, D = Q.shape
+    rows = Q[:, prefix:, :, :] if prefix < N else Q
+    L = np.empty((B, H, D, D))
+    for b in range(B):
+        for h in range(H):
+            X = rows[b, :, h, :]
+            M = X.T @ X / X.shape[0]
+            tr = np.trace(M)
+            M = M + (1e-4 * tr / D if tr > 0 else 1.0) * np.eye(D)
+            L[b, h] = np.linalg.cholesky(M)
+    return L
+
+
+def _split_group(Y: np.ndarray, members: np.ndarray, bs: int, iters: int, leaves: list):
+    """Recursive size-balanced principal-axis bisection (step 9); ``members``
+    ascending positions into Y (the whitened unit vectors)."""
+    n = len(members)
+    if n <= bs:
+        leaves.append(members)
+        return
+    left = bs * (-(-(-(-n // bs)) // 2))   # bs * ceil(ceil(n / bs) / 2)
+    X = Y[members]
+    C = X - X.mean(axis=0)
+    w = C[0].copy()
+    nw = np.linalg.norm(w)
+    if nw > 0:
+        w /= nw
+    else:
+        w = np.zeros(Y.shape[1])
+        w[0] = 1.0
+    for _ in range(iters):
+        z = C.T @ (C @ w)
+        nz = np.linalg.norm(z)
+        if nz == 0:
+            break
+        w = z / nz
+    p = X @ w
+    order = np.lexsort((members, p))       # ascending projection, ties to the lower row
+    go_left = np.zeros(n, dtype=bool)
+    go_left[order[:left]] = True
+    _split_group(Y, members[go_left], bs, iters, leaves)    # boolean selection keeps ascending order
+    _split_group(Y, members[~go_left], bs, iters, leaves)
+
+
+def reblock_partition(Q: np.ndarray, K: np.ndarray, prefix: int, bs: int = 64,
+                      iters: int = REBLOCK_ITERS) -> np.ndarray:
+    """perm[b, h, pos] = original row at position ``pos`` of the adaptive
+    partition's order (step 9); blocks holding prefix rows stay in place."""
+    B, N, H, D = K.shape
+    n_fix = min(N, bs * n_blocks(prefix, bs))
+    perm = np.tile(np.arange(N, dtype=np.int64), (B, H, 1))
+    if N - n_fix == 0:
+        return perm
+    L = second_moment_whitener(Q, prefix)
+    for b in range(B):
+        for h in range(H):
+            Xw = K[b, n_fix:, h, :] @ L[b, h]
+            nrm = np.linalg.norm(Xw, axis=1, keepdims=True)
+            Y = np.divide(Xw, nrm, out=np.zeros_like(Xw), where=nrm > 0)
+            leaves: list = []
+            _split_group(Y, np.arange(N - n_fix), bs, iters, leaves)
+            perm[b, h, n_fix:] = n_fix + np.concatenate(leaves)
+    return perm
+
+
+def permute_rows(X: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Xp[b, pos, h] = X[b, perm[b, h, pos], h] for X [B, N, H, ...]."""
+    B, N, H = X.shape[:3]
+    out = np.empty_like(X)
+    for b in range(B):
+        for h in range(H):
+            out[b, :, h] = X[b, perm[b, h], h]
+    return out
+
+
+def unpermute_rows(Xp: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Inverse of ``permute_rows``: X[b, perm[b, h, pos], h] = Xp[b, pos, h]."""
+    B, N, H = Xp.shape[:3]
+    out = np.empty_like(Xp)
+    for b in range(B):
+        for h in range(H):
+            out[b, perm[b, h], h] = Xp[b, :, h]
+    return out
+
+
 def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: int = 64,
                 scale: Optional[float] = None, log_mass_bias_on: bool = False,
                 mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None,
-                reweight_on: bool = False, topk_ratio: Optional[float] = None, compressed: bool = False):
+                reweight_on: bool = False, topk_ratio: Optional[float] = None, compressed: bool = False,
+                reblock: bool = False, perm_override: Optional[np.ndarray] = None):
     """The whole forward pass; returns a dict of every intermediate.
 
     ``reweight_on`` (step 6) gives the centroid terms the anchor-weighted
@@ -280,7 +393,22 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
     centroid terms; tau and the bias options are then unused.  With
     ``compressed`` Top-K keeps the compressed branch (step 8): the sink, the
     centroid terms and the bias options work as under threshold routing.
+    ``reblock`` (step 9) runs all of it on the rows permuted per head by the
+    adaptive partition (``perm_override`` replaces the computed order) and
+    returns O and the LSE in the original row order; the block
+    intermediates, ``mask_override`` and ``rows`` refer to permuted rows.
     """
+    if reblock:
+        perm = reblock_partition(Q, K, prefix, bk) if perm_override is None else perm_override
+        r = sol_forward(permute_rows(Q, perm), permute_rows(K, perm), permute_rows(V, perm), tau, prefix,
+                        bq, bk, scale, log_mass_bias_on, mask_override, rows, reweight_on, topk_ratio,
+                        compressed)
+        r["O_permuted"], r["perm"] = r["O"], perm
+        r["O"] = unpermute_rows(r["O"], perm)
+        lse = r["lse"]   # [B, H, N]
+        r["lse"] = np.stack([np.stack([lse[b, h][np.argsort(perm[b, h])] for h in range(lse.shape[1])])
+                             for b in range(lse.shape[0])])
+        return r
     D = Q.shape[-1]
     s = (1.0 / math.sqrt(D)) if not scale else float(scale)
     qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
