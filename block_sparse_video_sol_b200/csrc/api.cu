@@ -280,6 +280,98 @@ sol_status sol_last_device_status(void* stream) {
   return fail((sol_status)v, "device status: %s", sol_status_string((sol_status)v));
 }
 
+// ---- adaptive partition (Spark-Reblock reading) and row gathers ------------------------------
+namespace {
+struct ReblockLayout {
+  int n_fix, n_v, q_lo, n_q, mchunks;
+  size_t mpart, L, Y, ord, tmp, key, total;
+};
+ReblockLayout reblock_layout(const sol_params& p) {
+  ReblockLayout R{};
+  const int nsink = (p.prefix_len + kBlock - 1) / kBlock;
+  R.n_fix = std::min(p.N, kBlock * nsink);
+  R.n_v = p.N - R.n_fix;
+  R.q_lo = p.prefix_len < p.N ? p.prefix_len : 0;   // the video query rows (all rows if none)
+  R.n_q = p.N - R.q_lo;
+  R.mchunks = R.n_q > 0 ? reblock_moment_chunks(R.n_q) : 0;
+  const size_t bh = (size_t)p.B * p.H, D = p.D;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  R.mpart = take(bh * R.mchunks * D * D * 4);
+  R.L = take(bh * D * D * 4);
+  R.Y = take(bh * R.n_v * D * 4);
+  R.ord = take(bh * R.n_v * 4);
+  R.tmp = take(bh * R.n_v * 4);
+  R.key = take(bh * R.n_v * 8);
+  R.total = R.n_v > 0 ? off : 0;
+  return R;
+}
+constexpr int kReblockIters = 4;   // power steps per split
+}  // namespace
+
+size_t sol_reblock_workspace_bytes(const sol_params* p) {
+  if (validate(p) != SOL_OK || empty(p)) return 0;
+  return reblock_layout(*p).total;
+}
+
+sol_status sol_reblock(const sol_params* p, const void* q, const void* k, void* ws, size_t ws_bytes, int32_t* perm,
+                       void* stream) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!q || !k || !perm) return fail(SOL_ERR_INVALID_ARG, "sol_reblock: NULL pointer");
+  if (!aligned16(q) || !aligned16(k)) return fail(SOL_ERR_INVALID_ARG, "sol_reblock: q/k not 16-byte aligned");
+  const ReblockLayout R = reblock_layout(*p);
+  if (R.total > 0) {
+    if (!ws) return fail(SOL_ERR_INVALID_ARG, "sol_reblock: NULL workspace");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+      return fail(SOL_ERR_INVALID_ARG, "sol_reblock: workspace not 256-byte aligned");
+    if (ws_bytes < R.total) return fail(SOL_ERR_WORKSPACE, "sol_reblock: workspace %zu < %zu bytes", ws_bytes, R.total);
+  }
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
+  ReblockArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.sb = p->in_stride_b; a.sn = p->in_stride_n; a.sh = p->in_stride_h;
+  a.B = p->B; a.H = p->H; a.N = p->N; a.D = p->D;
+  a.n_fix = R.n_fix; a.n_v = R.n_v; a.q_lo = R.q_lo; a.n_q = R.n_q; a.mchunks = R.mchunks;
+  if (R.total > 0) {
+    a.mpart = at<float>(ws, R.mpart); a.L = at<float>(ws, R.L); a.Y = at<float>(ws, R.Y);
+    a.ord = at<int32_t>(ws, R.ord); a.tmp = at<int32_t>(ws, R.tmp); a.key = at<uint64_t>(ws, R.key);
+  }
+  a.perm = perm;
+  a.status = status;
+  const cudaError_t e = launch_reblock(a, kReblockIters, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sol_reblock launch");
+  return SOL_OK;
+}
+
+static sol_status rows_entry(const sol_params* p, const int32_t* perm, const void* src, void* dst, bool gather,
+                             void* stream, const char* name) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (empty(p)) return SOL_OK;
+  if (!perm || !src || !dst) return fail(SOL_ERR_INVALID_ARG, "%s: NULL pointer", name);
+  if (!aligned16(src) || !aligned16(dst)) return fail(SOL_ERR_INVALID_ARG, "%s: tensors not 16-byte aligned", name);
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
+  const int64_t sb = gather ? p->in_stride_b : p->out_stride_b, sn = gather ? p->in_stride_n : p->out_stride_n,
+                sh = gather ? p->in_stride_h : p->out_stride_h;
+  const cudaError_t e = launch_rows(perm, static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), p->B,
+                                    p->H, p->N, p->D, sb, sn, sh, gather, status, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return SOL_OK;
+}
+
+sol_status sol_gather_rows(const sol_params* p, const int32_t* perm, const void* x, void* xp, void* stream) {
+  return rows_entry(p, perm, x, xp, true, stream, "sol_gather_rows");
+}
+
+sol_status sol_scatter_rows(const sol_params* p, const int32_t* perm, const void* xp, void* x, void* stream) {
+  return rows_entry(p, perm, xp, x, false, stream, "sol_scatter_rows");
+}
+
 sol_status sol_debug_drop_arrive(int32_t step) {
 #ifdef SOL_FAULT_TEST
   sol_status s = check_arch();

@@ -115,6 +115,30 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st);
 cudaError_t launch_scan_compact(const uint32_t* mask, const int32_t* counts, int rows, int mask_words,
                                 int32_t* row_ptr, int32_t* col_idx, cudaStream_t st);
 cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st);
+
+// Adaptive partition (sol_reblock).  Workspace pieces are caller-owned.
+struct ReblockArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  int64_t sb, sn, sh;            // element strides of q and k
+  int B, H, N, D;
+  int n_fix, n_v;                // rows kept in place (prefix blocks); rows partitioned
+  int q_lo, n_q;                 // video query rows [q_lo, q_lo + n_q) of the second moment
+  int mchunks;                   // partial-moment chunks per head
+  float* mpart;                  // [B*H][mchunks][D][D]
+  float* L;                      // [B*H][D][D] lower Cholesky factor
+  float* Y;                      // [B*H][n_v][D] whitened unit keys
+  int32_t* ord;                  // [B*H][n_v] current order (indices into the partitioned rows)
+  int32_t* tmp;                  // [B*H][n_v]
+  uint64_t* key;                 // [B*H][n_v] split keys
+  int32_t* perm;                 // [B*H][N] output: original row at each position
+  int* status;
+};
+int reblock_levels(int n_v);
+int reblock_moment_chunks(int n_q);
+cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st);
+cudaError_t launch_rows(const int32_t* perm, const __nv_bfloat16* src, __nv_bfloat16* dst, int B, int H, int N, int D,
+                        int64_t sb, int64_t sn, int64_t sh, bool gather, int* status, cudaStream_t st);
 #ifdef SOL_FAULT_TEST
 cudaError_t set_drop_p_arrive(int step);   // fault-test build only
 #endif

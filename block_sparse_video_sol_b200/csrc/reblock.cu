@@ -1,0 +1,519 @@
+// sol_reblock kernels: the adaptive partition of the keys and the row
+// gathers / scatters around the unchanged Sol kernels.
+//
+// Spark-H3 news page, Spark-Reblock bullet: the fixed tiles are replaced by
+// an adaptive partition; two rows are similar when their score patterns
+// against the other side are, measured by the cosine under the Mahalanobis
+// metric of the opposite side's second moment; a hierarchical splitter
+// divides groups until every leaf has the block size.  The workflow
+// paragraph fixes reblock_layout=q_reuse_k: queries take the keys' order.
+//
+// Reading (the same as the oracle's): per (b, h)
+//   M  = mean of q q^T over the video query rows, + 1e-4 trace(M) / D * I;
+//   y_t = normalise(k_t L), L the lower Cholesky factor of M, for the key rows
+//        past the prefix blocks (which stay in place), so y.y' is the
+//        Mahalanobis cosine;
+//   a group of n > 64 rows splits along its principal axis (REBLOCK_ITERS
+//        power steps on its covariance, started from its first row minus its
+//        mean): the 64 * ceil(ceil(n / 64) / 2) rows of lowest projection
+//        (ties to the lower row) go left, the rest right, each part keeping
+//        ascending row order; so the partial leaf is last and every leaf
+//        lists its rows ascending.
+//
+// Kernels, in launch order:
+//   rb_moment_kernel  -- partial sums of q q^T over 2048-row chunks (fp32);
+//   rb_factor_kernel  -- one CTA per head: the partials summed in a fixed
+//                        order, the ridge, the Cholesky factor in shared memory;
+//   rb_whiten_kernel  -- y = normalise(k L) for 64 rows per CTA, and the
+//                        initial (identity) order;
+//   rb_split_kernel   -- one launch per level of the hierarchy, one CTA per
+//                        group: mean, power steps, projections as 64-bit keys
+//                        (order-preserving float bits, row index), the split
+//                        rank found by an 8-pass radix select, then a stable
+//                        partition of the group's rows;
+//   rb_perm_kernel    -- perm[pos] = original row at position pos;
+//   gather / scatter  -- rows of a BTHD tensor into / out of a head-major
+//                        [B, H, N, D] copy in the partition's order.
+//
+// Every reduction runs in a fixed order, so the partition is deterministic.
+#include <math.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace sol {
+
+namespace {
+
+constexpr int kMomRows = 2048;       // query rows per partial-moment CTA
+constexpr int kMomStage = 32;        // rows staged in shared memory at a time
+constexpr int kSplitThreads = 1024;  // threads of a split CTA
+constexpr int kSplitWarps = kSplitThreads / 32;
+constexpr int kSplitUnroll = 4;      // rows in flight per row slot
+
+__host__ __device__ inline int rb_left(int n) { return kBlock * ((((n + kBlock - 1) / kBlock) + 1) / 2); }
+
+// Group s of level lvl (its bits, most significant first, choose left / right
+// at each level above): start and length in the video rows' order; false if
+// an ancestor is already a leaf.
+__device__ inline bool rb_segment(int n_v, int lvl, int s, int& start, int& len) {
+  start = 0;
+  len = n_v;
+  for (int l = lvl - 1; l >= 0; --l) {
+    if (len <= kBlock) return false;
+    const int left = rb_left(len);
+    if ((s >> l) & 1) { start += left; len -= left; } else { len = left; }
+  }
+  return true;
+}
+
+__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// Partial second moment of the video query rows: grid (chunks, B*H).
+template <int D>
+__global__ void __launch_bounds__(256) rb_moment_kernel(const ReblockArgs a) {
+  constexpr int TS = D / 16;   // each thread owns a TS x TS tile of the D x D moment
+  __shared__ __align__(16) float xs[kMomStage][D];
+  const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int r0 = a.q_lo + blockIdx.x * kMomRows, r1 = min(a.q_lo + a.n_q, r0 + kMomRows);
+  const __nv_bfloat16* qb = a.q + (int64_t)b * a.sb + (int64_t)h * a.sh;
+  float acc[TS][TS];
+#pragma unroll
+  for (int i = 0; i < TS; ++i)
+#pragma unroll
+    for (int j = 0; j < TS; ++j) acc[i][j] = 0.f;
+  for (int s0 = r0; s0 < r1; s0 += kMomStage) {
+    __syncthreads();
+    for (int idx = tid; idx < kMomStage * (D / 4); idx += 256) {
+      const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4, row = s0 + r;
+      const float4 v = row < r1 ? ld_bf16x4(qb + (int64_t)row * a.sn + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(&xs[r][c4]) = v;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < kMomStage; ++r) {
+      float u[TS], w[TS];
+#pragma unroll
+      for (int i = 0; i < TS; i += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(&xs[r][ti * TS + i]);
+        const float4 y = *reinterpret_cast<const float4*>(&xs[r][tj * TS + i]);
+        u[i] = x.x; u[i + 1] = x.y; u[i + 2] = x.z; u[i + 3] = x.w;
+        w[i] = y.x; w[i + 1] = y.y; w[i + 2] = y.z; w[i + 3] = y.w;
+      }
+#pragma unroll
+      for (int i = 0; i < TS; ++i)
+#pragma unroll
+        for (int j = 0; j < TS; ++j) acc[i][j] = fmaf(u[i], w[j], acc[i][j]);
+    }
+  }
+  float* out = a.mpart + ((int64_t)bh * a.mchunks + blockIdx.x) * D * D;
+#pragma unroll
+  for (int i = 0; i < TS; ++i)
+#pragma unroll
+    for (int j = 0; j < TS; ++j) out[(ti * TS + i) * D + tj * TS + j] = acc[i][j];
+}
+
+// M = (sum of the partials, chunk order) / n_q + ridge; its lower Cholesky
+// factor L (left-looking, one column at a time): one CTA per (b, h).
+template <int D>
+__global__ void __launch_bounds__(256) rb_factor_kernel(const ReblockArgs a) {
+  constexpr int LD = D + 1;                    // padded rows: column reads hit distinct banks
+  extern __shared__ __align__(16) float M[];   // [D][LD]
+  __shared__ float s_ridge;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, bh = blockIdx.x;
+  const float* part = a.mpart + (int64_t)bh * a.mchunks * D * D;
+  const float inv_n = 1.f / (float)a.n_q;
+  for (int idx = tid; idx < D * D; idx += 256) {
+    float s = 0.f;
+    for (int c = 0; c < a.mchunks; ++c) s += part[(int64_t)c * D * D + idx];
+    M[(idx / D) * LD + idx % D] = s * inv_n;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float t = 0.f;
+    for (int i = lane; i < D; i += 32) t += M[i * LD + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) s_ridge = t > 0.f ? 1e-4f * t / (float)D : 1.f;
+  }
+  __syncthreads();
+  if (tid < D) M[tid * LD + tid] += s_ridge;
+  __syncthreads();
+  for (int j = 0; j < D; ++j) {
+    if (warp == 0) {   // diagonal: M[j][j] - sum_c<j L[j][c]^2, lanes strided, fixed-order tree
+      float t = 0.f;
+      for (int c = lane; c < j; c += 32) t = fmaf(M[j * LD + c], M[j * LD + c], t);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) {
+        float d = M[j * LD + j] - t;
+        if (!(d > 0.f)) d = s_ridge;   // cannot happen with the ridge; keeps L finite
+        M[j * LD + j] = sqrtf(d);
+      }
+    }
+    __syncthreads();
+    const float ljj = M[j * LD + j];
+    for (int i = j + 1 + tid; i < D; i += 256) {
+      float t = M[i * LD + j];
+      for (int c = 0; c < j; ++c) t = fmaf(-M[i * LD + c], M[j * LD + c], t);
+      M[i * LD + j] = t / ljj;
+    }
+    __syncthreads();
+  }
+  float* L = a.L + (int64_t)bh * D * D;
+  for (int idx = tid; idx < D * D; idx += 256) L[idx] = (idx % D) <= (idx / D) ? M[(idx / D) * LD + idx % D] : 0.f;
+}
+
+// y = normalise(k L) for 64 video key rows per CTA: grid (ceil(n_v/64), B*H).
+template <int D>
+__global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
+  constexpr int LK = D + 4;   // padded key rows (16-byte aligned, rows on distinct banks)
+  extern __shared__ __align__(16) float sm[];
+  float* Ls = sm;             // [D][D]
+  float* ks = sm + D * D;     // [64][LK]
+  __shared__ float s_inv[kBlock];
+  const int tid = threadIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t0 = blockIdx.x * kBlock;
+  const float* Lg = a.L + (int64_t)bh * D * D;
+  for (int idx = tid * 4; idx < D * D; idx += 256 * 4)
+    *reinterpret_cast<float4*>(&Ls[idx]) = *reinterpret_cast<const float4*>(&Lg[idx]);
+  const __nv_bfloat16* kb = a.k + (int64_t)b * a.sb + (int64_t)h * a.sh;
+  for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
+    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4, t = t0 + r;
+    const float4 v = t < a.n_v ? ld_bf16x4(kb + (int64_t)(a.n_fix + t) * a.sn + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(&ks[r * LK + c4]) = v;
+  }
+  __syncthreads();
+  // thread (r = tid / 4, cg = tid % 4) computes columns cg + 4u of row r
+  const int r = tid >> 2, cg = tid & 3;
+  float y[D / 4];
+#pragma unroll
+  for (int u = 0; u < D / 4; ++u) y[u] = 0.f;
+  for (int i = 0; i < D; ++i) {
+    const float kv = ks[r * LK + i];
+#pragma unroll
+    for (int u = 0; u < D / 4; ++u) y[u] = fmaf(kv, Ls[i * D + cg + 4 * u], y[u]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < D / 4; ++u) ss = fmaf(y[u], y[u], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  if (cg == 0) s_inv[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+  __syncthreads();   // every thread has read ks
+  const float inv = s_inv[r];
+#pragma unroll
+  for (int u = 0; u < D / 4; ++u) ks[r * LK + cg + 4 * u] = y[u] * inv;
+  __syncthreads();
+  float* Yg = a.Y + ((int64_t)bh * a.n_v + t0) * D;
+  for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
+    const int rr = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    if (t0 + rr < a.n_v) *reinterpret_cast<float4*>(&Yg[(int64_t)rr * D + c4]) = *reinterpret_cast<const float4*>(&ks[rr * LK + c4]);
+  }
+  if (tid < kBlock && t0 + tid < a.n_v) a.ord[(int64_t)bh * a.n_v + t0 + tid] = t0 + tid;
+}
+
+// Sum of a per-lane float4 over the CTA's row slots into out[D] (fixed order).
+template <int D>
+__device__ __forceinline__ void rb_block_sum(float4 v, float4 (*red)[D / 4], float* out, float scale) {
+  constexpr int LPR = D / 4, RPW = 32 / LPR;   // lanes per row, rows per warp
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (RPW == 2) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
+    v.z += __shfl_xor_sync(0xffffffffu, v.z, 16);
+    v.w += __shfl_xor_sync(0xffffffffu, v.w, 16);
+  }
+  if (lane < LPR) red[warp][lane] = v;
+  __syncthreads();
+  if (threadIdx.x < LPR) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < kSplitWarps; ++w) {
+      const float4 t = red[w][threadIdx.x];
+      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+    }
+    out[4 * threadIdx.x + 0] = s.x * scale;
+    out[4 * threadIdx.x + 1] = s.y * scale;
+    out[4 * threadIdx.x + 2] = s.z * scale;
+    out[4 * threadIdx.x + 3] = s.w * scale;
+  }
+  __syncthreads();
+}
+
+// Dot product of a row's lane quad with x over the row's lanes (all of them get it).
+template <int D>
+__device__ __forceinline__ float rb_row_dot(float4 y, float4 x) {
+  float t = y.x * x.x;
+  t = fmaf(y.y, x.y, t);
+  t = fmaf(y.z, x.z, t);
+  t = fmaf(y.w, x.w, t);
+#pragma unroll
+  for (int o = D / 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
+}
+
+__device__ __forceinline__ float rb_norm(const float* v, int D, float* s_tmp) {
+  // single-warp fixed-order norm of v[D], broadcast through shared memory
+  if (threadIdx.x < 32) {
+    float t = 0.f;
+    for (int i = threadIdx.x; i < D; i += 32) t = fmaf(v[i], v[i], t);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) *s_tmp = sqrtf(t);
+  }
+  __syncthreads();
+  const float n = *s_tmp;
+  __syncthreads();
+  return n;
+}
+
+// One level of the hierarchy: grid (2^lvl, B*H); group blockIdx.x of every head.
+template <int D>
+__global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockArgs a, int lvl, int iters) {
+  constexpr int LPR = D / 4, RPW = 32 / LPR, SLOTS = kSplitWarps * RPW;
+  __shared__ __align__(16) float4 red[kSplitWarps][LPR];
+  __shared__ __align__(16) float mean[D], w[D], z[D];
+  __shared__ uint32_t hist[256];
+  __shared__ int s_int[4];
+  __shared__ float s_tmp;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane / LPR, fl = lane % LPR;   // row slot within the warp, lane quad of the row
+  const int bh = blockIdx.y;
+  int start, len;
+  if (!rb_segment(a.n_v, lvl, blockIdx.x, start, len) || len <= kBlock) return;
+  const int left = rb_left(len);
+  int32_t* ord = a.ord + (int64_t)bh * a.n_v + start;
+  const float* Y = a.Y + (int64_t)bh * a.n_v * D;
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(a.key) + (int64_t)bh * a.n_v + start;
+
+  // pass over the group's rows, kSplitUnroll rows of a slot in flight
+  // (the loop bound is warp-uniform, so the row dot products' shuffles see every lane)
+  auto rows_pass = [&](auto&& body) {
+    for (int w0 = warp * RPW; w0 < len; w0 += SLOTS * kSplitUnroll) {
+      int id[kSplitUnroll];
+      float4 y[kSplitUnroll];
+#pragma unroll
+      for (int u = 0; u < kSplitUnroll; ++u) {
+        const int m = w0 + sub + u * SLOTS;
+        id[u] = m < len ? ord[m] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < kSplitUnroll; ++u)
+        y[u] = id[u] >= 0 ? *reinterpret_cast<const float4*>(Y + (int64_t)id[u] * D + 4 * fl)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kSplitUnroll; ++u) body(w0 + sub + u * SLOTS, id[u], y[u]);
+    }
+  };
+
+  // mean
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  rows_pass([&](int, int id, float4 y) {
+    if (id >= 0) { acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w; }
+  });
+  rb_block_sum<D>(acc, red, mean, 1.f / (float)len);
+  // start: the first row minus the mean, normalised (e_0 if that is zero)
+  if (tid < D) w[tid] = Y[(int64_t)ord[0] * D + tid] - mean[tid];
+  __syncthreads();
+  {
+    const float n0 = rb_norm(w, D, &s_tmp);
+    if (tid < D) w[tid] = n0 > 0.f ? w[tid] / n0 : (tid == 0 ? 1.f : 0.f);
+    __syncthreads();
+  }
+  // power steps on the covariance: z = sum (y - mean) ((y - mean) . w)
+  for (int it = 0; it < iters; ++it) {
+    const float4 mq = *reinterpret_cast<const float4*>(&mean[4 * fl]);
+    const float4 wq = *reinterpret_cast<const float4*>(&w[4 * fl]);
+    float4 zq = make_float4(0.f, 0.f, 0.f, 0.f);
+    rows_pass([&](int, int id, float4 y) {
+      const float4 c = make_float4(y.x - mq.x, y.y - mq.y, y.z - mq.z, y.w - mq.w);
+      const float p = rb_row_dot<D>(c, wq);
+      if (id >= 0) { zq.x = fmaf(c.x, p, zq.x); zq.y = fmaf(c.y, p, zq.y); zq.z = fmaf(c.z, p, zq.z); zq.w = fmaf(c.w, p, zq.w); }
+    });
+    rb_block_sum<D>(zq, red, z, 1.f);
+    const float nz = rb_norm(z, D, &s_tmp);
+    if (!(nz > 0.f)) break;   // uniform
+    if (tid < D) w[tid] = z[tid] / nz;
+    __syncthreads();
+  }
+  // projections as 64-bit keys: order-preserving float bits, then the row
+  {
+    const float4 wq = *reinterpret_cast<const float4*>(&w[4 * fl]);
+    rows_pass([&](int m, int id, float4 y) {
+      const float p = rb_row_dot<D>(y, wq) + 0.f;   // + 0: -0 -> +0 (ties then go by row)
+      if (id >= 0 && fl == 0) {
+        const uint32_t u = __float_as_uint(p);
+        const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        key[m] = ((unsigned long long)o << 32) | (uint32_t)id;
+      }
+    });
+  }
+  __syncthreads();
+  // radix select of the key of rank left-1 (keys are distinct: the row is in them)
+  unsigned long long prefix = 0ull, pmask = 0ull;
+  int want = left - 1;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = tid; i < 256; i += kSplitThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int m = tid; m < len; m += kSplitThreads) {
+      const unsigned long long k = key[m];
+      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, d = 0;
+      for (; d < 255; ++d) {
+        if (cum + (int)hist[d] > want) break;
+        cum += (int)hist[d];
+      }
+      s_int[0] = d;
+      s_int[1] = want - cum;
+    }
+    __syncthreads();
+    prefix |= (unsigned long long)s_int[0] << shift;
+    pmask |= 255ull << shift;
+    want = s_int[1];
+    __syncthreads();
+  }
+  const unsigned long long pivot = prefix;
+  // stable partition into tmp: rows with key <= pivot first, in their order
+  int32_t* tmp = a.tmp + (int64_t)bh * a.n_v + start;
+  int base_l = 0, base_r = left;
+  for (int c0 = 0; c0 < len; c0 += kSplitThreads) {
+    const int m = c0 + tid;
+    const bool valid = m < len;
+    const bool f = valid && key[m] <= pivot;
+    const uint32_t bl = __ballot_sync(0xffffffffu, f), bv = __ballot_sync(0xffffffffu, valid);
+    const uint32_t below = (1u << lane) - 1u;
+    if (lane == 0) { hist[warp] = __popc(bl); hist[32 + warp] = __popc(bv & ~bl); }
+    __syncthreads();
+    if (tid == 0) {
+      int sl = 0, sr = 0;
+      for (int w2 = 0; w2 < kSplitWarps; ++w2) {
+        const int l2 = (int)hist[w2], r2 = (int)hist[32 + w2];
+        hist[64 + w2] = (uint32_t)sl;
+        hist[96 + w2] = (uint32_t)sr;
+        sl += l2;
+        sr += r2;
+      }
+      s_int[2] = sl;
+      s_int[3] = sr;
+    }
+    __syncthreads();
+    if (valid) {
+      const int dst = f ? base_l + (int)hist[64 + warp] + __popc(bl & below)
+                        : base_r + (int)hist[96 + warp] + __popc(bv & ~bl & below);
+      tmp[dst] = ord[m];
+    }
+    base_l += s_int[2];
+    base_r += s_int[3];
+    __syncthreads();
+  }
+  for (int m = tid; m < len; m += kSplitThreads) ord[m] = tmp[m];
+  if (tid == 0 && base_l != left) raise_status(a.status, SOL_ERR_INVALID_ARG);   // cannot happen: keys are distinct
+}
+
+__global__ void rb_perm_kernel(const ReblockArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)a.B * a.H * a.N;
+  if (i >= total) return;
+  const int bh = (int)(i / a.N), pos = (int)(i % a.N);
+  a.perm[i] = pos < a.n_fix ? pos : a.n_fix + a.ord[(int64_t)bh * a.n_v + pos - a.n_fix];
+}
+
+// One warp per row: xp[b, h, pos] = x[b, perm[b, h, pos], h] (gather) or the reverse (scatter).
+template <int D, bool kGather>
+__global__ void __launch_bounds__(256) rb_rows_kernel(const int32_t* perm, const __nv_bfloat16* src, __nv_bfloat16* dst,
+                                                      int B, int H, int N, int64_t sb, int64_t sn, int64_t sh, int* status) {
+  constexpr int kPerLane = D / 32;   // bf16 per lane: 4 (D=128) or 2 (D=64)
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (int64_t)B * H * N) return;
+  const int bh = (int)(row / N), b = bh / H, h = bh % H;
+  const int t = perm[row];
+  if (t < 0 || t >= N) { if (lane == 0) raise_status(status, SOL_ERR_INVALID_ARG); return; }
+  const int64_t strided = (int64_t)b * sb + (int64_t)t * sn + (int64_t)h * sh + lane * kPerLane;
+  const int64_t packed = row * D + lane * kPerLane;
+  const __nv_bfloat16* s = src + (kGather ? strided : packed);
+  __nv_bfloat16* d = dst + (kGather ? packed : strided);
+  if (kPerLane == 4) *reinterpret_cast<uint2*>(d) = *reinterpret_cast<const uint2*>(s);
+  else *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(s);
+}
+
+}  // namespace
+
+int reblock_levels(int n_v) {
+  int lv = 0;
+  for (int leaves = (n_v + kBlock - 1) / kBlock; leaves > 1; leaves = (leaves + 1) / 2) ++lv;
+  return lv;
+}
+
+int reblock_moment_chunks(int n_q) { return (n_q + kMomRows - 1) / kMomRows; }
+
+cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
+  const int BH = a.B * a.H;
+  if (BH == 0 || a.N == 0) return cudaSuccess;
+  const int D = a.D;
+  static std::atomic<int> prepared[64];   // once per device: shared-memory opt-in
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int f128 = 128 * 129 * 4, w128 = (128 * 128 + 64 * 132) * 4, f64 = 64 * 65 * 4, w64 = (64 * 64 + 64 * 68) * 4;
+  if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
+    if ((e = cudaFuncSetAttribute(rb_factor_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, f128)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_whiten_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, w128)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_factor_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, f64)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_whiten_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, w64)) != cudaSuccess)
+      return e;
+    if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
+  }
+  if (a.n_v > 0) {
+    dim3 gm(a.mchunks, BH), gw((a.n_v + kBlock - 1) / kBlock, BH);
+    if (D == 128) {
+      rb_moment_kernel<128><<<gm, 256, 0, st>>>(a);
+      rb_factor_kernel<128><<<BH, 256, f128, st>>>(a);
+      rb_whiten_kernel<128><<<gw, 256, w128, st>>>(a);
+    } else {
+      rb_moment_kernel<64><<<gm, 256, 0, st>>>(a);
+      rb_factor_kernel<64><<<BH, 256, f64, st>>>(a);
+      rb_whiten_kernel<64><<<gw, 256, w64, st>>>(a);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int levels = reblock_levels(a.n_v);
+    for (int lvl = 0; lvl < levels; ++lvl) {
+      dim3 gs(1u << lvl, BH);
+      if (D == 128) rb_split_kernel<128><<<gs, kSplitThreads, 0, st>>>(a, lvl, iters);
+      else rb_split_kernel<64><<<gs, kSplitThreads, 0, st>>>(a, lvl, iters);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+  const int64_t total = (int64_t)BH * a.N;
+  rb_perm_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rows(const int32_t* perm, const __nv_bfloat16* src, __nv_bfloat16* dst, int B, int H, int N, int D,
+                        int64_t sb, int64_t sn, int64_t sh, bool gather, int* status, cudaStream_t st) {
+  const int64_t rows = (int64_t)B * H * N;
+  if (rows == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (D == 128) {
+    if (gather) rb_rows_kernel<128, true><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
+    else rb_rows_kernel<128, false><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
+  } else {
+    if (gather) rb_rows_kernel<64, true><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
+    else rb_rows_kernel<64, false><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sol

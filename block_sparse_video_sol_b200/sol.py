@@ -25,7 +25,8 @@ SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUD
 # Every entry point declared in include/sol.h.
 EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
            "sol_attn_fwd", "sol_forward_host", "sol_host_staging_bytes", "sol_last_device_status",
-           "sol_status_string", "sol_last_error_text", "sol_debug_drop_arrive")
+           "sol_status_string", "sol_last_error_text", "sol_debug_drop_arrive",
+           "sol_reblock_workspace_bytes", "sol_reblock", "sol_gather_rows", "sol_scatter_rows")
 
 
 class sol_params(ctypes.Structure):
@@ -66,6 +67,14 @@ lib.sol_last_error_text.argtypes = []
 lib.sol_last_error_text.restype = ctypes.c_char_p
 lib.sol_debug_drop_arrive.argtypes = [ctypes.c_int32]
 lib.sol_debug_drop_arrive.restype = ctypes.c_int
+lib.sol_reblock_workspace_bytes.argtypes = [_P]
+lib.sol_reblock_workspace_bytes.restype = ctypes.c_size_t
+lib.sol_reblock.argtypes = [_P, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]
+lib.sol_reblock.restype = ctypes.c_int
+lib.sol_gather_rows.argtypes = [_P, _vp, _vp, _vp, _vp]
+lib.sol_gather_rows.restype = ctypes.c_int
+lib.sol_scatter_rows.argtypes = [_P, _vp, _vp, _vp, _vp]
+lib.sol_scatter_rows.restype = ctypes.c_int
 
 
 class SolError(RuntimeError):
@@ -195,6 +204,30 @@ def sol_debug_drop_arrive(step: int):
     _check(lib.sol_debug_drop_arrive(step), "sol_debug_drop_arrive")
 
 
+def sol_reblock_workspace_bytes(p: sol_params) -> int:
+    return lib.sol_reblock_workspace_bytes(ctypes.byref(p))
+
+
+def sol_reblock(p: sol_params, q, k, ws: torch.Tensor, perm: torch.Tensor, stream=None):
+    _check(lib.sol_reblock(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(ws), ws.numel(), _ptr(perm), _stream(stream)),
+           "sol_reblock")
+
+
+def sol_gather_rows(p: sol_params, perm: torch.Tensor, x, xp: torch.Tensor, stream=None):
+    _check(lib.sol_gather_rows(ctypes.byref(p), _ptr(perm), _ptr(x), _ptr(xp), _stream(stream)), "sol_gather_rows")
+
+
+def sol_scatter_rows(p: sol_params, perm: torch.Tensor, xp: torch.Tensor, x, stream=None):
+    _check(lib.sol_scatter_rows(ctypes.byref(p), _ptr(perm), _ptr(xp), _ptr(x), _stream(stream)), "sol_scatter_rows")
+
+
+def head_major_params(p: sol_params) -> sol_params:
+    """The same problem on head-major [B, H, N, D] copies (inputs and output)."""
+    hm = (p.H * p.N * p.D, p.D, p.N * p.D)
+    return sol_params(p.B, p.N, p.H, p.D, p.q_block, p.k_block, p.tau, p.scale, p.prefix_len, p.log_mass_bias,
+                      *hm, *hm, p.routing, p.topk_ratio)
+
+
 @dataclass
 class Buffers:
     """Caller-owned device buffers of one problem shape (allocated by torch)."""
@@ -215,6 +248,40 @@ def alloc_buffers(p: sol_params, device, with_lse: bool = False) -> Buffers:
     return Buffers(ws, row_ptr, col_idx, o, lse)
 
 
+@dataclass
+class ReblockBuffers:
+    """Caller-owned buffers of a reblocked pass: the partition's workspace and
+    order, the head-major row copies and the Sol buffers of the copies (whose
+    ``o`` is the head-major output, in the partition's order)."""
+    ws: torch.Tensor
+    perm: torch.Tensor
+    qp: torch.Tensor
+    kp: torch.Tensor
+    vp: torch.Tensor
+    hm: sol_params
+    buf: Buffers
+
+
+def alloc_reblock(p: sol_params, device) -> ReblockBuffers:
+    hm = head_major_params(p)
+    ws = torch.empty(max(1, sol_reblock_workspace_bytes(p)), dtype=torch.uint8, device=device)
+    perm = torch.empty(max(1, p.B * p.H * p.N), dtype=torch.int32, device=device)
+    qp, kp, vp = (torch.empty((p.B, p.H, p.N, p.D), dtype=torch.bfloat16, device=device) for _ in range(3))
+    b = alloc_buffers(hm, device)
+    b.o = torch.empty((p.B, p.H, p.N, p.D), dtype=torch.bfloat16, device=device)
+    return ReblockBuffers(ws, perm, qp, kp, vp, hm, b)
+
+
+def forward_reblocked(p: sol_params, q, k, v, o: torch.Tensor, rb: ReblockBuffers, stream=None):
+    """Partition, gather q/k/v, pool -> route -> attention on the copies, scatter into ``o``."""
+    sol_reblock(p, q, k, rb.ws, rb.perm, stream)
+    for x, xp in ((q, rb.qp), (k, rb.kp), (v, rb.vp)):
+        sol_gather_rows(p, rb.perm, x, xp, stream)
+    forward(rb.hm, rb.qp, rb.kp, rb.vp, rb.buf, stream)
+    sol_scatter_rows(p, rb.perm, rb.buf.o, o, stream)
+    return o
+
+
 def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
     """Enqueue pool -> route -> attention on one stream; returns ``buf``."""
     sol_pool(p, q, k, v, buf.ws, stream)
@@ -225,10 +292,13 @@ def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
               log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False,
-              topk_ratio: Optional[float] = None, compressed: bool = False):
+              topk_ratio: Optional[float] = None, compressed: bool = False, reblock: bool = False):
     """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
 
-    Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.
+    Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.  With
+    ``reblock`` the rows are first ordered by the adaptive partition (sol_reblock) and the
+    buffers are a ReblockBuffers (its ``perm``, and the Sol buffers of the permuted rows;
+    ``with_lse`` is not offered there: the LSE would be in the permuted order).
     """
     B, N, H, D = q.shape
     for t in (q, k, v):
@@ -237,6 +307,13 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.
     p = make_params(B, N, H, D, tau, prefix_len, log_mass_bias, scale,
                     in_strides=(q.stride(0), q.stride(1), q.stride(2)), topk_ratio=topk_ratio,
                     compressed=compressed)
+    if reblock:
+        if with_lse:
+            raise ValueError("with_lse is not offered with reblock")
+        rb = alloc_reblock(p, q.device)
+        o = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=q.device)
+        forward_reblocked(p, q, k, v, o, rb)
+        return o, rb
     buf = alloc_buffers(p, q.device, with_lse)
     forward(p, q, k, v, buf)
     return buf.o, buf

@@ -187,3 +187,35 @@ def random_bf16(shape, seed: int, scale: float = 1.0) -> np.ndarray:
     """Plain i.i.d. N(0, scale^2) tensor as bf16 bits (for edge-case tests)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     return f32_to_bf16_bits(scale * rng.standard_normal(shape, dtype=np.float32))
+
+
+def planted_clusters(levels: int, D: int, H: int = 1, B: int = 1, prefix: int = 0, seed: int = 0,
+                     scale0: float = 16.0, offset: float = 10.0, noise: float = 0.05):
+    """Inputs with a planted hierarchy of key clusters (bf16 bit patterns, BTHD).
+
+    The rows past the prefix blocks form 2**levels clusters of 64 rows at random
+    positions; cluster c's keys are offset * e_(D-1) + sum_l scale0 / 2**l * s_l(c) e_l
+    plus Gaussian noise, s_l(c) = +1 or -1 from bit l of c (most significant
+    first).  Queries, values and the prefix rows are standard normal.  Returns
+    (q, k, v, cluster id of every partitioned row, number of prefix-block rows).
+    """
+    assert levels + 1 <= D
+    rng = np.random.default_rng(seed)
+    n_fix = 64 * (-(-prefix // 64))
+    n_v = 64 * 2 ** levels
+    N = n_fix + n_v
+    q = rng.standard_normal((B, N, H, D)).astype(np.float32)
+    k = rng.standard_normal((B, N, H, D)).astype(np.float32)
+    v = rng.standard_normal((B, N, H, D)).astype(np.float32)
+    cid = np.empty((B, H, n_v), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            c = rng.permutation(np.repeat(np.arange(2 ** levels), 64))
+            cid[b, h] = c
+            centers = np.zeros((2 ** levels, D), dtype=np.float32)
+            centers[:, D - 1] = offset
+            for lvl in range(levels):
+                sign = np.where((np.arange(2 ** levels) >> (levels - 1 - lvl)) & 1, 1.0, -1.0)
+                centers[:, lvl] = scale0 / 2 ** lvl * sign
+            k[b, n_fix:, h, :] = centers[c] + noise * rng.standard_normal((n_v, D)).astype(np.float32)
+    return f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v), cid, n_fix

@@ -224,6 +224,41 @@ size_t sol_host_staging_bytes(const sol_params* p, int32_t heads_per_chunk);
  * entry is out of range (SOL_ERR_INVALID_ARG). */
 sol_status sol_last_device_status(void* stream);
 
+/* ---- Adaptive partition (optional; Spark-H3 news page, Spark-Reblock
+ * bullet, and its workflow paragraph: reblock_layout=q_reuse_k) ----------
+ * sol_reblock computes, per (b, h), an order of the rows in which every 64
+ * consecutive rows are one adaptive block: the key rows past the prefix
+ * blocks (which stay in place) are whitened by the Cholesky factor of the
+ * video queries' second moment (mean q q^T + 1e-4 trace / D * I), so that
+ * the plain cosine of the unit vectors is the Mahalanobis cosine, and split
+ * recursively along each group's principal axis (4 power steps on its
+ * covariance from its first row minus its mean) at the size-balanced rank
+ * 64 * ceil(ceil(n / 64) / 2), lowest projections left, ties to the lower
+ * row; every group keeps ascending row order.  Queries reuse the keys' order.
+ * perm[(b*H + h)*N + pos] (int32, device, caller-owned) = the original row
+ * at position pos.  Fields used: B, N, H, D, prefix_len, in_stride_*; the
+ * other fields must still pass the common validation.  The workspace (device,
+ * 256-byte aligned, >= sol_reblock_workspace_bytes, which may be 0 when
+ * every row is a prefix-block row) holds fp32 whitened keys, partial
+ * moments, the factor and the split scratch (about 1.03 GB at B=1, H=56,
+ * N=32768, D=128); it may be reused once the stream has passed the call.
+ *
+ * A reblocked forward pass: sol_reblock; sol_gather_rows of q, k and v into
+ * head-major copies [B, H, N, D] (in_stride_* describe the source); the
+ * usual sol_pool / sol_route / sol_attn_fwd on the copies (strides
+ * b = H*N*D, n = D, h = N*D); sol_scatter_rows of the head-major output
+ * into o (out_stride_* describe the destination).  A perm entry outside
+ * [0, N) is skipped and reported as SOL_ERR_INVALID_ARG through the device
+ * status word.  All three enqueue on `stream` and return before the work
+ * runs. */
+size_t sol_reblock_workspace_bytes(const sol_params* p);
+sol_status sol_reblock(const sol_params* p, const void* q, const void* k, void* ws, size_t ws_bytes,
+                       int32_t* perm, void* stream);
+/* xp[b, h, pos, :] = x[b, perm[b, h, pos], h, :]  (x strided by in_stride_*) */
+sol_status sol_gather_rows(const sol_params* p, const int32_t* perm, const void* x, void* xp, void* stream);
+/* x[b, perm[b, h, pos], h, :] = xp[b, h, pos, :]  (x strided by out_stride_*) */
+sol_status sol_scatter_rows(const sol_params* p, const int32_t* perm, const void* xp, void* x, void* stream);
+
 /* Fault injection for testing the bounded waits (the device-side failure
  * path).  Only a library built with SOL_FAULT_TEST (libsol_fault.so, whose
  * waits expire after 2^16 polls instead of 2^22) acts on it: from the next
