@@ -190,10 +190,11 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
     if w.topk_ratio is not None:
         out = sol_ref.sol_forward(q, k, v, prefix=w.prefix, bq=64 if w.compressed else 128,
                                   topk_ratio=w.topk_ratio, compressed=w.compressed,
-                                  log_mass_bias_on=int(w.log_mass_bias) == 1, reweight_on=int(w.log_mass_bias) == 2)
+                                  log_mass_bias_on=int(w.log_mass_bias) == 1, reweight_on=int(w.log_mass_bias) == 2,
+                                  reblock=w.reblock)
     else:
         out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
-                                  reweight_on=int(w.log_mass_bias) == 2)
+                                  reweight_on=int(w.log_mass_bias) == 2, reblock=w.reblock)
     dt = time.perf_counter() - t0
     nk = sol_ref.block_rows(w.N, 64)
     nq = sol_ref.block_rows(w.N, 128 if (w.topk_ratio is not None and not w.compressed) else 64)
@@ -203,11 +204,12 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
 
 
 def routing_config(w: synth.Workload) -> dict:
+    rb = {"reblock": True} if w.reblock else {}
     if w.topk_ratio is None:
-        return {"routing": "threshold"}
+        return {"routing": "threshold", **rb}
     if w.compressed:
-        return {"routing": "topk+compressed", "topk_ratio": w.topk_ratio, "q_block": 64}
-    return {"routing": "topk", "topk_ratio": w.topk_ratio, "q_block": 128}
+        return {"routing": "topk+compressed", "topk_ratio": w.topk_ratio, "q_block": 64, **rb}
+    return {"routing": "topk", "topk_ratio": w.topk_ratio, "q_block": 128, **rb}
 
 
 def cpu_threads():
@@ -265,22 +267,41 @@ def run_ours(args, w):
     q, k, v = (h.to(dev) for h in host)
     p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
                         topk_ratio=w.topk_ratio, compressed=w.compressed)
-    buf = sol.alloc_buffers(p, dev)
     stream = torch.cuda.current_stream()
     launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 2   # pool (+ anchor, K/V), route + scan + compact, plan + attention
+    if w.reblock:
+        # the adaptive partition, then the Sol passes on head-major copies in its order
+        rb = sol.alloc_reblock(p, dev)
+        o_out = torch.empty_like(q)
+        rp_, rq, rk, rv, buf = rb.hm, rb.qp, rb.kp, rb.vp, rb.buf
+        launches_per_step += 4 + sol.reblock_levels(w.N - 64 * (-(-w.prefix // 64))) + 4   # partition, 3 gathers + scatter
+    else:
+        buf = sol.alloc_buffers(p, dev)
+        rp_, rq, rk, rv = p, q, k, v
+    n_ev = 7 if w.reblock else 4
 
     def step(ev=None):
-        if ev:
-            ev[0].record()
-        sol.sol_pool(p, q, k, v, buf.ws)
-        if ev:
-            ev[1].record()
-        sol.sol_route(p, buf.ws, buf.row_ptr, buf.col_idx)
-        if ev:
-            ev[2].record()
-        sol.sol_attn_fwd(p, q, k, v, buf.ws, buf.row_ptr, buf.col_idx, buf.o)
-        if ev:
-            ev[3].record()
+        def mark(i):
+            if ev:
+                ev[i].record()
+        mark(0)
+        j = 0
+        if w.reblock:
+            sol.sol_reblock(p, q, k, rb.ws, rb.perm)
+            mark(1)
+            for x, xp in ((q, rb.qp), (k, rb.kp), (v, rb.vp)):
+                sol.sol_gather_rows(p, rb.perm, x, xp)
+            mark(2)
+            j = 2
+        sol.sol_pool(rp_, rq, rk, rv, buf.ws)
+        mark(j + 1)
+        sol.sol_route(rp_, buf.ws, buf.row_ptr, buf.col_idx)
+        mark(j + 2)
+        sol.sol_attn_fwd(rp_, rq, rk, rv, buf.ws, buf.row_ptr, buf.col_idx, buf.o)
+        mark(j + 3)
+        if w.reblock:
+            sol.sol_scatter_rows(p, rb.perm, buf.o, o_out)
+            mark(6)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
 
@@ -297,7 +318,7 @@ def run_ours(args, w):
     flop = 4.0 * w.D * work   # work is summed over every (b, h)
     cent_flop = 4.0 * w.D * w.B * w.H * w.N * nb
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -314,22 +335,33 @@ def run_ours(args, w):
         dist.barrier()
     sol.sol_last_device_status()
     total_ms = t0.elapsed_time(t1)
-    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
-    pool_ms, route_ms, attn_ms = per.mean(axis=0)
+    per = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_ev - 1)] for e in evs]).mean(axis=0)
+    if w.reblock:
+        reblock_ms, gather_ms, pool_ms, route_ms, attn_ms, scatter_ms = per
+    else:
+        pool_ms, route_ms, attn_ms = per
 
     # e2e through the C ABI's host-buffer entry point: every step copies q, k, v from pinned host
     # memory, runs the forward pass and copies o back (pipelined over head chunks inside the call)
     o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
-    staging = torch.empty(sol.sol_host_staging_bytes(p), dtype=torch.uint8, device=dev)
+    staging = None if w.reblock else torch.empty(sol.sol_host_staging_bytes(p), dtype=torch.uint8, device=dev)
     h2d = 3 * q.numel() * q.element_size()
     d2h = o_host.numel() * o_host.element_size()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    sol.sol_forward_host(p, host[0], host[1], host[2], o_host, staging)   # warm-up (creates the copy streams)
+    def e2e_step():
+        if w.reblock:   # pinned host -> device copies, the reblocked pass, the output back
+            for hsrc, dsts in zip(host, (q, k, v)):
+                dsts.copy_(hsrc, non_blocking=True)
+            sol.forward_reblocked(p, q, k, v, o_out, rb)
+            o_host.copy_(o_out, non_blocking=True)
+        else:
+            sol.sol_forward_host(p, host[0], host[1], host[2], o_host, staging)
+    e2e_step()   # warm-up (creates the copy streams)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
-        sol.sol_forward_host(p, host[0], host[1], host[2], o_host, staging)
+        e2e_step()
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -368,13 +400,18 @@ def run_ours(args, w):
                               "GB/s": route_bytes / (route_ms * 1e-3) / 1e9},
                 "sol_attn_fwd": {"ms": attn_ms, "TFLOP/s_effective": attn_tf,
                                  "TFLOP/s_incl_centroids": (flop + cent_flop) / (attn_ms * 1e-3) / 1e12},
+                **({"sol_reblock": {"ms": reblock_ms},
+                    "sol_gather_rows": {"ms": gather_ms, "GB/s": 2 * in_bytes / (gather_ms * 1e-3) / 1e9},
+                    "sol_scatter_rows": {"ms": scatter_ms,
+                                         "GB/s": 2 * in_bytes / 3 / (scatter_ms * 1e-3) / 1e9}} if w.reblock else {}),
             },
             "density": float(density), "density_video_blocks": dens_video,
             "union_waste": union_waste, "exponentials_per_step": exps,
             "exact_flop_per_step": flop, "clocks": clocks.summary(),
             "e2e": {"value": flop_all / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "api": "sol_forward_host, pinned host buffers, 4-head chunks"},
+                    "api": ("pinned host copies + sol_reblock, gathers, pool/route/attention, scatter"
+                            if w.reblock else "sol_forward_host, pinned host buffers, 4-head chunks")},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -403,6 +440,8 @@ def main():
                     help="Top-K routing (the SLA variant: 128-row query blocks, no centroid terms)")
     ap.add_argument("--compressed", action="store_true",
                     help="with --topk-ratio: keep the compressed branch (64-row blocks, sink, centroid terms)")
+    ap.add_argument("--reblock", action="store_true",
+                    help="order the rows by the adaptive partition first (sol_reblock, gathers, scatter)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")
@@ -421,14 +460,15 @@ def main():
         ap.error("--topk-ratio takes no tau, and centroid options only with --compressed")
     if args.compressed and args.topk_ratio is None:
         ap.error("--compressed needs --topk-ratio")
-    if args.tau is not None or mode or args.topk_ratio is not None:
+    if args.tau is not None or mode or args.topk_ratio is not None or args.reblock:
         import dataclasses
         w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau, log_mass_bias=mode,
-                                topk_ratio=args.topk_ratio, compressed=args.compressed,
+                                topk_ratio=args.topk_ratio, compressed=args.compressed, reblock=args.reblock,
                                 name=w.name + (f"_tau{args.tau:g}" if args.tau is not None else "")
                                      + synth.mode_suffix(mode)
                                      + (f"_topk{args.topk_ratio:g}" if args.topk_ratio is not None else "")
-                                     + ("_compressed" if args.compressed else ""))
+                                     + ("_compressed" if args.compressed else "")
+                                     + ("_reblock" if args.reblock else ""))
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -221,6 +221,14 @@ def sol_scatter_rows(p: sol_params, perm: torch.Tensor, xp: torch.Tensor, x, str
     _check(lib.sol_scatter_rows(ctypes.byref(p), _ptr(perm), _ptr(xp), _ptr(x), _stream(stream)), "sol_scatter_rows")
 
 
+def reblock_levels(n_v: int) -> int:
+    """Split levels (sol_reblock launches one kernel per level) for n_v partitioned rows."""
+    lv, leaves = 0, -(-n_v // 64)
+    while leaves > 1:
+        leaves, lv = -(-leaves // 2), lv + 1
+    return lv
+
+
 def head_major_params(p: sol_params) -> sol_params:
     """The same problem on head-major [B, H, N, D] copies (inputs and output)."""
     hm = (p.H * p.N * p.D, p.D, p.N * p.D)

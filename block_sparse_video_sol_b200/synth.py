@@ -56,6 +56,7 @@ class Workload:
     log_mass_bias: int = 0     # centroid mode: 0 means, 1 + log-mass bias, 2 weighted summaries
     topk_ratio: Optional[float] = None   # Top-K routing instead of tau
     compressed: bool = False             # Top-K keeps the compressed branch (64-row blocks, centroids)
+    reblock: bool = False                # rows ordered by the adaptive partition first
     q_block: int = 64
     k_block: int = 64
 

@@ -138,3 +138,19 @@ def test_host_entry_validation(sol):
     assert sol.lib.sol_forward_host(ctypes.byref(p), h, h, h, h, 2, h, one, None) == sol.SOL_ERR_WORKSPACE
     assert sol.lib.sol_forward_host(ctypes.byref(sol.make_params(0, 1000, 4, 128)), None, None, None, None, 0,
                                     None, 0, None) == sol.SOL_OK
+
+
+def test_reblock_sizes_and_argument_checks(sol):
+    p = sol.make_params(1, 32768, 56, 128)
+    ws = sol.sol_reblock_workspace_bytes(p)
+    # fp32 whitened keys dominate: B*H*N*D*4, plus partial moments, factor, orders and keys
+    assert 56 * 32768 * 128 * 4 < ws < 56 * 32768 * 128 * 4 * 1.15
+    assert sol.sol_reblock_workspace_bytes(sol.make_params(1, 300, 2, 64, prefix_len=300)) == 0   # all prefix
+    assert sol.sol_reblock_workspace_bytes(sol.make_params(1, 0, 2, 64)) == 0
+    assert sol.reblock_levels(32768) == 9 and sol.reblock_levels(64) == 0 and sol.reblock_levels(65) == 1
+    P = ctypes.byref(p)
+    assert sol.lib.sol_reblock(P, None, None, None, 0, None, None) == sol.SOL_ERR_INVALID_ARG
+    assert sol.lib.sol_gather_rows(P, None, None, None, None) == sol.SOL_ERR_INVALID_ARG
+    assert sol.lib.sol_scatter_rows(P, None, None, None, None) == sol.SOL_ERR_INVALID_ARG
+    bad = sol.make_params(1, 100, 2, 96)
+    assert sol.lib.sol_reblock(ctypes.byref(bad), None, None, None, 0, None, None) == sol.SOL_ERR_UNSUPPORTED
