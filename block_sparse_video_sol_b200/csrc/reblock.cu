@@ -179,7 +179,6 @@ __global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* Ls = sm;             // [D][D]
   float* ks = sm + D * D;     // [64][LK]
-  __shared__ float s_inv[kBlock];
   const int tid = threadIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int t0 = blockIdx.x * kBlock;
   const float* Lg = a.L + (int64_t)bh * D * D;
@@ -192,26 +191,46 @@ __global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
     *reinterpret_cast<float4*>(&ks[r * LK + c4]) = v;
   }
   __syncthreads();
-  // thread (r = tid / 4, cg = tid % 4) computes columns cg + 4u of row r
-  const int r = tid >> 2, cg = tid & 3;
-  float y[D / 4];
+  // thread (rg = tid / 16, cq = tid % 16): rows 4 rg .. 4 rg + 3, columns CPT cq .. + CPT - 1;
+  // per head-dim step two (one) float4 loads of L and four broadcast loads of k feed 4 CPT FMAs
+  constexpr int CPT = D / 16;
+  const int rg = tid >> 4, cq = tid & 15;
+  float y[4][CPT];
 #pragma unroll
-  for (int u = 0; u < D / 4; ++u) y[u] = 0.f;
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) y[r][c] = 0.f;
   for (int i = 0; i < D; ++i) {
-    const float kv = ks[r * LK + i];
+    float lv[CPT];
 #pragma unroll
-    for (int u = 0; u < D / 4; ++u) y[u] = fmaf(kv, Ls[i * D + cg + 4 * u], y[u]);
+    for (int c = 0; c < CPT; c += 4) {
+      const float4 l4 = *reinterpret_cast<const float4*>(&Ls[i * D + CPT * cq + c]);
+      lv[c] = l4.x; lv[c + 1] = l4.y; lv[c + 2] = l4.z; lv[c + 3] = l4.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float kv = ks[(4 * rg + r) * LK + i];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) y[r][c] = fmaf(kv, lv[c], y[r][c]);
+    }
   }
-  float ss = 0.f;
+  float inv[4];
 #pragma unroll
-  for (int u = 0; u < D / 4; ++u) ss = fmaf(y[u], y[u], ss);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  if (cg == 0) s_inv[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+  for (int r = 0; r < 4; ++r) {   // row norms over the 16 lanes holding the row
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) ss = fmaf(y[r][c], y[r][c], ss);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    inv[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+  }
   __syncthreads();   // every thread has read ks
-  const float inv = s_inv[r];
 #pragma unroll
-  for (int u = 0; u < D / 4; ++u) ks[r * LK + cg + 4 * u] = y[u] * inv;
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CPT; c += 4)
+      *reinterpret_cast<float4*>(&ks[(4 * rg + r) * LK + CPT * cq + c]) =
+          make_float4(y[r][c] * inv[r], y[r][c + 1] * inv[r], y[r][c + 2] * inv[r], y[r][c + 3] * inv[r]);
   __syncthreads();
   float* Yg = a.Y + ((int64_t)bh * a.n_v + t0) * D;
   for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
@@ -364,9 +383,17 @@ __global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockAr
     const int shift = 56 - 8 * pass;
     for (int i = tid; i < 256; i += kSplitThreads) hist[i] = 0u;
     __syncthreads();
-    for (int m = tid; m < len; m += kSplitThreads) {
-      const unsigned long long k = key[m];
-      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255ull], 1u);
+    // warp-aggregated counts: the lanes holding one digit add it once (the top
+    // digits of nearby projections coincide, so plain atomics would serialise)
+    for (int m0 = warp * 32; m0 < len; m0 += kSplitThreads) {
+      const int m = m0 + lane;
+      uint32_t dig = 256u;
+      if (m < len) {
+        const unsigned long long k = key[m];
+        if ((k & pmask) == prefix) dig = (uint32_t)((k >> shift) & 255ull);
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+      if (dig < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (tid == 0) {
@@ -430,23 +457,23 @@ __global__ void rb_perm_kernel(const ReblockArgs a) {
   a.perm[i] = pos < a.n_fix ? pos : a.n_fix + a.ord[(int64_t)bh * a.n_v + pos - a.n_fix];
 }
 
-// One warp per row: xp[b, h, pos] = x[b, perm[b, h, pos], h] (gather) or the reverse (scatter).
+// xp[b, h, pos] = x[b, perm[b, h, pos], h] (gather) or the reverse (scatter):
+// D/8 lanes per row, 16 bytes each, so a warp moves 2 (D = 128) or 4 rows.
 template <int D, bool kGather>
 __global__ void __launch_bounds__(256) rb_rows_kernel(const int32_t* perm, const __nv_bfloat16* src, __nv_bfloat16* dst,
                                                       int B, int H, int N, int64_t sb, int64_t sn, int64_t sh, int* status) {
-  constexpr int kPerLane = D / 32;   // bf16 per lane: 4 (D=128) or 2 (D=64)
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  constexpr int LPR = D / 8, RPW = 32 / LPR, RPB = 8 * RPW;   // lanes per row, rows per warp, rows per block
+  const int lane = threadIdx.x & 31, fl = lane % LPR;
+  const int64_t row = (int64_t)blockIdx.x * RPB + (threadIdx.x >> 5) * RPW + lane / LPR;
   if (row >= (int64_t)B * H * N) return;
   const int bh = (int)(row / N), b = bh / H, h = bh % H;
   const int t = perm[row];
-  if (t < 0 || t >= N) { if (lane == 0) raise_status(status, SOL_ERR_INVALID_ARG); return; }
-  const int64_t strided = (int64_t)b * sb + (int64_t)t * sn + (int64_t)h * sh + lane * kPerLane;
-  const int64_t packed = row * D + lane * kPerLane;
+  if (t < 0 || t >= N) { if (fl == 0) raise_status(status, SOL_ERR_INVALID_ARG); return; }
+  const int64_t strided = (int64_t)b * sb + (int64_t)t * sn + (int64_t)h * sh + fl * 8;
+  const int64_t packed = row * D + fl * 8;
   const __nv_bfloat16* s = src + (kGather ? strided : packed);
   __nv_bfloat16* d = dst + (kGather ? packed : strided);
-  if (kPerLane == 4) *reinterpret_cast<uint2*>(d) = *reinterpret_cast<const uint2*>(s);
-  else *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(s);
+  *reinterpret_cast<uint4*>(d) = *reinterpret_cast<const uint4*>(s);
 }
 
 }  // namespace
@@ -505,7 +532,8 @@ cudaError_t launch_rows(const int32_t* perm, const __nv_bfloat16* src, __nv_bflo
                         int64_t sb, int64_t sn, int64_t sh, bool gather, int* status, cudaStream_t st) {
   const int64_t rows = (int64_t)B * H * N;
   if (rows == 0) return cudaSuccess;
-  const unsigned grid = (unsigned)((rows + 7) / 8);
+  const int rpb = 8 * (32 / (D / 8));   // rows per 256-thread block
+  const unsigned grid = (unsigned)((rows + rpb - 1) / rpb);
   if (D == 128) {
     if (gather) rb_rows_kernel<128, true><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
     else rb_rows_kernel<128, false><<<grid, 256, 0, st>>>(perm, src, dst, B, H, N, sb, sn, sh, status);
