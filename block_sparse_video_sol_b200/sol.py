@@ -246,12 +246,15 @@ class Buffers:
     lse: Optional[torch.Tensor]
 
 
-def alloc_buffers(p: sol_params, device, with_lse: bool = False) -> Buffers:
+def alloc_buffers(p: sol_params, device, with_lse: bool = False, head_major_out: bool = False) -> Buffers:
+    """Workspace, CSR and output of one problem; the output is [B, N, H, D], or
+    [B, H, N, D] with ``head_major_out`` (the layout of the reblocked copies)."""
     nqb = -(-p.N // 64)   # CSR rows are 64-row query blocks whatever the routing
     ws = torch.empty(max(1, sol_workspace_bytes(p)), dtype=torch.uint8, device=device)
     row_ptr = torch.empty(p.B * p.H * nqb + 1, dtype=torch.int32, device=device)
     col_idx = torch.empty(max(1, sol_col_capacity(p)), dtype=torch.int32, device=device)
-    o = torch.empty((p.B, p.N, p.H, p.D), dtype=torch.bfloat16, device=device)
+    shape = (p.B, p.H, p.N, p.D) if head_major_out else (p.B, p.N, p.H, p.D)
+    o = torch.empty(shape, dtype=torch.bfloat16, device=device)
     lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device=device) if with_lse else None
     return Buffers(ws, row_ptr, col_idx, o, lse)
 
@@ -275,9 +278,7 @@ def alloc_reblock(p: sol_params, device) -> ReblockBuffers:
     ws = torch.empty(max(1, sol_reblock_workspace_bytes(p)), dtype=torch.uint8, device=device)
     perm = torch.empty(max(1, p.B * p.H * p.N), dtype=torch.int32, device=device)
     qp, kp, vp = (torch.empty((p.B, p.H, p.N, p.D), dtype=torch.bfloat16, device=device) for _ in range(3))
-    b = alloc_buffers(hm, device)
-    b.o = torch.empty((p.B, p.H, p.N, p.D), dtype=torch.bfloat16, device=device)
-    return ReblockBuffers(ws, perm, qp, kp, vp, hm, b)
+    return ReblockBuffers(ws, perm, qp, kp, vp, hm, alloc_buffers(hm, device, head_major_out=True))
 
 
 def forward_reblocked(p: sol_params, q, k, v, o: torch.Tensor, rb: ReblockBuffers, stream=None):

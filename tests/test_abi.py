@@ -154,3 +154,17 @@ def test_reblock_sizes_and_argument_checks(sol):
     assert sol.lib.sol_scatter_rows(P, None, None, None, None) == sol.SOL_ERR_INVALID_ARG
     bad = sol.make_params(1, 100, 2, 96)
     assert sol.lib.sol_reblock(ctypes.byref(bad), None, None, None, 0, None, None) == sol.SOL_ERR_UNSUPPORTED
+
+
+def test_reblock_buffers_layout(sol):
+    p = sol.make_params(2, 300, 3, 64, prefix_len=70)
+    rb = sol.alloc_reblock(p, "cpu")   # allocation only: no kernel runs
+    assert rb.ws.numel() == sol.sol_reblock_workspace_bytes(p) > 0
+    assert rb.perm.numel() == 2 * 3 * 300 and rb.perm.dtype.is_floating_point is False
+    for t in (rb.qp, rb.kp, rb.vp, rb.buf.o):
+        assert tuple(t.shape) == (2, 3, 300, 64)
+    hm = rb.hm
+    assert (hm.in_stride_b, hm.in_stride_n, hm.in_stride_h) == (3 * 300 * 64, 64, 300 * 64)
+    assert (hm.out_stride_b, hm.out_stride_n, hm.out_stride_h) == (3 * 300 * 64, 64, 300 * 64)
+    assert (hm.B, hm.N, hm.H, hm.D, hm.prefix_len, hm.routing) == (2, 300, 3, 64, 70, p.routing)
+    assert rb.buf.ws.numel() == sol.sol_workspace_bytes(hm)
