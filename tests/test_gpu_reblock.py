@@ -157,3 +157,42 @@ def test_all_exact_reblocked_pass_is_dense_attention():
     err = (o.float() - ref.transpose(1, 2)).abs()
     assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS
     assert not torch.equal(rb.perm[:w.N].cpu(), torch.arange(w.N, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("N,D,prefix", [(1000, 64, 70), (777, 128, 13)])
+def test_ragged_reblocked_forward(N, D, prefix):
+    """Ragged lengths: a partial last leaf, a prefix that is not block aligned."""
+    from block_sparse_video_sol_b200 import sol
+    B, H = 1, 2
+    q, k, v = (synth.random_bf16((B, N, H, D), seed=s) for s in (21, 22, 23))
+    Q, K, V = to_dev(q), to_dev(k), to_dev(v)
+    p = sol.make_params(B, N, H, D, tau=1.0, prefix_len=prefix)
+    rb = sol.alloc_reblock(p, Q.device)
+    o = torch.empty_like(Q)
+    sol.forward_reblocked(p, Q, K, V, o, rb)
+    sol.sol_last_device_status()
+    perm = rb.perm.cpu().numpy().astype(np.int64).reshape(B, H, N)
+    _valid(perm, N, prefix)
+    Qd, Kd, Vd = (synth.bf16_bits_to_f64(x) for x in (q, k, v))
+    _first_split_band(Qd, Kd, perm, prefix)
+    nb = -(-N // 64)
+    rp = rb.buf.row_ptr.cpu().numpy().astype(np.int64)
+    ci = rb.buf.col_idx[:int(rp[-1])].cpu().numpy().astype(np.int64)
+    gm = sol_ref.from_csr(rp, ci, (B, H, nb, nb))
+    ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=1.0, prefix=prefix, reblock=True, perm_override=perm, mask_override=gm)
+    err = np.abs(o.float().cpu().numpy() - ref["O"])
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+
+
+def test_all_prefix_and_empty_partitions():
+    """P = N: nothing to partition, the order is the identity; N = 0: nothing runs."""
+    from block_sparse_video_sol_b200 import sol
+    N, H, D = 300, 2, 64
+    q, k = (to_dev(synth.random_bf16((1, N, H, D), seed=s)) for s in (31, 32))
+    perm = _gpu_perm(q, k, N, D)
+    assert np.array_equal(perm, np.tile(np.arange(N), (1, H, 1)))
+    p0 = sol.make_params(1, 0, H, D)
+    assert sol.sol_reblock_workspace_bytes(p0) == 0
+    e = torch.empty(16, dtype=torch.int32, device="cuda")
+    sol.sol_reblock(p0, q, k, torch.empty(1, dtype=torch.uint8, device="cuda"), e)
+    sol.sol_last_device_status()
