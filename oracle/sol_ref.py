@@ -76,6 +76,21 @@ What it computes, step by step, in the order the sources describe it:
                  holding prefix rows keep their place.  Q, K and V are
                  permuted per head, steps 1-8 run on the permuted rows, and O
                  is permuted back.
+ 10. INT8 QK with per-block residual keys (optional; thakicloud "MiniMax-H3
+                 ComfyUI accel stack", section 실제 실험 결과, closing accuracy
+                 paragraph: only each key block's residual from its mean is
+                 quantized to INT8, the mean term stays bf16; relative L2 error
+                 0.008 against the exact path, 0.030 when the whole key is
+                 quantized).  Reading: k_bar16_j = the block mean rounded to
+                 bf16; r_t = k_t - k_bar16_j; one symmetric scale per key block,
+                 sigma_j = max |r| / 127, codes rint(r / sigma_j) in [-127, 127];
+                 each query row quantized the same way with its own scale
+                 (the INT8 product needs an INT8 left operand); every exact
+                 logit becomes s * (q . k_bar16_j + sigma_q sigma_j (q_code .
+                 r_code)), with q . k_bar16_j taken from the unquantized bf16
+                 query.  Scales and codes are decided in fp32 (the kernel's
+                 precision): the quotient is rounded to the nearest integer,
+                 ties to even.  Centroid terms and routing are unchanged.
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -240,8 +255,63 @@ def reweighted_summaries(Q: np.ndarray, K: np.ndarray, V: np.ndarray, prefix: in
     return ktil, vtil, bias
 
 
+def int8_codes(X: np.ndarray, axis) -> tuple:
+    """Symmetric INT8 codes of X with one scale per slice reduced over ``axis``
+    (step 10): sigma = max |x| / 127 and code = rint(x / sigma) (ties to
+    even), both in fp32; sigma = 0 gives zero codes.  Returns (codes int64,
+    sigma float64 with the reduced axes kept)."""
+    x = np.asarray(X, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=axis, keepdims=True)
+    sigma = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(sigma > 0, sigma, np.float32(1.0))
+    codes = np.where(sigma > 0, np.rint(x / safe), np.float32(0.0))
+    return np.clip(codes, -127, 127).astype(np.int64), sigma.astype(np.float64)
+
+
+def int8_residual_keys(K: np.ndarray, bk: int) -> dict:
+    """Per-block residual quantization of the keys (step 10): the block mean
+    rounded to bf16 (``kmean16`` [B, H, nkb, D]), the residual codes
+    (``kcode`` [B, N, H, D]) and one scale per key block (``ksig`` [B, H, nkb])."""
+    B, N, H, D = K.shape
+    kmean16 = bf16_round(pool(K, bk))
+    kcode = np.zeros((B, N, H, D), dtype=np.int64)
+    ksig = np.zeros((B, H, n_blocks(N, bk)))
+    for j in range(n_blocks(N, bk)):
+        lo, hi = j * bk, min((j + 1) * bk, N)
+        # fp32 difference of two bf16 values (exact), [B, rows, H, D]
+        r = K[:, lo:hi].astype(np.float32) - kmean16[:, :, j][:, None, :, :].astype(np.float32)
+        c, sg = int8_codes(r, axis=(1, 3))
+        kcode[:, lo:hi] = c
+        ksig[:, :, j] = sg[:, 0, :, 0]
+    return dict(kmean16=kmean16, kcode=kcode, ksig=ksig)
+
+
+def int8_query_rows(Q: np.ndarray) -> dict:
+    """Per-row INT8 codes of the queries (step 10): ``qcode`` [B, N, H, D],
+    ``qsig`` [B, N, H]."""
+    c, sg = int8_codes(Q, axis=3)
+    return dict(qcode=c, qsig=sg[..., 0])
+
+
+def int8_logits(Q: np.ndarray, z: dict, b: int, h: int, r: np.ndarray, key_rows: np.ndarray, bk: int,
+                scale: float) -> np.ndarray:
+    """Exact-branch logits of query rows ``r`` against key rows ``key_rows`` of
+    (b, h) under step 10: s * (q . kmean16_j + sigma_q sigma_j (q_code . r_code))."""
+    blk = key_rows // bk
+    codes = (z["qcode"][b, r, h, :] @ z["kcode"][b, key_rows, h, :].T).astype(np.float64)
+    return scale * (Q[b, r, h, :] @ z["kmean16"][b, h, blk, :].T
+                    + z["qsig"][b, r, h][:, None] * z["ksig"][b, h, blk][None, :] * codes)
+
+
+def bf16_round(X: np.ndarray) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), through fp32."""
+    u = np.ascontiguousarray(X, dtype=np.float32).view(np.uint32)
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)) << np.uint32(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
-              rows: Optional[dict] = None, centroids: bool = True):
+              rows: Optional[dict] = None, centroids: bool = True, qk_int8: Optional[dict] = None):
     """Exact + centroid attention (step 4).
 
     For every query row r of block i (per b, h): logits are s*q_r.k_t for the
@@ -251,6 +321,9 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
     the natural-log normaliser.  ``rows`` optionally maps (b, h) to an array
     of query rows to compute; other rows are left NaN.  With ``centroids``
     False unselected blocks contribute nothing (Top-K routing, step 7).
+    ``qk_int8`` (the union of int8_residual_keys and int8_query_rows) makes
+    every exact logit the step-10 form s * (q . kmean16_j + sigma_q sigma_j
+    (q_code . r_code_t)).
     """
     B, N, H, D = Q.shape
     nqb, nkb = sel.shape[-2], sel.shape[-1]
@@ -275,7 +348,11 @@ def attention(Q, K, V, sel, kbar, vbar, bias, scale: float, bq: int, bk: int,
                                            for j in np.nonzero(s_j)[0]] or [np.zeros(0, int)])
                 cent = np.nonzero(~s_j)[0] if centroids else np.zeros(0, int)
                 q = Q[b, r, h, :]
-                lg = np.concatenate([scale * q @ K[b, key_rows, h, :].T,
+                if qk_int8 is None:
+                    exact = scale * q @ K[b, key_rows, h, :].T
+                else:
+                    exact = int8_logits(Q, qk_int8, b, h, r, key_rows, bk, scale)
+                lg = np.concatenate([exact,
                                      scale * q @ kbar[b, h, cent, :].T
                                      + (logn[cent] + bias[b, h, cent])[None, :]], axis=1)
                 vals = np.concatenate([V[b, key_rows, h, :], vbar[b, h, cent, :]], axis=0)
@@ -307,14 +384,11 @@ def second_moment_whitener(Q: np.ndarray, prefix: int) -> np.ndarray:
     return L
 
 
-def _split_group(Y: np.ndarray, members: np.ndarray, bs: int, iters: int, leaves: list):
-    """Recursive size-balanced principal-axis bisection (step 9); ``members``
-    ascending positions into Y (the whitened unit vectors)."""
-    n = len(members)
-    if n <= bs:
-        leaves.append(members)
-        return
-    left = bs * (-(-(-(-n // bs)) // 2))   # bs * ceil(ceil(n / bs) / 2)
+def split_projections(Y: np.ndarray, members: np.ndarray, iters: int = REBLOCK_ITERS) -> np.ndarray:
+    """Projections of one group's whitened unit vectors on its principal axis
+    (step 9): the axis comes from ``iters`` power-iteration steps on the
+    group's covariance, started from its first member minus its mean (e_0 if
+    that is zero); ``members`` are ascending positions into Y."""
     X = Y[members]
     C = X - X.mean(axis=0)
     w = C[0].copy()
@@ -330,12 +404,42 @@ def _split_group(Y: np.ndarray, members: np.ndarray, bs: int, iters: int, leaves
         if nz == 0:
             break
         w = z / nz
-    p = X @ w
+    return X @ w
+
+
+def split_left_count(n: int, bs: int = 64) -> int:
+    """Rows of the left part of a group of n > bs rows: bs * ceil(ceil(n / bs) / 2)
+    (the size-balanced split of step 9)."""
+    return bs * (-(-(-(-n // bs)) // 2))
+
+
+def _split_group(Y: np.ndarray, members: np.ndarray, bs: int, iters: int, leaves: list):
+    """Recursive size-balanced principal-axis bisection (step 9); ``members``
+    ascending positions into Y (the whitened unit vectors)."""
+    n = len(members)
+    if n <= bs:
+        leaves.append(members)
+        return
+    left = split_left_count(n, bs)
+    p = split_projections(Y, members, iters)
     order = np.lexsort((members, p))       # ascending projection, ties to the lower row
     go_left = np.zeros(n, dtype=bool)
     go_left[order[:left]] = True
     _split_group(Y, members[go_left], bs, iters, leaves)    # boolean selection keeps ascending order
     _split_group(Y, members[~go_left], bs, iters, leaves)
+
+
+def whitened_unit_keys(K: np.ndarray, L: np.ndarray, n_fix: int) -> np.ndarray:
+    """Y[b, h] = normalise(k_t L[b, h]) for the key rows t >= n_fix (step 9; a
+    zero row stays zero), so that Y[t] . Y[u] is the Mahalanobis cosine."""
+    B, N, H, D = K.shape
+    Y = np.zeros((B, H, N - n_fix, D))
+    for b in range(B):
+        for h in range(H):
+            Xw = K[b, n_fix:, h, :] @ L[b, h]
+            nrm = np.linalg.norm(Xw, axis=1, keepdims=True)
+            Y[b, h] = np.divide(Xw, nrm, out=np.zeros_like(Xw), where=nrm > 0)
+    return Y
 
 
 def reblock_partition(Q: np.ndarray, K: np.ndarray, prefix: int, bs: int = 64,
@@ -347,14 +451,11 @@ def reblock_partition(Q: np.ndarray, K: np.ndarray, prefix: int, bs: int = 64,
     perm = np.tile(np.arange(N, dtype=np.int64), (B, H, 1))
     if N - n_fix == 0:
         return perm
-    L = second_moment_whitener(Q, prefix)
+    Y = whitened_unit_keys(K, second_moment_whitener(Q, prefix), n_fix)
     for b in range(B):
         for h in range(H):
-            Xw = K[b, n_fix:, h, :] @ L[b, h]
-            nrm = np.linalg.norm(Xw, axis=1, keepdims=True)
-            Y = np.divide(Xw, nrm, out=np.zeros_like(Xw), where=nrm > 0)
             leaves: list = []
-            _split_group(Y, np.arange(N - n_fix), bs, iters, leaves)
+            _split_group(Y[b, h], np.arange(N - n_fix), bs, iters, leaves)
             perm[b, h, n_fix:] = n_fix + np.concatenate(leaves)
     return perm
 
@@ -383,8 +484,11 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
                 scale: Optional[float] = None, log_mass_bias_on: bool = False,
                 mask_override: Optional[np.ndarray] = None, rows: Optional[dict] = None,
                 reweight_on: bool = False, topk_ratio: Optional[float] = None, compressed: bool = False,
-                reblock: bool = False, perm_override: Optional[np.ndarray] = None):
+                reblock: bool = False, perm_override: Optional[np.ndarray] = None, qk_int8: bool = False):
     """The whole forward pass; returns a dict of every intermediate.
+
+    ``qk_int8`` (step 10) computes every exact logit from INT8 query codes
+    and INT8 per-block residual key codes plus the bf16 mean term.
 
     ``reweight_on`` (step 6) gives the centroid terms the anchor-weighted
     summaries ``kc``/``vc`` and their bias; otherwise ``kc``/``vc`` are the
@@ -402,7 +506,7 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
         perm = reblock_partition(Q, K, prefix, bk) if perm_override is None else perm_override
         r = sol_forward(permute_rows(Q, perm), permute_rows(K, perm), permute_rows(V, perm), tau, prefix,
                         bq, bk, scale, log_mass_bias_on, mask_override, rows, reweight_on, topk_ratio,
-                        compressed)
+                        compressed, qk_int8=qk_int8)
         r["O_permuted"], r["perm"] = r["O"], perm
         r["O"] = unpermute_rows(r["O"], perm)
         lse = r["lse"]   # [B, H, N]
@@ -413,12 +517,13 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
     s = (1.0 / math.sqrt(D)) if not scale else float(scale)
     qbar, kbar, vbar = pool(Q, bq), pool(K, bk), pool(V, bk)
     S = scores(qbar, kbar, s)
+    z = {**int8_residual_keys(K, bk), **int8_query_rows(Q)} if qk_int8 else None
     if topk_ratio is not None and not compressed:
         k = topk_count(topk_ratio, kbar.shape[2])
         sel = route_topk(S, k, prefix, bq)
         bias = np.zeros(kbar.shape[:3])
         used = sel if mask_override is None else mask_override
-        O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows, centroids=False)
+        O, lse = attention(Q, K, V, used, kbar, vbar, bias, s, bq, bk, rows=rows, centroids=False, qk_int8=z)
         return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kbar, vc=vbar, S=S, thr=None, sel=sel, k=k,
                     bias=bias, O=O, lse=lse, scale=s)
     k = None
@@ -437,6 +542,6 @@ def sol_forward(Q, K, V, tau: float = 1.0, prefix: int = 0, bq: int = 64, bk: in
     else:
         bias = np.zeros(kbar.shape[:3])
     used = sel if mask_override is None else mask_override
-    O, lse = attention(Q, K, V, used, kc, vc, bias, s, bq, bk, rows=rows)
+    O, lse = attention(Q, K, V, used, kc, vc, bias, s, bq, bk, rows=rows, qk_int8=z)
     return dict(qbar=qbar, kbar=kbar, vbar=vbar, kc=kc, vc=vc, S=S, thr=thr, sel=sel, k=k,
                 bias=bias, O=O, lse=lse, scale=s)
