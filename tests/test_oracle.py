@@ -302,9 +302,9 @@ def test_planted_mistakes_are_caught(monkeypatch):
     good_attention, good_thr, good_bias, good_pool = (sol_ref.attention, sol_ref.thresholds,
                                                       sol_ref.log_mass_bias, sol_ref.pool)
 
-    def no_log_n(Q, K, V, sel, kbar, vbar, bias, scale, bq, bk, rows=None):
+    def no_log_n(Q, K, V, sel, kbar, vbar, bias, scale, bq, bk, rows=None, **kw):
         return good_attention(Q, K, V, sel, kbar, vbar, bias - np.log(
-            sol_ref.block_rows(Q.shape[1], bk))[None, None, :], scale, bq, bk, rows)
+            sol_ref.block_rows(Q.shape[1], bk))[None, None, :], scale, bq, bk, rows, **kw)
 
     def sample_std(S, tau):
         mu = S.mean(-1)
