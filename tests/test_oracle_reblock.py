@@ -233,3 +233,82 @@ def test_planted_reblock_mistakes_are_caught(monkeypatch):
         monkeypatch.setattr(sol_ref, name, fn)
         assert all_pins() > 0, (name, fn.__name__)
         monkeypatch.undo()
+
+
+# ---- the split-by-split checker the GPU tests apply to the GPU's order --------------------------
+
+def _topic_inputs(N=1000, H=2, D=32, prefix=70, seed=11):
+    """Keys with a mild cluster structure (16 topics) and isotropic queries."""
+    rng = np.random.default_rng(seed)
+    topics = rng.standard_normal((16, D))
+    K = topics[rng.integers(0, 16, size=(1, N, H))] + rng.standard_normal((1, N, H, D))
+    Q = rng.standard_normal((1, N, H, D))
+    return Q, K, prefix
+
+
+@pytest.mark.parametrize("N,H,D,prefix", [(1000, 2, 32, 70), (777, 1, 16, 13), (4096, 1, 16, 0), (300, 2, 8, 300)])
+def test_split_checker_accepts_the_oracles_partition(N, H, D, prefix):
+    from tests.reblock_check import check_splits
+    Q, K, P = _topic_inputs(N, H, D, prefix)
+    perm = sol_ref.reblock_partition(Q, K, P)
+    rep = check_splits(Q, K, perm, P, band=0.0)
+    assert rep.exact == rep.groups   # the oracle's own splits, recomputed on their own members
+    n_v = N - min(N, 64 * (-(-P // 64)))
+    assert rep.levels == (math.ceil(math.log2(n_v / 64)) if n_v > 64 else 0)
+
+
+def _swap_across(perm, n_fix, start, n, which):
+    """Move the left part's highest-projecting row and the right part's
+    lowest-projecting row of one group across its split (each leaf re-sorted, so
+    only the split itself is wrong)."""
+    out = perm.copy()
+    left = sol_ref.split_left_count(n)
+    a, b = n_fix + start + which[0], n_fix + start + left + which[1]
+    out[0, 0, a], out[0, 0, b] = perm[0, 0, b], perm[0, 0, a]
+    for s in range(n_fix, out.shape[-1], 64):
+        out[0, 0, s:s + 64] = np.sort(out[0, 0, s:s + 64])
+    return out
+
+
+def test_split_checker_catches_planted_mistakes():
+    from tests.reblock_check import check_splits
+    Q, K, P = _topic_inputs(N=1000, H=1, D=32, prefix=70)
+    perm = sol_ref.reblock_partition(Q, K, P)
+    n_fix = 128
+    Y = sol_ref.whitened_unit_keys(K, sol_ref.second_moment_whitener(Q, P), n_fix)[0, 0]
+
+    def extremes(start, n):
+        part = perm[0, 0, n_fix + start:n_fix + start + n] - n_fix
+        members = np.sort(part)
+        p = sol_ref.split_projections(Y, members)[np.searchsorted(members, part)]
+        left = sol_ref.split_left_count(n)
+        return int(np.argmax(p[:left])), int(np.argmin(p[left:]))
+
+    n_v = 1000 - n_fix
+    first = _swap_across(perm, n_fix, 0, n_v, extremes(0, n_v))
+    # 872 video rows: groups [0, 448), [0, 256), [0, 128); the last splits the first two leaves
+    deep = _swap_across(perm, n_fix, 0, 128, extremes(0, 128))
+    moved = perm.copy()
+    moved[0, 0, [0, 500]] = moved[0, 0, [500, 0]]
+    unsorted = perm.copy()
+    unsorted[0, 0, [n_fix, n_fix + 1]] = unsorted[0, 0, [n_fix + 1, n_fix]]
+    for bad in (first, deep, moved, unsorted):
+        with pytest.raises(AssertionError):
+            check_splits(Q, K, bad, P, band=1e-3)
+
+
+@pytest.mark.parametrize("levels,prefix", [(8, 100), (9, 0)])
+def test_planted_hierarchy_is_recovered_at_full_depth(levels, prefix):
+    """The depth of the 16,384- and 32,768-row workloads: every leaf is one planted
+    cluster and every split is the oracle's own, far from a tie (the inputs the GPU
+    tests compare bit for bit)."""
+    from block_sparse_video_sol_b200 import synth
+    from tests.reblock_check import check_splits
+    q, k, _, cid, n_fix = synth.planted_clusters(levels, 128, H=1, prefix=prefix, seed=10 * levels + 128, noise=0.004)
+    Q, K = synth.bf16_bits_to_f64(q), synth.bf16_bits_to_f64(k)
+    perm = sol_ref.reblock_partition(Q, K, prefix)
+    for s in range(n_fix, perm.shape[-1], 64):
+        assert len(set(cid[0, 0][perm[0, 0, s:s + 64] - n_fix].tolist())) == 1
+    rep = check_splits(Q, K, perm, prefix, band=0.0)
+    assert rep.levels == levels and rep.exact == rep.groups == 2 ** levels - 1
+    assert rep.worst < -0.1   # every left part ends well below its right part
