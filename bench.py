@@ -55,7 +55,10 @@ def exact_work(row_ptr: np.ndarray, col_idx: np.ndarray, B: int, H: int, N: int)
 
 def route_stats(row_ptr, col_idx, B, H, N, prefix, q128, centroids):
     """Density over video query blocks, union waste of the attention's two-block tiles
-    (MMA work over needed work on exact tiles) and the exponentials per step."""
+    (MMA work over needed work on exact tiles), the exponentials per step, and the
+    S tiles the attention kernel issues (each = QK^T and PV of 128 rows x 128 keys):
+    ceil(union / 2) exact tiles per query tile, plus one per 128-block centroid chunk
+    holding a block that a present half leaves unselected."""
     nb = -(-N // 64)
     rows = B * H * nb
     mask = np.zeros((rows, nb), bool)
@@ -67,15 +70,23 @@ def route_stats(row_ptr, col_idx, B, H, N, prefix, q128, centroids):
     video = mask[:, first_video:]
     dens_video = float(video.mean()) if video.size else 0.0
     a, b = mask[:, 0::2], mask[:, 1::2]
+    present_b = np.arange(a.shape[1]) * 2 + 1 < nb
     b = np.concatenate([b, np.zeros_like(a[:, :a.shape[1] - b.shape[1]])], axis=1)
-    union = (a | b).sum()
+    uni = (a | b).sum(-1)                                 # [B*H, query tile]
+    union = uni.sum()
     needed = a.sum() + b.sum()
+    tiles = int(((uni + 1) // 2).sum())
+    if centroids:
+        unsel = ~a | (~b & present_b[None, :, None])      # a block some present half leaves out
+        pad = (-nb) % 128
+        unsel = np.concatenate([unsel, np.zeros(unsel.shape[:2] + (pad,), bool)], axis=-1)
+        tiles += int(unsel.reshape(unsel.shape[0], unsel.shape[1], -1, 128).any(-1).sum())
     nrows = np.minimum(np.arange(nb) * 64 + 64, N) - np.arange(nb) * 64   # valid rows of each block
     exact_keys = (mask * nrows[None, None, :]).sum(-1)                    # [B*H, query block]
     exps = int((exact_keys * nrows[None, :]).sum())
     if centroids:   # one term per unselected key block
         exps += int(((~mask).sum(-1) * nrows[None, :]).sum())
-    return dens_video, float(2 * union / max(needed, 1)), exps
+    return dens_video, float(2 * union / max(needed, 1)), exps, tiles
 
 
 def read_peaks():
@@ -117,11 +128,12 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.index, self.rows, self.proc = index, [], None
+        self.t0, self.t1 = 0.0, float("inf")
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -134,7 +146,15 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 8:
-                self.rows.append(parts)
+                self.rows.append((time.perf_counter(), parts))
+
+    def mark(self, start: bool):
+        """Host time at the start / end of the timed region: only samples read in
+        between (plus one sampling interval for the output's delay) are summarised."""
+        if start:
+            self.t0 = time.perf_counter()
+        else:
+            self.t1 = time.perf_counter()
 
     def __exit__(self, *exc):
         if self.proc:
@@ -143,15 +163,16 @@ class ClockSampler:
             self.proc.wait(timeout=5)
 
     def summary(self):
-        if not self.rows:
+        rows = [r for t, r in self.rows if self.t0 <= t <= self.t1 + 0.05] or [r for _, r in self.rows]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = max(float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit())
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
-        loaded = sorted(sm)[len(sm) // 4:] or sm
-        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(self.rows)}
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "window": "samples read during the timed region"}
 
 
 def dist_env():
@@ -162,6 +183,13 @@ def dist_env():
 def shard_b_offset(rank: int, w: synth.Workload) -> int:
     """Batch index of this rank's first sequence: rank r runs sequences r*B .. r*B+B-1 of the job."""
     return rank * w.B
+
+
+def shard_heads(rank: int, world: int, H: int) -> list:
+    """Heads of one call that rank r runs when the call is split by head: a contiguous run,
+    sizes differing by at most one.  Every stage is per head, so no collective is needed
+    when the heads arrive sharded (as after a head-parallel QKV projection)."""
+    return list(range(rank * H // world, (rank + 1) * H // world))
 
 
 def job_reduce(values, device, world: int):
@@ -233,12 +261,17 @@ def run_reference(args, w):
         times.append(dt)
         works.append(work)
     sec = float(np.mean(times))
-    # scale the sample to the whole step (all heads) for the per-call time
+    # The whole call (all heads) would take minutes per step on the host, so each step runs
+    # a head sample; ms_per_step is that sample's time scaled to all heads (an extrapolation,
+    # labelled in the line), while value is a plain rate measured on the sample itself.
     ms_call = sec * 1e3 * w.H / len(heads)
     val = 4 * w.D * float(np.mean(works)) / sec / 1e12
     sample = f"{len(heads)} of {w.H} heads of {w.name} per step (full pool/route/attention of those heads)"
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call,
+            "ms_per_step_basis": (f"extrapolated: {sec * 1e3:.0f} ms measured per step on {len(heads)} of "
+                                  f"{w.H} heads, x {w.H / len(heads):g}"),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
                        "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, **routing_config(w)},
@@ -259,13 +292,17 @@ def run_ours(args, w):
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=300))
     from block_sparse_video_sol_b200 import sol
 
-    # this rank's sequence: batch element `rank` of a world-size batch (pinned host copies for e2e)
-    shape = (w.B, w.N, w.H, w.D)
+    # this rank's work (pinned host copies for e2e): batch element `rank` of a world-size batch,
+    # or with --shard heads its run of heads of the one call
+    by_heads = args.shard == "heads"
+    heads = shard_heads(rank, world, w.H) if by_heads else None
+    Hr = len(heads) if by_heads else w.H
+    shape = (w.B, w.N, Hr, w.D)
     host = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-    synth.generate(w, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host),
-                   b_offset=shard_b_offset(rank, w))
+    synth.generate(w, heads=heads, out=tuple(h.view(torch.int16).numpy().view(np.uint16) for h in host),
+                   b_offset=0 if by_heads else shard_b_offset(rank, w))
     q, k, v = (h.to(dev) for h in host)
-    p = sol.make_params(w.B, w.N, w.H, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
+    p = sol.make_params(w.B, w.N, Hr, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
                         topk_ratio=w.topk_ratio, compressed=w.compressed)
     stream = torch.cuda.current_stream()
     launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 2   # pool (+ anchor, K/V), route + scan + compact, plan + attention
@@ -310,13 +347,14 @@ def run_ours(args, w):
     sol.sol_last_device_status()
     rp = buf.row_ptr.cpu().numpy().astype(np.int64)
     ci = buf.col_idx[:int(rp[-1])].cpu().numpy().astype(np.int64)
-    work = exact_work(rp, ci, w.B, w.H, w.N)
+    work = exact_work(rp, ci, w.B, Hr, w.N)
     nb = -(-w.N // 64)
-    density = rp[-1] / (w.B * w.H * nb * nb)
+    density = rp[-1] / (w.B * Hr * nb * nb)
     sla = w.topk_ratio is not None and not w.compressed
-    dens_video, union_waste, exps = route_stats(rp, ci, w.B, w.H, w.N, w.prefix, sla, not sla)
+    dens_video, union_waste, exps, tiles = route_stats(rp, ci, w.B, Hr, w.N, w.prefix, sla, not sla)
+    issued_flop = 4.0 * 128 * 128 * w.D * tiles   # what the tensor cores execute (QK^T + PV per S tile)
     flop = 4.0 * w.D * work   # work is summed over every (b, h)
-    cent_flop = 4.0 * w.D * w.B * w.H * w.N * nb
+    cent_flop = 4.0 * w.D * w.B * Hr * w.N * nb
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -324,6 +362,7 @@ def run_ours(args, w):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        clocks.mark(True)
         t0.record()
         for s in range(args.steps):
             if flush is not None:
@@ -331,6 +370,7 @@ def run_ours(args, w):
             step(evs[s])
         t1.record()
         torch.cuda.synchronize()
+        clocks.mark(False)
     if world > 1:
         dist.barrier()
     sol.sol_last_device_status()
@@ -373,30 +413,42 @@ def run_ours(args, w):
         ms_step = total_ms / args.steps
         value = flop_all / (ms_step * 1e-3) / 1e12
         attn_tf = flop / (attn_ms * 1e-3) / 1e12
+        issued_tf = issued_flop / (attn_ms * 1e-3) / 1e12
         traffic, tnote = profiled_traffic("sol_attn_fwd")
-        in_bytes = 3 * w.B * w.N * w.H * w.D * 2
+        in_bytes = 3 * w.B * w.N * Hr * w.D * 2
         # route: fp32 centroids in, bitmap + counts + CSR out (not its bound: it is ALU work)
-        route_bytes = 2 * w.B * w.H * nb * w.D * 4 + w.B * w.H * nb * (4 * (-(-nb // 32)) + 8) + 4 * int(rp[-1])
-        pool_bytes = (2 if sla else 3) * w.B * w.N * w.H * w.D * 2   # the SLA variant pools no V
+        route_bytes = 2 * w.B * Hr * nb * w.D * 4 + w.B * Hr * nb * (4 * (-(-nb // 32)) + 8) + 4 * int(rp[-1])
+        pool_bytes = (2 if sla else 3) * w.B * w.N * Hr * w.D * 2   # the SLA variant pools no V
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if by_heads else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "tau": w.tau,
                        "prefix": w.prefix, "log_mass_bias": w.log_mass_bias, **routing_config(w),
-                       "global_batch": w.B * world,
-                       "parallelism": f"dp{world} (one sequence per GPU)",
+                       "global_batch": w.B if by_heads else w.B * world,
+                       "parallelism": (f"heads split {world} ways ({Hr} of {w.H} heads on rank 0), no collective"
+                                       if by_heads else f"dp{world} (one sequence per GPU)"),
                        "l2": (f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step vs 126 MB)"
                               + (", 256 MB written before each step" if args.flush_l2 else ", no flush"))},
+            # The attention kernel runs for milliseconds back to back under the 1 kW cap
+            # (sw_power_cap active, SM clock ~1.4 GHz in its phase trace), the regime of the
+            # sustained bf16 figure; the burst fraction is kept beside it.
             "roofline": {"kernel": "sol_attn_fwd", "bound": "tensor", "achieved": attn_tf,
-                         "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16"],
-                         "peak_source": f"{peaks['source']} bf16 burst", "traffic": traffic,
-                         "traffic_note": tnote},
+                         "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_sus"],
+                         "peak_source": f"{peaks['source']} bf16 sustained (a kernel timed inside a long run "
+                                        "under the power cap)",
+                         "frac_of_burst": attn_tf / peaks["bf16"],
+                         "issued_mma_tflops": issued_tf, "issued_frac": issued_tf / peaks["bf16_sus"],
+                         "issued_note": "tensor-core work executed: 4*128*128*D per S tile (exact tiles = "
+                                        "ceil(union/2) per query tile, plus centroid tiles); achieved counts "
+                                        "only the exact keys the rows need",
+                         "traffic": traffic, "traffic_note": tnote},
             "kernels": {
                 "sol_pool": {"ms": pool_ms, "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9,
                              "frac_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / peaks["hbm"]},
                 "sol_route": {"ms": route_ms,
-                              "TFLOP/s_fp32": 2.0 * w.B * w.H * nb * nb * w.D / (route_ms * 1e-3) / 1e12,
+                              "TFLOP/s_fp32": 2.0 * w.B * Hr * nb * nb * w.D / (route_ms * 1e-3) / 1e12,
                               "GB/s": route_bytes / (route_ms * 1e-3) / 1e9},
                 "sol_attn_fwd": {"ms": attn_ms, "TFLOP/s_effective": attn_tf,
                                  "TFLOP/s_incl_centroids": (flop + cent_flop) / (attn_ms * 1e-3) / 1e12},
@@ -442,6 +494,9 @@ def main():
                     help="with --topk-ratio: keep the compressed branch (64-row blocks, sink, centroid terms)")
     ap.add_argument("--reblock", action="store_true",
                     help="order the rows by the adaptive partition first (sol_reblock, gathers, scatter)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="with --gpus N: one sequence per GPU (batch, weak scaling) or the heads of one "
+                         "call split over the GPUs (heads, strong scaling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-heads", type=int, default=None,
                     help="heads per oracle sample (default: 1 for --impl reference steps, 6 for cpu_baseline)")

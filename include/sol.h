@@ -41,6 +41,13 @@
  *     addresses must be 16-byte aligned and every stride a multiple of 8
  *     elements.
  *   - B == 0 or N == 0 is a valid empty problem: nothing is enqueued.
+ *   - Heads are independent in every stage, so a call may cover any run of
+ *     heads [h0, h0 + Hg) of a larger tensor: set H = Hg, keep the strides,
+ *     and offset each base pointer by h0 * in_stride_h (O by h0 *
+ *     out_stride_h) elements.  Workspace, CSR and LSE then hold those Hg
+ *     heads only (CSR rows in (b, h - h0, i) order), and every output equals
+ *     that head's slice of the whole call bit for bit.  This is how one call
+ *     is split over GPUs (each takes H / G heads, no collective).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).
  */
 #ifndef SOL_H_

@@ -353,3 +353,42 @@ def test_forward_captures_into_a_cuda_graph(kw):
         assert torch.equal(buf.o, ref_buf.o)
         assert torch.equal(buf.row_ptr, ref_buf.row_ptr)
     sol.sol_last_device_status()
+
+
+# ---------------------------------------------------------------- head split (one call over several GPUs)
+@pytest.mark.parametrize("kw", [dict(), dict(prefix_len=100, log_mass_bias=2, topk_ratio=0.2, compressed=True),
+                                dict(topk_ratio=0.15)])
+def test_head_runs_equal_the_whole_call(kw):
+    """Heads are independent in every stage: calls on the head runs [0, 21) and [21, 56)
+    of the same tensors (H = the run's length, base pointers offset by h0 heads, strides
+    kept) give the whole call's O and LSE bit for bit, and their CSR lists, concatenated,
+    are the whole call's.  This is how one call is split over GPUs."""
+    from block_sparse_video_sol_b200 import sol
+    w = synth.h56_n4096()
+    q, k, v = (parity.to_dev(x) for x in synth.generate(w))
+    B, N, H, D = q.shape
+    whole_p = sol.make_params(B, N, H, D, **kw)
+    whole = sol.alloc_buffers(whole_p, "cuda", with_lse=True)
+    sol.forward(whole_p, q, k, v, whole)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    rp_all, ci_all, base = [], [], 0
+    for h0, h1 in ((0, 21), (21, 56)):
+        p = sol.make_params(B, N, h1 - h0, D, in_strides=q.stride()[:3], out_strides=o.stride()[:3], **kw)
+        buf = sol.alloc_buffers(p, "cuda")
+        qs, ks, vs, os_ = (x[:, :, h0:h1] for x in (q, k, v, o))
+        sol.sol_pool(p, qs, ks, vs, buf.ws)
+        sol.sol_route(p, buf.ws, buf.row_ptr, buf.col_idx)
+        part_lse = torch.empty((B, h1 - h0, N), device="cuda")
+        sol.sol_attn_fwd(p, qs, ks, vs, buf.ws, buf.row_ptr, buf.col_idx, os_, part_lse)
+        lse[:, h0:h1] = part_lse
+        nnz = int(buf.row_ptr[-1])
+        rp_all.append(buf.row_ptr[:-1] + base)
+        ci_all.append(buf.col_idx[:nnz])
+        base += nnz
+    sol.sol_last_device_status()
+    assert torch.equal(o, whole.o)
+    assert torch.equal(lse, whole.lse)
+    rp = torch.cat(rp_all + [torch.tensor([base], dtype=torch.int32, device="cuda")])
+    assert torch.equal(rp, whole.row_ptr)
+    assert torch.equal(torch.cat(ci_all), whole.col_idx[:base])
