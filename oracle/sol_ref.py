@@ -89,8 +89,9 @@ What it computes, step by step, in the order the sources describe it:
                  logit becomes s * (q . k_bar16_j + sigma_q sigma_j (q_code .
                  r_code)), with q . k_bar16_j taken from the unquantized bf16
                  query.  Scales and codes are decided in fp32 (the kernel's
-                 precision): the quotient is rounded to the nearest integer,
-                 ties to even.  Centroid terms and routing are unchanged.
+                 precision): x times the fp32 reciprocal of sigma, rounded to
+                 the nearest integer, ties to even.  Centroid terms and routing
+                 are unchanged.
 
 Readings where the sources are silent (each is listed in the design notes):
 blocks are consecutive rows tiling the whole packed sequence from row 0 (the
@@ -257,14 +258,15 @@ def reweighted_summaries(Q: np.ndarray, K: np.ndarray, V: np.ndarray, prefix: in
 
 def int8_codes(X: np.ndarray, axis) -> tuple:
     """Symmetric INT8 codes of X with one scale per slice reduced over ``axis``
-    (step 10): sigma = max |x| / 127 and code = rint(x / sigma) (ties to
-    even), both in fp32; sigma = 0 gives zero codes.  Returns (codes int64,
-    sigma float64 with the reduced axes kept)."""
+    (step 10): sigma = max |x| / 127 and code = rint(x * (1 / sigma)) (ties to
+    even), all in fp32 with the reciprocal rounded to fp32 (the kernel's
+    precision, which decides the integer); sigma = 0 gives zero codes.
+    Returns (codes int64, sigma float64 with the reduced axes kept)."""
     x = np.asarray(X, dtype=np.float32)
     amax = np.max(np.abs(x), axis=axis, keepdims=True)
     sigma = (amax / np.float32(127.0)).astype(np.float32)
-    safe = np.where(sigma > 0, sigma, np.float32(1.0))
-    codes = np.where(sigma > 0, np.rint(x / safe), np.float32(0.0))
+    inv = (np.float32(1.0) / np.where(sigma > 0, sigma, np.float32(1.0))).astype(np.float32)
+    codes = np.where(sigma > 0, np.rint((x * inv).astype(np.float32)), np.float32(0.0))
     return np.clip(codes, -127, 127).astype(np.int64), sigma.astype(np.float64)
 
 

@@ -168,14 +168,14 @@ def test_planted_int8_mistakes_are_caught(monkeypatch):
     def codes_128(X, axis):               # scale max/128 instead of max/127
         x = np.asarray(X, dtype=np.float32)
         sg = (np.max(np.abs(x), axis=axis, keepdims=True) / np.float32(128.0)).astype(np.float32)
-        safe = np.where(sg > 0, sg, np.float32(1.0))
-        return np.clip(np.where(sg > 0, np.rint(x / safe), 0), -127, 127).astype(np.int64), sg.astype(np.float64)
+        inv = (np.float32(1.0) / np.where(sg > 0, sg, np.float32(1.0))).astype(np.float32)
+        return np.clip(np.where(sg > 0, np.rint(x * inv), 0), -127, 127).astype(np.int64), sg.astype(np.float64)
 
     def codes_trunc(X, axis):             # truncation instead of rounding to nearest
         c, sg = real_codes(X, axis)
         x = np.asarray(X, dtype=np.float32)
-        safe = np.where(sg > 0, sg, 1.0).astype(np.float32)
-        return np.clip(np.where(sg > 0, np.trunc(x / safe), 0), -127, 127).astype(np.int64), sg
+        inv = (1.0 / np.where(sg > 0, sg, 1.0)).astype(np.float32)
+        return np.clip(np.where(sg > 0, np.trunc(x * inv), 0), -127, 127).astype(np.int64), sg
 
     def keys_without_mean(K, bk):         # the whole key quantized, mean term dropped
         B, N, H, D = K.shape
