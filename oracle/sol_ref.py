@@ -81,9 +81,11 @@ What it computes, step by step, in the order the sources describe it:
                  paragraph: only each key block's residual from its mean is
                  quantized to INT8, the mean term stays bf16; relative L2 error
                  0.008 against the exact path, 0.030 when the whole key is
-                 quantized).  Reading: k_bar16_j = the block mean rounded to
-                 bf16; r_t = k_t - k_bar16_j; one symmetric scale per key block,
-                 sigma_j = max |r| / 127, codes rint(r / sigma_j) in [-127, 127];
+                 quantized).  Reading: k_bar16_j = the block mean (an fp32 sum
+                 in row order times the fp32 reciprocal of the count, the
+                 kernel's precision, since its rounding decides integer codes)
+                 rounded to bf16; r_t = k_t - k_bar16_j; one symmetric scale per key block,
+                 sigma_j = max |r| / 127, codes rint(r * (1 / sigma_j)) in [-127, 127];
                  each query row quantized the same way with its own scale
                  (the INT8 product needs an INT8 left operand); every exact
                  logit becomes s * (q . k_bar16_j + sigma_q sigma_j (q_code .
@@ -270,12 +272,26 @@ def int8_codes(X: np.ndarray, axis) -> tuple:
     return np.clip(codes, -127, 127).astype(np.int64), sigma.astype(np.float64)
 
 
+def mean_fp32(K: np.ndarray, bk: int) -> np.ndarray:
+    """Block means as the kernels compute them: an fp32 sum over the block's rows
+    in row order, times the fp32 reciprocal of the row count ([B, H, nkb, D])."""
+    B, N, H, D = K.shape
+    out = np.empty((B, H, n_blocks(N, bk), D), dtype=np.float32)
+    for j in range(n_blocks(N, bk)):
+        lo, hi = j * bk, min((j + 1) * bk, N)
+        acc = np.cumsum(K[:, lo:hi].astype(np.float32), axis=1, dtype=np.float32)[:, -1]   # sequential fp32
+        out[:, :, j] = acc * (np.float32(1.0) / np.float32(hi - lo))
+    return out.astype(np.float64)
+
+
 def int8_residual_keys(K: np.ndarray, bk: int) -> dict:
     """Per-block residual quantization of the keys (step 10): the block mean
     rounded to bf16 (``kmean16`` [B, H, nkb, D]), the residual codes
-    (``kcode`` [B, N, H, D]) and one scale per key block (``ksig`` [B, H, nkb])."""
+    (``kcode`` [B, N, H, D]) and one scale per key block (``ksig`` [B, H, nkb]).
+    The mean is summed in fp32 in row order (the kernel's precision): its bf16
+    rounding decides the residuals, hence integer codes."""
     B, N, H, D = K.shape
-    kmean16 = bf16_round(pool(K, bk))
+    kmean16 = bf16_round(mean_fp32(K, bk))
     kcode = np.zeros((B, N, H, D), dtype=np.int64)
     ksig = np.zeros((B, H, n_blocks(N, bk)))
     for j in range(n_blocks(N, bk)):
