@@ -24,8 +24,8 @@
 //   rb_moment_kernel  -- partial sums of q q^T over 2048-row chunks (fp32);
 //   rb_factor_kernel  -- one CTA per head: the partials summed in a fixed
 //                        order, the ridge, the Cholesky factor in shared memory;
-//   rb_whiten_kernel  -- y = normalise(k L) for 64 rows per CTA, and the
-//                        initial (identity) order;
+//   rb_whiten_kernel  -- y = normalise(k L), L loaded once per CTA for 8 tiles
+//                        of 64 rows, and the initial (identity) order;
 //   rb_split_kernel   -- one launch per level of the hierarchy, one CTA per
 //                        group: mean, power steps, projections as 64-bit keys
 //                        (order-preserving float bits, row index), the split
@@ -41,6 +41,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "ptx.cuh"   // packed f32x2 arithmetic
 
 namespace sol {
 
@@ -48,8 +49,6 @@ namespace {
 
 constexpr int kMomRows = 2048;       // query rows per partial-moment CTA
 constexpr int kMomStage = 32;        // rows staged in shared memory at a time
-constexpr int kSplitThreads = 1024;  // threads of a split CTA
-constexpr int kSplitWarps = kSplitThreads / 32;
 constexpr int kSplitUnroll = 4;      // rows in flight per row slot
 
 __host__ __device__ inline int rb_left(int n) { return kBlock * ((((n + kBlock - 1) / kBlock) + 1) / 2); }
@@ -85,11 +84,11 @@ __global__ void __launch_bounds__(256) rb_moment_kernel(const ReblockArgs a) {
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int r0 = a.q_lo + blockIdx.x * kMomRows, r1 = min(a.q_lo + a.n_q, r0 + kMomRows);
   const __nv_bfloat16* qb = a.q + (int64_t)b * a.sb + (int64_t)h * a.sh;
-  float acc[TS][TS];
+  uint64_t acc[TS][TS / 2];   // packed column pairs
 #pragma unroll
   for (int i = 0; i < TS; ++i)
 #pragma unroll
-    for (int j = 0; j < TS; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < TS / 2; ++j) acc[i][j] = 0ull;
   for (int s0 = r0; s0 < r1; s0 += kMomStage) {
     __syncthreads();
     for (int idx = tid; idx < kMomStage * (D / 4); idx += 256) {
@@ -100,25 +99,34 @@ __global__ void __launch_bounds__(256) rb_moment_kernel(const ReblockArgs a) {
     __syncthreads();
 #pragma unroll 4
     for (int r = 0; r < kMomStage; ++r) {
-      float u[TS], w[TS];
+      float u[TS];
+      uint64_t w2[TS / 2];
 #pragma unroll
       for (int i = 0; i < TS; i += 4) {
         const float4 x = *reinterpret_cast<const float4*>(&xs[r][ti * TS + i]);
         const float4 y = *reinterpret_cast<const float4*>(&xs[r][tj * TS + i]);
         u[i] = x.x; u[i + 1] = x.y; u[i + 2] = x.z; u[i + 3] = x.w;
-        w[i] = y.x; w[i + 1] = y.y; w[i + 2] = y.z; w[i + 3] = y.w;
+        w2[i / 2] = f2pack(y.x, y.y);
+        w2[i / 2 + 1] = f2pack(y.z, y.w);
       }
+      // packed f32x2 FMAs over column pairs (each half an ordinary fp32 FMA)
 #pragma unroll
-      for (int i = 0; i < TS; ++i)
+      for (int i = 0; i < TS; ++i) {
+        const uint64_t u2 = f2pack(u[i], u[i]);
 #pragma unroll
-        for (int j = 0; j < TS; ++j) acc[i][j] = fmaf(u[i], w[j], acc[i][j]);
+        for (int j = 0; j < TS / 2; ++j) acc[i][j] = ffma2(u2, w2[j], acc[i][j]);
+      }
     }
   }
   float* out = a.mpart + ((int64_t)bh * a.mchunks + blockIdx.x) * D * D;
 #pragma unroll
   for (int i = 0; i < TS; ++i)
 #pragma unroll
-    for (int j = 0; j < TS; ++j) out[(ti * TS + i) * D + tj * TS + j] = acc[i][j];
+    for (int j = 0; j < TS / 2; ++j) {
+      float lo, hi;
+      f2unpack(acc[i][j], lo, hi);
+      *reinterpret_cast<float2*>(&out[(ti * TS + i) * D + tj * TS + 2 * j]) = make_float2(lo, hi);
+    }
 }
 
 // M = (sum of the partials, chunk order) / n_q + ridge; its lower Cholesky
@@ -172,76 +180,94 @@ __global__ void __launch_bounds__(256) rb_factor_kernel(const ReblockArgs a) {
   for (int idx = tid; idx < D * D; idx += 256) L[idx] = (idx % D) <= (idx / D) ? M[(idx / D) * LD + idx % D] : 0.f;
 }
 
-// y = normalise(k L) for 64 video key rows per CTA: grid (ceil(n_v/64), B*H).
+// y = normalise(k L) for the video key rows: grid (ceil(n_v / (64 kWhTiles)), B*H).
+// A CTA loads L (D x D fp32) into shared memory once and whitens kWhTiles
+// tiles of 64 rows.  Warp w owns the 16 columns 16w .. 16w+15 of y, lane the
+// rows lane and lane+32 of the tile; L is lower triangular, so column j
+// gathers only i >= j and warp w's dot products start at i = 16w (the
+// skipped terms are exact zeros: the sums are those of the full loop).
+constexpr int kWhTiles = 8;
 template <int D>
 __global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
-  constexpr int LK = D + 4;   // padded key rows (16-byte aligned, rows on distinct banks)
+  constexpr int LK = D + 1;   // padded key rows: lanes read rows lane, lane+32 on distinct banks
+  constexpr int CPW = D / 8;  // columns per warp
   extern __shared__ __align__(16) float sm[];
-  float* Ls = sm;             // [D][D]
-  float* ks = sm + D * D;     // [64][LK]
-  const int tid = threadIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-  const int t0 = blockIdx.x * kBlock;
+  float* Ls = sm;                     // [D][D]
+  float* ks = sm + D * D;             // [64][LK]
+  float* ssq = ks + kBlock * LK;      // [8][64] partial squared norms
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const float* Lg = a.L + (int64_t)bh * D * D;
   for (int idx = tid * 4; idx < D * D; idx += 256 * 4)
     *reinterpret_cast<float4*>(&Ls[idx]) = *reinterpret_cast<const float4*>(&Lg[idx]);
   const __nv_bfloat16* kb = a.k + (int64_t)b * a.sb + (int64_t)h * a.sh;
-  for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
-    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4, t = t0 + r;
-    const float4 v = t < a.n_v ? ld_bf16x4(kb + (int64_t)(a.n_fix + t) * a.sn + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    *reinterpret_cast<float4*>(&ks[r * LK + c4]) = v;
-  }
-  __syncthreads();
-  // thread (rg = tid / 16, cq = tid % 16): rows 4 rg .. 4 rg + 3, columns CPT cq .. + CPT - 1;
-  // per head-dim step two (one) float4 loads of L and four broadcast loads of k feed 4 CPT FMAs
-  constexpr int CPT = D / 16;
-  const int rg = tid >> 4, cq = tid & 15;
-  float y[4][CPT];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) y[r][c] = 0.f;
-  for (int i = 0; i < D; ++i) {
-    float lv[CPT];
-#pragma unroll
-    for (int c = 0; c < CPT; c += 4) {
-      const float4 l4 = *reinterpret_cast<const float4*>(&Ls[i * D + CPT * cq + c]);
-      lv[c] = l4.x; lv[c + 1] = l4.y; lv[c + 2] = l4.z; lv[c + 3] = l4.w;
+  const int c0 = CPW * warp;
+  for (int it = 0; it < kWhTiles; ++it) {
+    const int t0 = (blockIdx.x * kWhTiles + it) * kBlock;
+    if (t0 >= a.n_v) break;   // uniform over the CTA
+    __syncthreads();          // the previous tile's ks and ssq are consumed (and L has landed)
+    for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
+      const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4, t = t0 + r;
+      const float4 v = t < a.n_v ? ld_bf16x4(kb + (int64_t)(a.n_fix + t) * a.sn + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float* dst = &ks[r * LK + c4];
+      dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
     }
+    __syncthreads();
+    uint64_t y2[2][CPW / 2];   // rows lane, lane+32; packed column pairs
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float kv = ks[(4 * rg + r) * LK + i];
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) y[r][c] = fmaf(kv, lv[c], y[r][c]);
+      for (int c = 0; c < CPW / 2; ++c) y2[r][c] = 0ull;
+    for (int i = c0; i < D; ++i) {
+      uint64_t l2[CPW / 2];
+#pragma unroll
+      for (int c = 0; c < CPW; c += 4) {   // broadcast: the whole warp reads the same columns
+        const float4 l4 = *reinterpret_cast<const float4*>(&Ls[i * D + c0 + c]);
+        l2[c / 2] = f2pack(l4.x, l4.y);
+        l2[c / 2 + 1] = f2pack(l4.z, l4.w);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float kv = ks[(lane + 32 * r) * LK + i];
+        const uint64_t k2 = f2pack(kv, kv);
+#pragma unroll
+        for (int c = 0; c < CPW / 2; ++c) y2[r][c] = ffma2(k2, l2[c], y2[r][c]);
+      }
     }
+    float y[2][CPW];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPW / 2; ++c) {
+        f2unpack(y2[r][c], y[r][2 * c], y[r][2 * c + 1]);
+        ss = fmaf(y[r][2 * c], y[r][2 * c], ss);
+        ss = fmaf(y[r][2 * c + 1], y[r][2 * c + 1], ss);
+      }
+      ssq[warp * kBlock + lane + 32 * r] = ss;
+    }
+    __syncthreads();
+    float* Yg = a.Y + ((int64_t)bh * a.n_v + t0) * D;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = lane + 32 * r;
+      float ss = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2) ss += ssq[w2 * kBlock + row];   // fixed order over the column groups
+      const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+      if (t0 + row < a.n_v) {
+        float* dst = Yg + (int64_t)row * D + c0;
+#pragma unroll
+        for (int c = 0; c < CPW; c += 4)
+          *reinterpret_cast<float4*>(dst + c) =
+              make_float4(y[r][c] * inv, y[r][c + 1] * inv, y[r][c + 2] * inv, y[r][c + 3] * inv);
+      }
+    }
+    if (tid < kBlock && t0 + tid < a.n_v) a.ord[(int64_t)bh * a.n_v + t0 + tid] = t0 + tid;
   }
-  float inv[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {   // row norms over the 16 lanes holding the row
-    float ss = 0.f;
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) ss = fmaf(y[r][c], y[r][c], ss);
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    inv[r] = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
-  }
-  __syncthreads();   // every thread has read ks
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < CPT; c += 4)
-      *reinterpret_cast<float4*>(&ks[(4 * rg + r) * LK + CPT * cq + c]) =
-          make_float4(y[r][c] * inv[r], y[r][c + 1] * inv[r], y[r][c + 2] * inv[r], y[r][c + 3] * inv[r]);
-  __syncthreads();
-  float* Yg = a.Y + ((int64_t)bh * a.n_v + t0) * D;
-  for (int idx = tid; idx < kBlock * (D / 4); idx += 256) {
-    const int rr = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
-    if (t0 + rr < a.n_v) *reinterpret_cast<float4*>(&Yg[(int64_t)rr * D + c4]) = *reinterpret_cast<const float4*>(&ks[rr * LK + c4]);
-  }
-  if (tid < kBlock && t0 + tid < a.n_v) a.ord[(int64_t)bh * a.n_v + t0 + tid] = t0 + tid;
 }
 
 // Sum of a per-lane float4 over the CTA's row slots into out[D] (fixed order).
-template <int D>
+template <int D, int W>
 __device__ __forceinline__ void rb_block_sum(float4 v, float4 (*red)[D / 4], float* out, float scale) {
   constexpr int LPR = D / 4, RPW = 32 / LPR;   // lanes per row, rows per warp
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -255,7 +281,7 @@ __device__ __forceinline__ void rb_block_sum(float4 v, float4 (*red)[D / 4], flo
   __syncthreads();
   if (threadIdx.x < LPR) {
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < kSplitWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const float4 t = red[w][threadIdx.x];
       s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
     }
@@ -295,10 +321,12 @@ __device__ __forceinline__ float rb_norm(const float* v, int D, float* s_tmp) {
 }
 
 // One level of the hierarchy: grid (2^lvl, B*H); group blockIdx.x of every head.
-template <int D>
-__global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockArgs a, int lvl, int iters) {
+template <int D, int T>
+__global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lvl, int iters) {
+  constexpr int kSplitThreads = T, kSplitWarps = T / 32;
   constexpr int LPR = D / 4, RPW = 32 / LPR, SLOTS = kSplitWarps * RPW;
   __shared__ __align__(16) float4 red[kSplitWarps][LPR];
+  __shared__ uint32_t wsum[8];
   __shared__ __align__(16) float mean[D], w[D], z[D];
   __shared__ uint32_t hist[256];
   __shared__ int s_int[4];
@@ -338,7 +366,7 @@ __global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockAr
   rows_pass([&](int, int id, float4 y) {
     if (id >= 0) { acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w; }
   });
-  rb_block_sum<D>(acc, red, mean, 1.f / (float)len);
+  rb_block_sum<D, kSplitWarps>(acc, red, mean, 1.f / (float)len);
   // start: the first row minus the mean, normalised (e_0 if that is zero)
   if (tid < D) w[tid] = Y[(int64_t)ord[0] * D + tid] - mean[tid];
   __syncthreads();
@@ -357,7 +385,7 @@ __global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockAr
       const float p = rb_row_dot<D>(c, wq);
       if (id >= 0) { zq.x = fmaf(c.x, p, zq.x); zq.y = fmaf(c.y, p, zq.y); zq.z = fmaf(c.z, p, zq.z); zq.w = fmaf(c.w, p, zq.w); }
     });
-    rb_block_sum<D>(zq, red, z, 1.f);
+    rb_block_sum<D, kSplitWarps>(zq, red, z, 1.f);
     const float nz = rb_norm(z, D, &s_tmp);
     if (!(nz > 0.f)) break;   // uniform
     if (tid < D) w[tid] = z[tid] / nz;
@@ -396,14 +424,24 @@ __global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockAr
       if (dig < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, d = 0;
-      for (; d < 255; ++d) {
-        if (cum + (int)hist[d] > want) break;
-        cum += (int)hist[d];
+    // the bin holding rank `want`: a parallel exclusive scan of the 256 counts
+    uint32_t c = 0u, incl = 0u;
+    if (tid < 256) {   // warps 0-7, whole warps
+      c = hist[tid];
+      incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      s_int[0] = d;
-      s_int[1] = want - cum;
+      if (lane == 31) wsum[warp] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t base = 0u;
+      for (int w2 = 0; w2 < warp; ++w2) base += wsum[w2];
+      const uint32_t excl = base + incl - c;
+      if (excl <= (uint32_t)want && (uint32_t)want < excl + c) { s_int[0] = tid; s_int[1] = want - (int)excl; }
     }
     __syncthreads();
     prefix |= (unsigned long long)s_int[0] << shift;
@@ -423,17 +461,16 @@ __global__ void __launch_bounds__(kSplitThreads) rb_split_kernel(const ReblockAr
     const uint32_t below = (1u << lane) - 1u;
     if (lane == 0) { hist[warp] = __popc(bl); hist[32 + warp] = __popc(bv & ~bl); }
     __syncthreads();
-    if (tid == 0) {
-      int sl = 0, sr = 0;
-      for (int w2 = 0; w2 < kSplitWarps; ++w2) {
-        const int l2 = (int)hist[w2], r2 = (int)hist[32 + w2];
-        hist[64 + w2] = (uint32_t)sl;
-        hist[96 + w2] = (uint32_t)sr;
-        sl += l2;
-        sr += r2;
+    if (warp == 0) {   // exclusive offsets of the warps' counts: one shuffle scan
+      const int l2 = lane < kSplitWarps ? (int)hist[lane] : 0, r2 = lane < kSplitWarps ? (int)hist[32 + lane] : 0;
+      int il = l2, ir = r2;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yl = __shfl_up_sync(0xffffffffu, il, o), yr = __shfl_up_sync(0xffffffffu, ir, o);
+        if (lane >= o) { il += yl; ir += yr; }
       }
-      s_int[2] = sl;
-      s_int[3] = sr;
+      if (lane < kSplitWarps) { hist[64 + lane] = (uint32_t)(il - l2); hist[96 + lane] = (uint32_t)(ir - r2); }
+      if (lane == 31) { s_int[2] = il; s_int[3] = ir; }
     }
     __syncthreads();
     if (valid) {
@@ -494,7 +531,8 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const int f128 = 128 * 129 * 4, w128 = (128 * 128 + 64 * 132) * 4, f64 = 64 * 65 * 4, w64 = (64 * 64 + 64 * 68) * 4;
+  const int f128 = 128 * 129 * 4, w128 = (128 * 128 + 64 * 129 + 8 * 64) * 4, f64 = 64 * 65 * 4,
+            w64 = (64 * 64 + 64 * 65 + 8 * 64) * 4;
   if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
     if ((e = cudaFuncSetAttribute(rb_factor_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, f128)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(rb_whiten_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, w128)) != cudaSuccess ||
@@ -504,7 +542,7 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
   if (a.n_v > 0) {
-    dim3 gm(a.mchunks, BH), gw((a.n_v + kBlock - 1) / kBlock, BH);
+    dim3 gm(a.mchunks, BH), gw((a.n_v + kBlock * kWhTiles - 1) / (kBlock * kWhTiles), BH);
     if (D == 128) {
       rb_moment_kernel<128><<<gm, 256, 0, st>>>(a);
       rb_factor_kernel<128><<<BH, 256, f128, st>>>(a);
@@ -518,8 +556,14 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
     const int levels = reblock_levels(a.n_v);
     for (int lvl = 0; lvl < levels; ++lvl) {
       dim3 gs(1u << lvl, BH);
-      if (D == 128) rb_split_kernel<128><<<gs, kSplitThreads, 0, st>>>(a, lvl, iters);
-      else rb_split_kernel<64><<<gs, kSplitThreads, 0, st>>>(a, lvl, iters);
+      const bool wide = (a.n_v >> lvl) > 4096;   // large groups: 1024 threads; small ones: 256, more CTAs per SM
+      if (D == 128) {
+        if (wide) rb_split_kernel<128, 1024><<<gs, 1024, 0, st>>>(a, lvl, iters);
+        else rb_split_kernel<128, 256><<<gs, 256, 0, st>>>(a, lvl, iters);
+      } else {
+        if (wide) rb_split_kernel<64, 1024><<<gs, 1024, 0, st>>>(a, lvl, iters);
+        else rb_split_kernel<64, 256><<<gs, 256, 0, st>>>(a, lvl, iters);
+      }
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
