@@ -219,10 +219,10 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
         out = sol_ref.sol_forward(q, k, v, prefix=w.prefix, bq=64 if w.compressed else 128,
                                   topk_ratio=w.topk_ratio, compressed=w.compressed,
                                   log_mass_bias_on=int(w.log_mass_bias) == 1, reweight_on=int(w.log_mass_bias) == 2,
-                                  reblock=w.reblock)
+                                  reblock=w.reblock, qk_int8=w.qk_int8)
     else:
         out = sol_ref.sol_forward(q, k, v, tau=w.tau, prefix=w.prefix, log_mass_bias_on=int(w.log_mass_bias) == 1,
-                                  reweight_on=int(w.log_mass_bias) == 2, reblock=w.reblock)
+                                  reweight_on=int(w.log_mass_bias) == 2, reblock=w.reblock, qk_int8=w.qk_int8)
     dt = time.perf_counter() - t0
     nk = sol_ref.block_rows(w.N, 64)
     nq = sol_ref.block_rows(w.N, 128 if (w.topk_ratio is not None and not w.compressed) else 64)
@@ -232,7 +232,7 @@ def oracle_sample(w: synth.Workload, heads, b_offset=0):
 
 
 def routing_config(w: synth.Workload) -> dict:
-    rb = {"reblock": True} if w.reblock else {}
+    rb = ({"reblock": True} if w.reblock else {}) | ({"qk": "int8 residual keys"} if w.qk_int8 else {})
     if w.topk_ratio is None:
         return {"routing": "threshold", **rb}
     if w.compressed:
@@ -303,9 +303,10 @@ def run_ours(args, w):
                    b_offset=0 if by_heads else shard_b_offset(rank, w))
     q, k, v = (h.to(dev) for h in host)
     p = sol.make_params(w.B, w.N, Hr, w.D, tau=w.tau, prefix_len=w.prefix, log_mass_bias=w.log_mass_bias,
-                        topk_ratio=w.topk_ratio, compressed=w.compressed)
+                        topk_ratio=w.topk_ratio, compressed=w.compressed, qk_int8=w.qk_int8)
     stream = torch.cuda.current_stream()
-    launches_per_step = (3 if w.log_mass_bias else 1) + 3 + 2   # pool (+ anchor, K/V), route + scan + compact, plan + attention
+    # pool (+ anchor, K/V; + residual key codes), route + scan + compact, plan + attention
+    launches_per_step = (3 if w.log_mass_bias else 1) + (1 if w.qk_int8 else 0) + 3 + 2
     if w.reblock:
         # the adaptive partition, then the Sol passes on head-major copies in its order
         rb = sol.alloc_reblock(p, dev)
@@ -492,6 +493,8 @@ def main():
                     help="Top-K routing (the SLA variant: 128-row query blocks, no centroid terms)")
     ap.add_argument("--compressed", action="store_true",
                     help="with --topk-ratio: keep the compressed branch (64-row blocks, sink, centroid terms)")
+    ap.add_argument("--qk-int8", action="store_true",
+                    help="exact logits from INT8 query codes and INT8 per-block residual key codes")
     ap.add_argument("--reblock", action="store_true",
                     help="order the rows by the adaptive partition first (sol_reblock, gathers, scatter)")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
@@ -515,15 +518,17 @@ def main():
         ap.error("--topk-ratio takes no tau, and centroid options only with --compressed")
     if args.compressed and args.topk_ratio is None:
         ap.error("--compressed needs --topk-ratio")
-    if args.tau is not None or mode or args.topk_ratio is not None or args.reblock:
+    if args.tau is not None or mode or args.topk_ratio is not None or args.reblock or args.qk_int8:
         import dataclasses
         w = dataclasses.replace(w, tau=w.tau if args.tau is None else args.tau, log_mass_bias=mode,
                                 topk_ratio=args.topk_ratio, compressed=args.compressed, reblock=args.reblock,
+                                qk_int8=args.qk_int8,
                                 name=w.name + (f"_tau{args.tau:g}" if args.tau is not None else "")
                                      + synth.mode_suffix(mode)
                                      + (f"_topk{args.topk_ratio:g}" if args.topk_ratio is not None else "")
                                      + ("_compressed" if args.compressed else "")
-                                     + ("_reblock" if args.reblock else ""))
+                                     + ("_reblock" if args.reblock else "")
+                                     + ("_int8" if args.qk_int8 else ""))
     if args.impl == "reference":
         run_reference(args, w)
     else:

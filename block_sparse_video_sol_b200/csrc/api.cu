@@ -96,6 +96,8 @@ sol_status validate(const sol_params* p) {
   if (!(p->scale >= 0.f) || isinf(p->scale)) return fail(SOL_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->prefix_len < 0 || p->prefix_len > p->N) return fail(SOL_ERR_INVALID_ARG, "prefix_len %d outside [0, N]", p->prefix_len);
   if (p->log_mass_bias < 0 || p->log_mass_bias > 2) return fail(SOL_ERR_INVALID_ARG, "log_mass_bias must be 0, 1 or 2");
+  if (p->qk_int8 != 0 && p->qk_int8 != 1) return fail(SOL_ERR_INVALID_ARG, "qk_int8 must be 0 or 1");
+  if (p->qk_int8 && p->D != 128) return fail(SOL_ERR_UNSUPPORTED, "qk_int8 needs head dim 128 (got %d)", p->D);
   const int64_t nb = (p->N + kBlock - 1) / kBlock;
   if (nb > kMaxKeyBlocks) return fail(SOL_ERR_UNSUPPORTED, "N=%d exceeds the supported %d rows", p->N, kMaxKeyBlocks * kBlock);
   if ((int64_t)p->B * p->H * nb * nb >= (int64_t)INT32_MAX)
@@ -155,6 +157,18 @@ sol_status sol_workspace_offsets(const sol_params* p, int64_t offsets[8]) {
   return SOL_OK;
 }
 
+sol_status sol_workspace_int8_offsets(const sol_params* p, int64_t offsets[3]) {
+  sol_status s = validate(p);
+  if (s != SOL_OK) return s;
+  if (!p->qk_int8) return fail(SOL_ERR_INVALID_ARG, "sol_workspace_int8_offsets: qk_int8 is 0");
+  if (!offsets) return fail(SOL_ERR_INVALID_ARG, "offsets is NULL");
+  const WsLayout L = ws_layout(*p);
+  offsets[0] = (int64_t)L.kcode;
+  offsets[1] = (int64_t)L.ksig;
+  offsets[2] = (int64_t)L.kmean16;
+  return SOL_OK;
+}
+
 int64_t sol_col_capacity(const sol_params* p) {
   if (validate(p) != SOL_OK || empty(p)) return 0;
   const int64_t nb = (p->N + kBlock - 1) / kBlock;
@@ -185,6 +199,7 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
   a.qbar = at<float>(ws, L.qbar); a.kbar = at<float>(ws, L.kbar);
   a.kbar16 = at<__nv_bfloat16>(ws, L.kbar16); a.vbar16 = at<__nv_bfloat16>(ws, L.vbar16);
   a.cbias = at<float>(ws, L.cbias); a.anchor = at<float>(ws, L.anchor);
+  a.kcode = at<int8_t>(ws, L.kcode); a.ksig = at<float>(ws, L.ksig); a.kmean16 = at<__nv_bfloat16>(ws, L.kmean16);
   cudaError_t e;
   if (p->routing == 1) {   // Top-K routing needs no V centroids
     a.tensor_mask = 3; a.with_bias = 0;
@@ -210,6 +225,7 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
     a.tensor_mask = 2; a.with_bias = 1;
     if ((e = launch_pool(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (k + bias)");
   }
+  if (p->qk_int8 && (e = launch_quant_k(a, p->D, st)) != cudaSuccess) return cuda_fail(e, "sol_pool launch (k residual codes)");
   return SOL_OK;
 }
 
@@ -262,6 +278,8 @@ sol_status sol_attn_fwd(const sol_params* p, const void* q, const void* k, const
   a.B = p->B; a.N = p->N; a.H = p->H; a.nqb = L.nqb; a.nkb = L.nkb;
   a.scale = eff_scale(p);
   a.centroids = p->routing == 1 ? 0 : 1;
+  a.qk_int8 = p->qk_int8;
+  a.kcode = at<int8_t>(ws, L.kcode); a.ksig = at<float>(ws, L.ksig); a.kmean16 = at<__nv_bfloat16>(ws, L.kmean16);
   cudaError_t e = launch_attn(a, p->D, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sol_attn_fwd launch");
   return SOL_OK;

@@ -100,12 +100,19 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxWords = kMaxKeyBlocks / 32;
 constexpr int kMaxCentTiles = kMaxKeyBlocks / 128;
 
-template <int D>
+template <int D, bool I8 = false>
 struct Cfg {
   static constexpr int kChunks = D / 64;               // 128-byte column chunks per row
   static constexpr int kChunkBytes = 128 * 128;        // one chunk of a 128-row tile
   static constexpr int kTileBytes = 128 * D * 2;       // Q, K or V tile of 128 rows
-  static constexpr int kSmemTiles = kTileBytes * (1 + kKStages + kVStages);
+  // INT8 QK: the query codes (128 rows x D bytes, one 128-byte chunk at D = 128); an exact
+  // K stage holds the residual codes of the tile's two key blocks and, after them, the
+  // two blocks' bf16 means (the mean term's keys)
+  static constexpr int kQ8Bytes = I8 ? 128 * D : 0;
+  static constexpr int kK8Bytes = 128 * D;
+  static constexpr int kKMeanOff = kK8Bytes;
+  static constexpr int kSmemTiles = kTileBytes * (1 + kKStages + kVStages) + kQ8Bytes;
+  static_assert(!I8 || (D == 128 && kKMeanOff + 2 * D * 2 <= kTileBytes), "INT8 stage layout");
 };
 
 struct Bars {
@@ -113,8 +120,11 @@ struct Bars {
   uint64_t k_full[kKStages], v_full[kVStages];
   uint64_t s_full[3], p_full[3], o_done[2], final_mma;
   uint64_t ref_full[kSoftmaxGroups][4];   // [group][warp]: the group's step published its reference max
+  uint64_t q8_ready;                      // INT8 QK: the query codes are in shared memory (softmax threads)
+  uint64_t kb_done[kKStages];             // INT8 QK: the softmax has read the stage's block means (4 warps)
 };
 
+template <bool I8>
 struct Extra {
   Bars bar;
   uint32_t tmem_base;
@@ -124,11 +134,14 @@ struct Extra {
   int cent[kMaxCentTiles];           // centroid tiles to visit
   int list[kMaxKeyBlocks];           // union entries: j | needA << 16 | needB << 17
   int cent_live[kMaxCentTiles][2][2];           // [slot][half][64-column half]: any live centroid
-  alignas(16) float cent_add[kMaxCentTiles][2][128];        // log2-unit offset of each centroid column, -inf if masked
+  // log2-unit offset of each centroid column, -inf if masked (the INT8 variant, short of
+  // shared memory, computes it from cbias and the bitmaps instead)
+  alignas(16) float cent_add[I8 ? 1 : kMaxCentTiles][2][128];
+  float qsig[I8 ? 128 : 1];                     // INT8 QK: each row's query scale
   alignas(16) float tail_add[64];                         // 0 for valid rows of the last key block, -inf beyond N
   float2 ml[kSoftmaxGroups][128];               // per warpgroup and row: (reference, partial sum)
   float m_ref[128];                             // per row: reference max after the latest step (log2 units)
-  float cbias[kMaxKeyBlocks];                   // this (b, h)'s centroid logit biases, prefetched
+  alignas(16) float cbias[kMaxKeyBlocks];       // this (b, h)'s centroid logit biases, prefetched
 #ifdef SOL_TRACE
   unsigned int trace[kTraceSlots * kTraceSteps];
 #endif
@@ -151,6 +164,16 @@ __device__ __forceinline__ void mma_ss_w(uint32_t d, uint64_t a, uint64_t b, uin
   asm volatile("{ .reg .pred p, e; setp.ne.b32 p, %4, 0; elect.sync _|e, 0xffffffff;\n"
                "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
                :: "r"(d), "l"(a), "l"(b), "r"(id), "r"(acc));
+}
+// INT8 x INT8 -> s32 (both operands signed), shared-memory descriptors, same warp-wide form.
+__device__ __forceinline__ void mma_ss_i8_w(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile("{ .reg .pred p, e; setp.ne.b32 p, %4, 0; elect.sync _|e, 0xffffffff;\n"
+               "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p; }"
+               :: "r"(d), "l"(a), "l"(b), "r"(id), "r"(acc));
+}
+// Instruction descriptor: s8 x s8 -> s32, M x N, both K-major.
+__host__ __device__ constexpr uint32_t idesc_s8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __device__ __forceinline__ void mma_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
   asm volatile("{ .reg .pred p, e; setp.ne.b32 p, %4, 0; elect.sync _|e, 0xffffffff;\n"
@@ -193,6 +216,20 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Exact float of an s32 stored in a float register (|S| < 2^22): 1.5 * 2^23 + S is a
+// float of the same bits plus 0x4B400000, from which 1.5 * 2^23 subtracts exactly.
+__device__ __forceinline__ float i2f_exact(float bits) {
+  return __int_as_float(__float_as_int(bits) + 0x4B400000) - 12582912.f;
+}
+__device__ __forceinline__ void bf16x8_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -321,19 +358,21 @@ __global__ void __launch_bounds__(kPlanWarps * 32) plan_kernel(const AttnArgs a,
   }
 }
 
-template <int D>
+template <int D, bool I8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mkb,
-               const __grid_constant__ CUtensorMap mvb, const TcParams prm) {
-  using C = Cfg<D>;
+               const __grid_constant__ CUtensorMap mvb, const __grid_constant__ CUtensorMap mk8,
+               const TcParams prm) {
+  using C = Cfg<D, I8>;
   const AttnArgs& a = prm.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::kTileBytes;
   uint8_t* sV = sK + kKStages * C::kTileBytes;
-  Extra& x = *reinterpret_cast<Extra*>(sV + kVStages * C::kTileBytes);
+  uint8_t* sQ8 = sV + kVStages * C::kTileBytes;   // INT8 QK: query codes (SW128, 128-byte rows)
+  Extra<I8>& x = *reinterpret_cast<Extra<I8>*>(sQ8 + C::kQ8Bytes);
   Bars& bar = x.bar;
   volatile int* abort_flag = &x.abort_flag;
 
@@ -356,6 +395,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     for (int g = 0; g < kSoftmaxGroups; ++g)
       for (int s = 0; s < 4; ++s) mbar_init(&bar.ref_full[g][s], 32);
     mbar_init(&bar.final_mma, 1);
+    if (I8) {
+      mbar_init(&bar.q8_ready, 128 * kSoftmaxGroups);
+      for (int s = 0; s < kKStages; ++s) mbar_init(&bar.kb_done[s], 4);
+    }
     x.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     // Q does not depend on the routing: its load starts at once
@@ -410,7 +453,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     for (int q = 0; q < 4; ++q) {
       const int c = lane + 32 * q, j = 128 * x.cent[slot] + c;
       const bool live = x.present[hf] && j < a.nkb && !((x.sel[hf][j >> 5] >> (j & 31)) & 1u);
-      x.cent_add[slot][hf][c] = live ? x.cbias[j] * kLog2e : -INFINITY;
+      if (!I8) x.cent_add[slot][hf][c] = live ? x.cbias[j] * kLog2e : -INFINITY;
       if (q < 2) l0 |= live; else l1 |= live;
     }
     const bool any0 = __any_sync(0xffffffffu, l0), any1 = __any_sync(0xffffffffu, l1);
@@ -455,16 +498,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         uint64_t* empty = is_k ? &bar.s_full[s] : &bar.o_done[s];
         uint64_t* full = is_k ? &bar.k_full[s] : &bar.v_full[s];
         if (!(ok = wait_bar(empty, (n & 1) ^ 1, abort_flag, a.status))) break;
+        // INT8: the stage's block means of step t-3 must also have been read by the softmax
+        if (I8 && is_k && !(ok = wait_bar(&bar.kb_done[s], (n & 1) ^ 1, abort_flag, a.status))) break;
         SOL_TRACE_AT(is_k ? 7 : 8, t);
-        mbar_expect_tx(full, C::kTileBytes);
-        ++nl;
         uint8_t* dst = ring + s * C::kTileBytes;
-        for (int c = 0; c < C::kChunks; ++c) {
-          if (ct < 0) {
-            tma_load_4d(dst + c * C::kChunkBytes, m4, c * 64, h, 64 * j0, b, full);
-            tma_load_4d(dst + c * C::kChunkBytes + C::kChunkBytes / 2, m4, c * 64, h, 64 * j1, b, full);
-          } else {
-            tma_load_3d(dst + c * C::kChunkBytes, m3, c * 64, 128 * ct, (int)bh, full);
+        ++nl;
+        if (I8 && is_k && ct < 0) {
+          // residual codes of the two key blocks (64 rows x 128 bytes each) and their bf16 means
+          mbar_expect_tx(full, C::kK8Bytes + 2 * D * 2);
+          tma_load_3d(dst, &mk8, 0, 64 * j0, (int)bh, full);
+          tma_load_3d(dst + C::kK8Bytes / 2, &mk8, 0, 64 * j1, (int)bh, full);
+          bulk_load(dst + C::kKMeanOff, a.kmean16 + ((int64_t)bh * a.nkb + j0) * D, D * 2, full);
+          bulk_load(dst + C::kKMeanOff + D * 2, a.kmean16 + ((int64_t)bh * a.nkb + j1) * D, D * 2, full);
+        } else {
+          mbar_expect_tx(full, C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c) {
+            if (ct < 0) {
+              tma_load_4d(dst + c * C::kChunkBytes, m4, c * 64, h, 64 * j0, b, full);
+              tma_load_4d(dst + c * C::kChunkBytes + C::kChunkBytes / 2, m4, c * 64, h, 64 * j1, b, full);
+            } else {
+              tma_load_3d(dst + c * C::kChunkBytes, m3, c * 64, 128 * ct, (int)bh, full);
+            }
           }
         }
       }
@@ -498,15 +552,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       const uint64_t vd0 = sdesc(smem_u32(sV), C::kChunkBytes, 1024);
       int kst = 0, vst = 0, sq = 0, sp = 0;        // K / V ring stages, S buffers of the next QK / PV
       uint32_t kph = 0, vph = 0, pph = 0;          // their phase parities
-      // QK(g) into S_sq from K stage kst (K must have landed)
+      // QK(g) into S_sq from K stage kst (K must have landed); with INT8 QK the exact
+      // tiles (the first n_ex) run s8 x s8 -> s32 on the query and residual key codes
+      // (K = 32 bytes per MMA, one 128-byte chunk per row), the centroid tiles bf16
+      int nqk = 0;
       auto qk = [&]() {
         const uint64_t kd = kd0 + (uint64_t)kst * kStageD;
         const uint32_t d = tmem + 128 * sq;
+        if (I8 && nqk < n_ex) {
+          constexpr uint32_t id_qk8 = idesc_s8(128, 128);
+          const uint64_t q8d = sdesc(smem_u32(sQ8), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < NQ; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
-          mma_ss_w(d, qd + off, kd + off, id_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_ss_i8_w(d, q8d + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), id_qk8, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < NQ; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
+            mma_ss_w(d, qd + off, kd + off, id_qk, kk > 0 ? 1u : 0u);
+          }
         }
+        ++nqk;
         mma_commit_w(&bar.s_full[sq]);   // also frees K stage kst (== sq)
         if (++kst == kKStages) { kst = 0; kph ^= 1u; }
         sq = sq == 2 ? 0 : sq + 1;
@@ -533,6 +599,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         return r;
       };
       bool ok = __all_sync(0xffffffffu, wait_bar(&bar.q_full, 0, abort_flag, a.status));
+      if (I8 && ok) {   // the softmax quantizes the query tile first
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.q8_ready, 0, abort_flag, a.status));
+        fence_after();
+      }
       const int nq0 = T < 3 ? T : 3;
       for (int g = 0; g < nq0 && ok; ++g) {
         if ((ok = wait_k())) qk();
@@ -595,10 +665,127 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     bool ok = true;
     const int bb = w;                         // S buffer of every step of this group: t % 3 = w
     static_assert(kSoftmaxGroups == 3, "one softmax warpgroup per S buffer");
+    float sigq = 0.f;                         // INT8 QK: this row's query scale
+    if constexpr (I8) {
+      // Quantize the query tile once: every softmax thread takes its row's max |q| (exact
+      // on bf16 values), sigma_q = max / 127, and writes the codes rint(q * (1 / sigma_q))
+      // of the 16-byte code units u = w, w + 3, ... of its row into the SW128 code tile.
+      ok = __all_sync(0xffffffffu, wait_bar(&bar.q_full, 0, abort_flag, a.status));
+      float amax = 0.f;
+      if (ok) {
+        for (int c = 0; c < C::kChunks; ++c) {
+#pragma unroll
+          for (int pu = 0; pu < 8; ++pu) {
+            float f[8];
+            bf16x8_f32(*reinterpret_cast<const uint4*>(sQ + c * C::kChunkBytes + r * 128 + pu * 16), f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+          }
+        }
+      }
+      const float sg = amax / 127.f;
+      const float inv = sg > 0.f ? 1.f / sg : 0.f;
+      if (ok) {
+        for (int u = w; u < D / 16; u += kSoftmaxGroups) {   // code unit u: dims 16u .. 16u+15
+          const int c = u >> 2, lu0 = 2 * (u & 3);           // its 64-dim chunk, first bf16 unit there
+          float f[16];
+          bf16x8_f32(*reinterpret_cast<const uint4*>(sQ + c * C::kChunkBytes + r * 128 + ((lu0 ^ (r & 7)) << 4)), f);
+          bf16x8_f32(*reinterpret_cast<const uint4*>(sQ + c * C::kChunkBytes + r * 128 + (((lu0 + 1) ^ (r & 7)) << 4)),
+                     f + 8);
+          uint32_t wd[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int qc = sg > 0.f ? min(127, max(-127, __float2int_rn(__fmul_rn(f[4 * q4 + i], inv)))) : 0;
+              word |= (uint32_t)(qc & 0xff) << (8 * i);
+            }
+            wd[q4] = word;
+          }
+          *reinterpret_cast<uint4*>(sQ8 + r * 128 + ((u ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+      }
+      if (w == 0) x.qsig[r] = sg;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the codes feed the tensor cores
+      mbar_arrive(&bar.q8_ready);
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bar.q8_ready, 0, abort_flag, a.status));
+      sigq = x.qsig[r];
+    }
     for (int t = w; t < T && ok; t += kSoftmaxGroups) {
 #ifdef SOL_TRACE
       if (tracer) SOL_TRACE_AT(15, t);
 #endif
+      // which 64-column halves of this S tile the row uses, and their additive offsets
+      bool need0, need1;
+      const float *add0 = nullptr, *add1 = nullptr;
+      const int slot = t - n_ex;                // centroid tiles: their slot
+      int j0 = 0, j1 = 0;                       // exact tiles: the two key blocks
+      if (t < n_ex) {
+        const int e0 = x.list[2 * t];
+        const int e1 = (2 * t + 1 < x.n_union) ? x.list[2 * t + 1] : -1;
+        j0 = e0 & 0xffff;
+        j1 = e1 >= 0 ? (e1 & 0xffff) : j0;
+        need0 = present && ((e0 >> (16 + hf)) & 1);
+        need1 = present && e1 >= 0 && ((e1 >> (16 + hf)) & 1);
+        add0 = (j0 == a.nkb - 1) ? x.tail_add : nullptr;
+        add1 = (e1 >= 0 && j1 == a.nkb - 1) ? x.tail_add : nullptr;
+      } else {
+        need0 = x.cent_live[slot][hf][0] != 0;
+        need1 = x.cent_live[slot][hf][1] != 0;
+        if (!I8) {
+          add0 = x.cent_add[slot][hf];
+          add1 = x.cent_add[slot][hf] + 64;
+        }
+      }
+      // INT8 exact tile: each half's logit is cc * S_int + mm (log2 units), with
+      // cc = s log2(e) sigma_q sigma_j and mm = s log2(e) q . kmean16_j, the mean term
+      // computed here, before S is ready, from the stage's bf16 block means
+      float cc0 = 0.f, cc1 = 0.f, mm0 = 0.f, mm1 = 0.f;
+      if constexpr (I8) {
+        // Every step, centroid tiles included, waits for its stage's load before it
+        // releases the stage: the producer has then passed its wait for this step, so
+        // the kb_done phases never run two ahead of it (its parity wait could not tell
+        // the phase it waits for from the one after next).
+        const int ks = t % kKStages;
+        ok = __all_sync(0xffffffffu, wait_bar(&bar.k_full[ks], (t / kKStages) & 1, abort_flag, a.status));
+        if (!ok) break;
+        if (t < n_ex) {
+          if (need0 || need1) {
+            const uint8_t* km = sK + ks * C::kTileBytes + C::kKMeanOff;
+            // packed f32x2 FMAs over dim pairs: two interleaved partial sums per block
+            uint64_t a0 = 0ull, a1 = 0ull;
+            auto pair = [](uint32_t w) { return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+#pragma unroll 4
+            for (int u = 0; u < D / 8; ++u) {   // 8 dims per 16-byte unit
+              const int c = u >> 3, lu = u & 7;
+              const uint4 qv = *reinterpret_cast<const uint4*>(sQ + c * C::kChunkBytes + r * 128 + ((lu ^ (r & 7)) << 4));
+              const uint4 k0 = *reinterpret_cast<const uint4*>(km + u * 16);
+              const uint4 k1 = *reinterpret_cast<const uint4*>(km + D * 2 + u * 16);
+              const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, k0w[4] = {k0.x, k0.y, k0.z, k0.w},
+                             k1w[4] = {k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint64_t q2 = pair(qw[e]);
+                a0 = ffma2(q2, pair(k0w[e]), a0);
+                a1 = ffma2(q2, pair(k1w[e]), a1);
+              }
+            }
+            float d0, d1, lo, hi;
+            f2unpack(a0, lo, hi);
+            d0 = lo + hi;
+            f2unpack(a1, lo, hi);
+            d1 = lo + hi;
+            const float sq = sl2 * sigq;
+            cc0 = sq * __ldg(a.ksig + bh * a.nkb + j0);
+            cc1 = sq * __ldg(a.ksig + bh * a.nkb + j1);
+            mm0 = sl2 * d0;
+            mm1 = sl2 * d1;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.kb_done[ks]);   // the stage may be reloaded (after QK(t) too)
+      }
       ok = __all_sync(0xffffffffu, wait_bar(&bar.s_full[bb], (t / 3) & 1, abort_flag, a.status));
       if (!ok) break;
       fence_after();
@@ -607,23 +794,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
       if (lane == 0) SOL_TRACE_AT(20 + sub, t);
 #endif
       const uint32_t s_addr = lane_addr + 128 * bb;   // S(t); P(t) is written over its first 64 columns
-      // which 64-column halves of this S tile the row uses, and their additive offsets
-      bool need0, need1;
-      const float *add0, *add1;
-      if (t < n_ex) {
-        const int e0 = x.list[2 * t];
-        const int e1 = (2 * t + 1 < x.n_union) ? x.list[2 * t + 1] : -1;
-        need0 = present && ((e0 >> (16 + hf)) & 1);
-        need1 = present && e1 >= 0 && ((e1 >> (16 + hf)) & 1);
-        add0 = ((e0 & 0xffff) == a.nkb - 1) ? x.tail_add : nullptr;
-        add1 = (e1 >= 0 && (e1 & 0xffff) == a.nkb - 1) ? x.tail_add : nullptr;
-      } else {
-        const int slot = t - n_ex;
-        need0 = x.cent_live[slot][hf][0] != 0;
-        need1 = x.cent_live[slot][hf][1] != 0;
-        add0 = x.cent_add[slot][hf];
-        add1 = x.cent_add[slot][hf] + 64;
-      }
+      const bool i8x = I8 && t < n_ex;                // this S tile holds s32 INT8 products
+      const bool i8c = I8 && t >= n_ex;               // INT8 variant, centroid tile: offsets computed here
+      // centroid-column offsets of columns col .. col+3 of half hh (INT8 variant: no table)
+      auto coff4 = [&](int hh, int col) {
+        const int j = 128 * x.cent[slot < 0 ? 0 : slot] + 64 * hh + col;
+        const float4 cb = *reinterpret_cast<const float4*>(&x.cbias[j]);
+        const uint32_t bits = x.sel[hf][j >> 5] >> (j & 31);
+        const bool pr = present;
+        float4 o;
+        o.x = (pr && j + 0 < a.nkb && !(bits & 1u)) ? cb.x * kLog2e : -INFINITY;
+        o.y = (pr && j + 1 < a.nkb && !(bits & 2u)) ? cb.y * kLog2e : -INFINITY;
+        o.z = (pr && j + 2 < a.nkb && !(bits & 4u)) ? cb.z * kLog2e : -INFINITY;
+        o.w = (pr && j + 3 < a.nkb && !(bits & 8u)) ? cb.w * kLog2e : -INFINITY;
+        return o;
+      };
       // pass 1: the tile's row max (log2 units), one 64-column half at a time;
       // pass 2 below reloads each half for its exponentials (the register
       // budget of three softmax warpgroups holds half a row, not a whole one)
@@ -636,12 +821,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         tmem_ld32(s_addr + 64 * hh, v);
         tmem_ld32(s_addr + 64 * hh + 32, v + 32);
         tmem_wait_ld();
-        if (ad) {
+        if (i8x) {
+          const float cc = hh ? cc1 : cc0, mm = hh ? mm1 : mm0;
+          if (ad) {   // the tail block: per column, with its -inf past N
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], fmaf(i2f_exact(v[c]), cc, mm) + ad[c]);
+          } else {    // cc >= 0: the largest code product gives the largest logit
+            int im = INT_MIN;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) im = max(im, __float_as_int(v[c]));
+            m4[0] = fmaxf(m4[0], fmaf((float)im, cc, mm));
+          }
+        } else if (ad || i8c) {
           const uint64_t sl22 = f2pack(sl2, sl2);
           const float4* ad4 = reinterpret_cast<const float4*>(ad);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float4 o = ad4[c];
+            const float4 o = i8c ? coff4(hh, 4 * c) : ad4[c];
             f2unpack(ffma2(f2pack(v[4 * c], v[4 * c + 1]), sl22, f2pack(o.x, o.y)), v[4 * c], v[4 * c + 1]);
             f2unpack(ffma2(f2pack(v[4 * c + 2], v[4 * c + 3]), sl22, f2pack(o.z, o.w)), v[4 * c + 2], v[4 * c + 3]);
             m4[c & 3] = fmax3(m4[c & 3], v[4 * c], v[4 * c + 1]);
@@ -688,17 +884,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
           tmem_ld32(s_addr + 64 * hh, v);
           tmem_ld32(s_addr + 64 * hh + 32, v + 32);
           tmem_wait_ld();
-          if (ad) {   // offset logits in log2 units, as in pass 1
-            const uint64_t sl22 = f2pack(sl2, sl2);
-            const float2* ad2 = reinterpret_cast<const float2*>(ad);
+          uint64_t mul2, nb2;
+          if (i8x) {   // s32 products: exact float, then cc * S + mm (+ tail offset) - base
+            const float cc = hh ? cc1 : cc0, mm = hh ? mm1 : mm0;
+            const uint64_t cc2 = f2pack(cc, cc), mb2 = f2pack(mm - base, mm - base);
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float2 o = ad2[c];
-              f2unpack(ffma2(f2pack(v[2 * c], v[2 * c + 1]), sl22, f2pack(o.x, o.y)), v[2 * c], v[2 * c + 1]);
+              f2unpack(ffma2(f2pack(i2f_exact(v[2 * c]), i2f_exact(v[2 * c + 1])), cc2, mb2), v[2 * c], v[2 * c + 1]);
+              if (ad) { v[2 * c] += ad[2 * c]; v[2 * c + 1] += ad[2 * c + 1]; }
             }
+            mul2 = f2pack(1.f, 1.f);
+            nb2 = 0ull;   // packed (0, 0): base already taken off
+          } else {
+            if (ad || i8c) {   // offset logits in log2 units, as in pass 1
+              const uint64_t sl22 = f2pack(sl2, sl2);
+              const float2* ad2 = reinterpret_cast<const float2*>(ad);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                float2 o;
+                if (i8c) {
+                  const float4 o4 = coff4(hh, 4 * (c >> 1));
+                  o = (c & 1) ? make_float2(o4.z, o4.w) : make_float2(o4.x, o4.y);
+                } else {
+                  o = ad2[c];
+                }
+                f2unpack(ffma2(f2pack(v[2 * c], v[2 * c + 1]), sl22, f2pack(o.x, o.y)), v[2 * c], v[2 * c + 1]);
+              }
+            }
+            const float mul = (ad != nullptr || i8c) ? 1.f : sl2;   // offset logits are in log2 units
+            mul2 = f2pack(mul, mul);
+            nb2 = f2pack(-base, -base);
           }
-          const float mul = ad != nullptr ? 1.f : sl2;   // offset logits are in log2 units
-          const uint64_t mul2 = f2pack(mul, mul), nb2 = f2pack(-base, -base);
           uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -802,9 +1018,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 }
 
 // ---- host side: tensor maps and launch ------------------------------------------------------------
-template <int D>
+static_assert(1024 + Cfg<128, false>::kSmemTiles + sizeof(Extra<false>) <= 232448, "bf16 variant: shared memory");
+static_assert(1024 + Cfg<128, true>::kSmemTiles + sizeof(Extra<true>) <= 232448, "INT8 variant: shared memory");
+
+template <int D, bool I8>
 cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mkb, mvb;
+  CUtensorMap mq, mk, mv, mkb, mvb, mk8;
   const cuuint64_t bstride = (cuuint64_t)(a.B > 1 ? a.sb : (int64_t)a.N * a.sn) * 2;
   const cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)a.H, (cuuint64_t)a.N, (cuuint64_t)a.B};
   const cuuint64_t str4[3] = {(cuuint64_t)a.sh * 2, (cuuint64_t)a.sn * 2, bstride};
@@ -816,12 +1035,20 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, 4, dims4, str4, box4, kSw128) || !make_map(&mkb, a.kbar16, 3, dims3, str3, box3, kSw128) ||
       !make_map(&mvb, a.vbar16, 3, dims3, str3, box3, kSw128))
     return cudaErrorInvalidValue;
+  mk8 = mk;   // unused by the bf16 variant
+  if (I8) {   // residual key codes, head-major [B*H, N, D] bytes: 64-row boxes of 128-byte rows
+    const cuuint64_t dims8[3] = {(cuuint64_t)D, (cuuint64_t)a.N, (cuuint64_t)a.B * a.H};
+    const cuuint64_t str8[2] = {(cuuint64_t)D, (cuuint64_t)a.N * D};
+    const cuuint32_t box8[3] = {(cuuint32_t)D, 64, 1};
+    if (!make_map(&mk8, a.kcode, 3, dims8, str8, box8, kSw128, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return cudaErrorInvalidValue;
+  }
   TcParams prm{a, (a.nkb + 31) / 32};
   const int64_t tiles = (int64_t)a.B * a.H * ((a.nqb + 1) / 2);
   plan_kernel<<<(unsigned)((tiles + kPlanWarps - 1) / kPlanWarps), kPlanWarps * 32, 0, st>>>(a, prm.mask_words);
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
-  const size_t smem = 1024 + Cfg<D>::kSmemTiles + sizeof(Extra);
+  const size_t smem = 1024 + Cfg<D, I8>::kSmemTiles + sizeof(Extra<I8>);
   // Once per device (so that launches stay free of attribute calls, e.g.
   // inside a stream capture): opt in to the shared memory, and check the
   // register count.  The setmaxnreg split is sized for exactly kRegsLaunch
@@ -832,22 +1059,23 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(attn_tc_kernel<D, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaFuncAttributes fa;
-    if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, I8>)) != cudaSuccess) return e;
     if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
   dim3 grid((a.nqb + 1) / 2, a.H, a.B);
-  attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkb, mvb, prm);
+  attn_tc_kernel<D, I8><<<grid, kThreads, smem, st>>>(mq, mk, mv, mkb, mvb, mk8, prm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs& a, int D, cudaStream_t st) {
-  return D == 128 ? launch_tc<128>(a, st) : launch_tc<64>(a, st);
+  if (a.qk_int8) return D == 128 ? launch_tc<128, true>(a, st) : cudaErrorInvalidValue;
+  return D == 128 ? launch_tc<128, false>(a, st) : launch_tc<64, false>(a, st);
 }
 
 #ifdef SOL_FAULT_TEST

@@ -38,6 +38,9 @@ struct WsLayout {
   size_t mask;      // uint32 [B*H*nqb, mask_words] exact-block bitmap
   size_t counts;    // int32 [B*H*nqb]
   size_t plan;      // int32 [B*H*ceil(nqb/2)][plan_ints]: per query tile, its attention plan
+  size_t kcode;     // int8 [B,H,N,D]  residual key codes (qk_int8 only)
+  size_t ksig;      // fp32 [B,H,nkb]  residual scales (qk_int8 only)
+  size_t kmean16;   // bf16 [B,H,nkb,D] block means rounded to bf16 (qk_int8 only)
   size_t total;
 };
 
@@ -59,6 +62,10 @@ inline WsLayout ws_layout(const sol_params& p) {
   L.mask = take(bh * L.nqb * L.mask_words * 4);
   L.counts = take(bh * L.nqb * 4);
   L.plan = take(bh * ((L.nqb + 1) / 2) * plan_ints(L.mask_words, L.nkb) * 4);
+  const size_t i8 = p.qk_int8 ? 1 : 0;
+  L.kcode = take(i8 * bh * p.N * p.D);
+  L.ksig = take(i8 * bh * L.nkb * 4);
+  L.kmean16 = take(i8 * bh * L.nkb * p.D * 2);
   L.total = off;
   return L;
 }
@@ -79,6 +86,7 @@ struct PoolArgs {
   int with_bias;                 // K pass also computes the log-mass bias (mean summaries)
   float* qbar; float* kbar; __nv_bfloat16* kbar16; __nv_bfloat16* vbar16;
   float* cbias; const float* anchor;
+  int8_t* kcode; float* ksig; __nv_bfloat16* kmean16;   // residual key quantization (qk_int8)
   int* status;                   // device status word (bounded waits)
 };
 
@@ -103,12 +111,15 @@ struct AttnArgs {
   int B, N, H, nqb, nkb;
   float scale;
   int centroids;                 // 1: a centroid term per unselected key block; 0: unselected blocks dropped
+  int qk_int8;                   // 1: exact QK^T from INT8 codes (kcode / ksig / kmean16)
+  const int8_t* kcode; const float* ksig; const __nv_bfloat16* kmean16;
   int* status;
 };
 
 // Launchers (defined in the kernel files; return the launch error).
 cudaError_t launch_pool(const PoolArgs& a, int D, cudaStream_t st);
 cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st);
+cudaError_t launch_quant_k(const PoolArgs& a, int D, cudaStream_t st);
 cudaError_t launch_anchor(const __nv_bfloat16* q, int64_t sb, int64_t sn, int64_t sh, const float* qbar,
                           int B, int N, int H, int D, int nqb, int prefix, float* anchor, cudaStream_t st);
 cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st);

@@ -288,6 +288,79 @@ __global__ void __launch_bounds__(128, 4) pool_kv_reweight_kernel(const PoolArgs
   if (c == 0) a.cbias[row] = m + logf(l) - a.scale * pooled;
 }
 
+// Residual key codes for INT8 QK (thakicloud "MiniMax-H3 ComfyUI accel stack",
+// section 실제 실험 결과, closing accuracy paragraph: only each key block's
+// residual from its mean is quantized, the mean term stays bf16).  Per (key
+// block, head): kmean16 = the fp32 block mean (kbar, written by the K pass)
+// rounded to bf16; r = k - kmean16 in fp32 (a difference of two bf16
+// values); sigma = max |r| / 127 over the block's valid rows and all dims;
+// codes rint(r * (1 / sigma)) (ties to even, the reciprocal rounded to fp32),
+// int8, head-major [B, H, N, D].  Like
+// the mean pass, a thread owns 8 dims of one head; the block's rows are read
+// twice (the second time from L2): once for the maximum, once for the codes.
+template <int D, int HPB>
+__global__ void __launch_bounds__(HPB * (D / 8)) quant_k_kernel(const PoolArgs a) {
+  constexpr int TPH = D / 8;  // threads per head
+  const int j = blockIdx.x;
+  const int h = blockIdx.y * HPB + threadIdx.x / TPH;
+  const int c = threadIdx.x % TPH;
+  const int b = blockIdx.z;
+  const bool active = h < a.H;
+  const int r0 = j * kBlock, r1 = min(a.N, r0 + kBlock);
+  const int64_t row = ((int64_t)b * a.H + h) * a.nb + j;
+  const __nv_bfloat16* base = a.src[1] + (int64_t)b * a.sb + (int64_t)h * a.sh + c * 8;
+  float m[8];
+  if (active) {
+    const float4 m0 = *reinterpret_cast<const float4*>(a.kbar + row * D + c * 8);
+    const float4 m1 = *reinterpret_cast<const float4*>(a.kbar + row * D + c * 8 + 4);
+    const uint4 pk = make_uint4(pack_bf16x2(m0.x, m0.y), pack_bf16x2(m0.z, m0.w), pack_bf16x2(m1.x, m1.y),
+                                pack_bf16x2(m1.z, m1.w));
+    *reinterpret_cast<uint4*>(a.kmean16 + row * D + c * 8) = pk;
+    bf16x8_to_f32(pk, m);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = 0.f;
+  }
+  float amax = 0.f;
+  for (int r = r0; r < r1; r += 8) {
+    uint4 u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      u[k] = make_uint4(0, 0, 0, 0);
+      if (active && r + k < r1) u[k] = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(r + k) * a.sn));
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (r + k < r1) {   // uniform over the CTA
+        float f[8];
+        bf16x8_to_f32(u[k], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i] - m[i]));
+      }
+    }
+  }
+#pragma unroll
+  for (int off = TPH / 2; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float sig = amax / 127.f;   // IEEE division (no fast-math)
+  const float inv = sig > 0.f ? 1.f / sig : 0.f;
+  if (!active) return;
+  if (c == 0) a.ksig[row] = sig;
+  int8_t* dst = a.kcode + (((int64_t)b * a.H + h) * a.N) * D + c * 8;
+  for (int r = r0; r < r1; ++r) {
+    const uint4 uk = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)r * a.sn));
+    float f[8];
+    bf16x8_to_f32(uk, f);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int q = 0;
+      if (sig > 0.f) q = min(127, max(-127, __float2int_rn(__fmul_rn(f[i] - m[i], inv))));
+      w[i >> 2] |= (uint32_t)(q & 0xff) << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint2*>(dst + (int64_t)r * D) = make_uint2(w[0], w[1]);
+  }
+}
+
 // Anchor a = mean of the query rows >= prefix (all rows when prefix >= N),
 // from the pooled Q block means (weighted by their row counts) plus the rows
 // of the block the prefix ends in.  One CTA per (head, batch) with 1024
@@ -360,6 +433,14 @@ cudaError_t launch_pool_kv_reweight(const PoolArgs& a, int D, cudaStream_t st) {
     dim3 grid(a.nb, (a.H + C::kHeads - 1) / C::kHeads, a.B);
     pool_kv_reweight_kernel<64><<<grid, C::kThreads, 0, st>>>(a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_k(const PoolArgs& a, int D, cudaStream_t st) {
+  if (D != 128) return cudaErrorInvalidValue;
+  constexpr int HPB = 8;
+  dim3 grid(a.nb, (a.H + HPB - 1) / HPB, a.B);
+  quant_k_kernel<128, HPB><<<grid, HPB * 16, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -127,14 +127,16 @@ inline EncodeTiledFn encode_fn() {
 constexpr CUtensorMapSwizzle kSw128 = CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr CUtensorMapSwizzle kSwNone = CU_TENSOR_MAP_SWIZZLE_NONE;
 
-// bf16 tiled map; out-of-range elements of a box read as zero.  The caller
-// guarantees a 16-byte aligned base and strides that are multiples of 16 bytes.
+// Tiled map (bf16 unless another element type is given); out-of-range
+// elements of a box read as zero.  The caller guarantees a 16-byte aligned
+// base and strides that are multiples of 16 bytes.
 inline bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-                     const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
+                     const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+  return enc(m, dtype, rank, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -23,7 +23,7 @@ lib = ctypes.CDLL(_LIB_PATH)
 SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_WORKSPACE, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(6)
 
 # Every entry point declared in include/sol.h.
-EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
+EXPORTS = ("sol_workspace_bytes", "sol_workspace_offsets", "sol_workspace_int8_offsets", "sol_col_capacity", "sol_pool", "sol_route", "sol_route_static",
            "sol_attn_fwd", "sol_forward_host", "sol_host_staging_bytes", "sol_last_device_status",
            "sol_status_string", "sol_last_error_text", "sol_debug_drop_arrive",
            "sol_reblock_workspace_bytes", "sol_reblock", "sol_gather_rows", "sol_scatter_rows")
@@ -36,7 +36,7 @@ class sol_params(ctypes.Structure):
                 ("prefix_len", ctypes.c_int32), ("log_mass_bias", ctypes.c_int32),
                 ("in_stride_b", ctypes.c_int64), ("in_stride_n", ctypes.c_int64), ("in_stride_h", ctypes.c_int64),
                 ("out_stride_b", ctypes.c_int64), ("out_stride_n", ctypes.c_int64), ("out_stride_h", ctypes.c_int64),
-                ("routing", ctypes.c_int32), ("topk_ratio", ctypes.c_float)]
+                ("routing", ctypes.c_int32), ("topk_ratio", ctypes.c_float), ("qk_int8", ctypes.c_int32)]
 
 
 _P = ctypes.POINTER(sol_params)
@@ -45,6 +45,8 @@ lib.sol_workspace_bytes.argtypes = [_P]
 lib.sol_workspace_bytes.restype = ctypes.c_size_t
 lib.sol_workspace_offsets.argtypes = [_P, ctypes.POINTER(ctypes.c_int64)]
 lib.sol_workspace_offsets.restype = ctypes.c_int
+lib.sol_workspace_int8_offsets.argtypes = [_P, ctypes.POINTER(ctypes.c_int64)]
+lib.sol_workspace_int8_offsets.restype = ctypes.c_int
 lib.sol_col_capacity.argtypes = [_P]
 lib.sol_col_capacity.restype = ctypes.c_int64
 lib.sol_pool.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -92,7 +94,7 @@ def _check(status: int, where: str):
 def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: int = 0,
                 log_mass_bias: int = 0, scale: float = 0.0, in_strides=None, out_strides=None,
                 q_block: Optional[int] = None, k_block: int = 64, topk_ratio: Optional[float] = None,
-                compressed: bool = False) -> sol_params:
+                compressed: bool = False, qk_int8: bool = False) -> sol_params:
     """Fill a sol_params; strides default to contiguous BTHD [B, N, H, D].
 
     ``log_mass_bias``: 0 (or False) mean-pooled centroids, 1 (or True) plus the
@@ -109,7 +111,7 @@ def make_params(B: int, N: int, H: int, D: int, tau: float = 1.0, prefix_len: in
     out_strides = out_strides or (N * H * D, H * D, D)
     return sol_params(B, N, H, D, q_block, k_block, float(tau), float(scale), prefix_len, int(log_mass_bias),
                       *[int(s) for s in in_strides], *[int(s) for s in out_strides], routing,
-                      float(topk_ratio or 0.0))
+                      float(topk_ratio or 0.0), int(bool(qk_int8)))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -147,6 +149,17 @@ def workspace_views(p: sol_params, ws: torch.Tensor) -> dict:
                 kbar16=view(2, torch.bfloat16, (B, H, nb, D)), vbar16=view(3, torch.bfloat16, (B, H, nb, D)),
                 cbias=view(4, torch.float32, (B, H, nb)), anchor=view(5, torch.float32, (B, H, D)),
                 mask=view(6, torch.int32, (B * H * nb, mw)), counts=view(7, torch.int32, (B * H * nb,)))
+
+
+def int8_views(p: sol_params, ws: torch.Tensor) -> dict:
+    """Typed views of the INT8 QK quantities sol_pool leaves in a workspace (qk_int8 = 1)."""
+    off = (ctypes.c_int64 * 3)()
+    _check(lib.sol_workspace_int8_offsets(ctypes.byref(p), off), "sol_workspace_int8_offsets")
+    nb = -(-p.N // 64)
+    B, H, N, D = p.B, p.H, p.N, p.D
+    return dict(kcode=ws[off[0]:off[0] + B * H * N * D].view(torch.int8).view(B, H, N, D),
+                ksig=ws[off[1]:off[1] + B * H * nb * 4].view(torch.float32).view(B, H, nb),
+                kmean16=ws[off[2]:off[2] + B * H * nb * D * 2].view(torch.bfloat16).view(B, H, nb, D))
 
 
 def sol_col_capacity(p: sol_params) -> int:
@@ -233,7 +246,7 @@ def head_major_params(p: sol_params) -> sol_params:
     """The same problem on head-major [B, H, N, D] copies (inputs and output)."""
     hm = (p.H * p.N * p.D, p.D, p.N * p.D)
     return sol_params(p.B, p.N, p.H, p.D, p.q_block, p.k_block, p.tau, p.scale, p.prefix_len, p.log_mass_bias,
-                      *hm, *hm, p.routing, p.topk_ratio)
+                      *hm, *hm, p.routing, p.topk_ratio, p.qk_int8)
 
 
 @dataclass
@@ -301,7 +314,8 @@ def forward(p: sol_params, q, k, v, buf: Buffers, stream=None) -> Buffers:
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.0, prefix_len: int = 0,
               log_mass_bias: int = 0, scale: float = 0.0, with_lse: bool = False,
-              topk_ratio: Optional[float] = None, compressed: bool = False, reblock: bool = False):
+              topk_ratio: Optional[float] = None, compressed: bool = False, reblock: bool = False,
+              qk_int8: bool = False):
     """Convenience call on BTHD bf16 CUDA tensors (views with unit head-dim stride allowed).
 
     Returns (o, buffers); the buffers hold row_ptr / col_idx / lse for inspection.  With
@@ -315,7 +329,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.
             raise ValueError("q, k, v must be bf16 CUDA tensors with identical strides and contiguous head dim")
     p = make_params(B, N, H, D, tau, prefix_len, log_mass_bias, scale,
                     in_strides=(q.stride(0), q.stride(1), q.stride(2)), topk_ratio=topk_ratio,
-                    compressed=compressed)
+                    compressed=compressed, qk_int8=qk_int8)
     if reblock:
         if with_lse:
             raise ValueError("with_lse is not offered with reblock")

@@ -57,6 +57,7 @@ class Workload:
     topk_ratio: Optional[float] = None   # Top-K routing instead of tau
     compressed: bool = False             # Top-K keeps the compressed branch (64-row blocks, centroids)
     reblock: bool = False                # rows ordered by the adaptive partition first
+    qk_int8: bool = False                # exact logits from INT8 query and residual key codes
     q_block: int = 64
     k_block: int = 64
 

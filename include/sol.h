@@ -108,6 +108,16 @@ typedef struct {
   float topk_ratio;          /* routing 1, 2: fraction of key blocks kept, in (0, 1];
                                 k = floor(topk_ratio * n_kb + 0.5) in double precision from this
                                 float (nearest, halves up), clamped to [1, n_kb]. */
+  int32_t qk_int8;           /* 1: INT8 QK with per-block residual keys (thakicloud "MiniMax-H3
+                                ComfyUI accel stack", section 실제 실험 결과, closing accuracy
+                                paragraph): every exact logit is
+                                s*(q.kmean16_j + sigma_q sigma_j (q_code . r_code)), where
+                                kmean16_j is key block j's mean rounded to bf16, r = k - kmean16_j
+                                is quantized to INT8 with one scale sigma_j = max|r| / 127 per
+                                block, and each query row with its own sigma_q = max|q| / 127
+                                (codes rint(x / sigma), ties to even, in fp32).  The tensor cores
+                                run QK^T as an INT8 product; centroid terms and routing are
+                                unchanged.  Needs D = 128.  0: bf16 QK. */
 } sol_params;
 
 /* Bytes of device workspace that sol_pool / sol_route / sol_attn_fwd share for
@@ -125,9 +135,19 @@ size_t sol_workspace_bytes(const sol_params* p);
  *   offsets[5] anchor fp32 [B, H, D] (log_mass_bias 1 or 2 only)
  *   offsets[6] exact-block bitmap uint32 [B*H*nqb, ceil(nkb/32)]
  *   offsets[7] row counts int32 [B*H*nqb]
- * with nqb = nkb = ceil(N/64).  Returns SOL_ERR_INVALID_ARG for a bad p or
+ * with nqb = nkb = ceil(N/64).  With qk_int8 the workspace also holds the
+ * residual key codes int8 [B, H, N, D], their scales fp32 [B, H, nkb] and the
+ * bf16 block means [B, H, nkb, D] (written by sol_pool).  Returns SOL_ERR_INVALID_ARG for a bad p or
  * a NULL offsets array. */
 sol_status sol_workspace_offsets(const sol_params* p, int64_t offsets[8]);
+
+/* Byte offsets, from the workspace base, of what sol_pool writes for INT8 QK
+ * (qk_int8 = 1), for inspection and tests:
+ *   offsets[0] residual key codes int8 [B, H, N, D]  (codes of rows >= N are not written)
+ *   offsets[1] residual scales fp32 [B, H, nkb]
+ *   offsets[2] block means rounded to bf16 [B, H, nkb, D]
+ * Returns SOL_ERR_INVALID_ARG for a bad p, qk_int8 = 0 or a NULL offsets array. */
+sol_status sol_workspace_int8_offsets(const sol_params* p, int64_t offsets[3]);
 
 /* Worst-case number of CSR column entries: B*H*ceil(N/64)*ceil(N/64) (64-row query-block rows). */
 int64_t sol_col_capacity(const sol_params* p);
@@ -141,7 +161,9 @@ int64_t sol_col_capacity(const sol_params* p);
  *            centroid-logit offset log n_j (+ bias_j when log_mass_bias).
  * Means are over each block's valid rows, accumulated in fp32.  With
  * log_mass_bias = 2 the bf16 key/value centroids are the anchor-weighted
- * summaries, computed in one pass over K and V after the anchor. */
+ * summaries, computed in one pass over K and V after the anchor.  With
+ * qk_int8 a further pass quantizes each key block's residual from its bf16
+ * mean. */
 sol_status sol_pool(const sol_params* p, const void* q, const void* k, const void* v,
                     void* ws, size_t ws_bytes, void* stream);
 
@@ -261,7 +283,12 @@ sol_status sol_last_device_status(void* stream);
 size_t sol_reblock_workspace_bytes(const sol_params* p);
 sol_status sol_reblock(const sol_params* p, const void* q, const void* k, void* ws, size_t ws_bytes,
                        int32_t* perm, void* stream);
-/* xp[b, h, pos, :] = x[b, perm[b, h, pos], h, :]  (x strided by in_stride_*) */
+/* perm must hold, for each (b, h), a permutation of 0 .. N-1 (as sol_reblock
+ * writes it).  Only the range of each entry is checked (an entry outside
+ * [0, N) is skipped and reported); a repeated entry is not detected, and a
+ * scatter through it then writes some rows twice and leaves others as they
+ * were.
+ * xp[b, h, pos, :] = x[b, perm[b, h, pos], h, :]  (x strided by in_stride_*) */
 sol_status sol_gather_rows(const sol_params* p, const int32_t* perm, const void* x, void* xp, void* stream);
 /* x[b, perm[b, h, pos], h, :] = xp[b, h, pos, :]  (x strided by out_stride_*) */
 sol_status sol_scatter_rows(const sol_params* p, const int32_t* perm, const void* xp, void* x, void* stream);

@@ -31,12 +31,13 @@ def to_dev(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None, topk_ratio=None, compressed=False):
+def run_gpu(q, k, v, tau, prefix, lmb, with_lse=True, in_strides=None, topk_ratio=None, compressed=False,
+            qk_int8=False):
     from block_sparse_video_sol_b200 import sol
     B, N, H, D = q.shape
     strides = in_strides or (q.stride(0), q.stride(1), q.stride(2))
     p = sol.make_params(B, N, H, D, tau=tau, prefix_len=prefix, log_mass_bias=lmb, in_strides=strides,
-                        topk_ratio=topk_ratio, compressed=compressed)
+                        topk_ratio=topk_ratio, compressed=compressed, qk_int8=qk_int8)
     buf = sol.alloc_buffers(p, q.device, with_lse=with_lse)
     sol.forward(p, q, k, v, buf)
     sol.sol_last_device_status()
@@ -133,18 +134,23 @@ def check_route_topk(p, buf, Qd, Kd, heads, ratio, prefix, compressed=False):
     return gm, g, int(((g != sel) & ~far).sum())
 
 
-def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None, topk_ratio=None,
-                    compressed=False):
-    """O (and lse) of the given heads vs the oracle run on the GPU mask."""
+def oracle_on_gpu_mask(Qd, Kd, Vd, gm_heads, tau, prefix, lmb, rows=None, topk_ratio=None, compressed=False,
+                       qk_int8=False):
+    """The oracle's forward pass of the given heads on the GPU's routing mask."""
     if topk_ratio is not None and compressed:
-        ref = sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, mask_override=gm_heads, rows=rows,
-                                  topk_ratio=topk_ratio, compressed=True, **oracle_modes(lmb))
-    elif topk_ratio is not None:
-        ref = sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, bq=128, mask_override=gm_heads, rows=rows,
-                                  topk_ratio=topk_ratio)
-    else:
-        ref = sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, mask_override=gm_heads, rows=rows,
-                                  **oracle_modes(lmb))
+        return sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, mask_override=gm_heads, rows=rows,
+                                   topk_ratio=topk_ratio, compressed=True, qk_int8=qk_int8, **oracle_modes(lmb))
+    if topk_ratio is not None:
+        return sol_ref.sol_forward(Qd, Kd, Vd, prefix=prefix, bq=128, mask_override=gm_heads, rows=rows,
+                                   topk_ratio=topk_ratio, qk_int8=qk_int8)
+    return sol_ref.sol_forward(Qd, Kd, Vd, tau=tau, prefix=prefix, mask_override=gm_heads, rows=rows,
+                               qk_int8=qk_int8, **oracle_modes(lmb))
+
+
+def check_attention(p, buf, Qd, Kd, Vd, gm_heads, heads, tau, prefix, lmb, rows=None, topk_ratio=None,
+                    compressed=False, qk_int8=False):
+    """O (and lse) of the given heads vs the oracle run on the GPU mask."""
+    ref = oracle_on_gpu_mask(Qd, Kd, Vd, gm_heads, tau, prefix, lmb, rows, topk_ratio, compressed, qk_int8)
     O = buf.o[:, :, heads].float().cpu().numpy().astype(np.float64)
     Oref = ref["O"]
     keep = ~np.isnan(Oref)
@@ -163,7 +169,8 @@ def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
     """Generate a workload, run it on the GPU, check pool/route/attention on `heads`."""
     q, k, v = synth.generate(w)
     Q, K, V = to_dev(q), to_dev(k), to_dev(v)
-    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias, topk_ratio=w.topk_ratio, compressed=w.compressed)
+    p, buf = run_gpu(Q, K, V, w.tau, w.prefix, w.log_mass_bias, topk_ratio=w.topk_ratio, compressed=w.compressed,
+                     qk_int8=w.qk_int8)
     heads = list(range(w.H)) if heads is None else list(heads)
     Qd, Kd, Vd = (synth.bf16_bits_to_f64(x[:, :, heads]) for x in (q, k, v))
     sla = w.topk_ratio is not None and not w.compressed
@@ -179,5 +186,6 @@ def full_check(w: synth.Workload, heads=None, rows_per_head=None, seed_rows=0):
                 for b in range(w.B) for hh in range(len(heads))}
     mask = g128 if w.topk_ratio is not None else gm[:, heads]
     errs = check_attention(p, buf, Qd, Kd, Vd, mask, heads, w.tau, w.prefix, w.log_mass_bias, rows,
-                           topk_ratio=w.topk_ratio, compressed=w.compressed)
-    return dict(flips=flips, errs=errs, nnz=int(buf.row_ptr[-1].item()), p=p, buf=buf)
+                           topk_ratio=w.topk_ratio, compressed=w.compressed, qk_int8=w.qk_int8)
+    return dict(flips=flips, errs=errs, nnz=int(buf.row_ptr[-1].item()), p=p, buf=buf, mask=mask, heads=heads,
+                Qd=Qd, Kd=Kd, Vd=Vd, rows=rows)
