@@ -21,11 +21,15 @@
 //        lists its rows ascending.
 //
 // Kernels, in launch order:
-//   rb_moment_kernel  -- partial sums of q q^T over 2048-row chunks (fp32);
+//   rb_moment_tc_kernel -- partial sums of q q^T over 2048-row chunks on the
+//                        tensor cores (D = 128; rb_moment_kernel, fp32 FMAs,
+//                        for D = 64);
 //   rb_factor_kernel  -- one CTA per head: the partials summed in a fixed
 //                        order, the ridge, the Cholesky factor in shared memory;
-//   rb_whiten_kernel  -- y = normalise(k L), L loaded once per CTA for 8 tiles
-//                        of 64 rows, and the initial (identity) order;
+//   rb_whiten_tc_kernel -- y = normalise(k L) on the tensor cores, L split into
+//                        three bf16 terms (D = 128; rb_whiten_kernel, fp32
+//                        FMAs with L loaded once per 8 tiles, for D = 64), and
+//                        the initial (identity) order;
 //   rb_split_kernel   -- one launch per level of the hierarchy, one CTA per
 //                        group: mean, power steps, projections as 64-bit keys
 //                        (order-preserving float bits, row index), the split
@@ -127,6 +131,104 @@ __global__ void __launch_bounds__(256) rb_moment_kernel(const ReblockArgs a) {
       f2unpack(acc[i][j], lo, hi);
       *reinterpret_cast<float2*>(&out[(ti * TS + i) * D + tj * TS + 2 * j]) = make_float2(lo, hi);
     }
+}
+
+// The same partial moments on the tensor cores (D = 128): grid (chunks, B*H),
+// 128 threads.  The products of bf16 queries are exact and tcgen05 sums them
+// in fp32, as the FMA kernel does (in another order).  Lane 0 of warp 0
+// streams 64-row Q tiles (both 64-dim chunks, SW128) through a kMomStages
+// ring; warp 1 issues M = N = D = 128, K = 16-row MMAs with A = Q^T and
+// B = Q read MN-major from the same tile, accumulating the chunk's moment in
+// TMEM; then every warp copies its 32 TMEM lanes (rows of the moment) out.
+constexpr int kMomTcRows = 64;    // query rows per tile
+constexpr int kMomStages = 4;     // tiles in flight
+struct MomBars {
+  uint64_t full[kMomStages], empty[kMomStages], done;
+  uint32_t tmem;
+  int abort_flag;
+};
+constexpr int kMomTile = kMomTcRows * 128 * 2;   // 16 KB: two 8 KB chunks of 64 dims
+constexpr size_t kMomTcSmem = 1024 + kMomStages * kMomTile + sizeof(MomBars);
+
+__global__ void __launch_bounds__(128) rb_moment_tc_kernel(const __grid_constant__ CUtensorMap mq, const ReblockArgs a) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t mom_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(mom_smem_raw) + 1023) & ~uintptr_t(1023));
+  MomBars& bar = *reinterpret_cast<MomBars*>(ring + kMomStages * kMomTile);
+  volatile int* abort_flag = &bar.abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int r0 = a.q_lo + blockIdx.x * kMomRows, r1 = min(a.q_lo + a.n_q, r0 + kMomRows);
+  const int ntile = (r1 - r0 + kMomTcRows - 1) / kMomTcRows;   // >= 1; rows past N read as zeros
+  if (tid == 0) {
+    for (int s = 0; s < kMomStages; ++s) { mbar_init(&bar.full[s], 1); mbar_init(&bar.empty[s], 1); }
+    mbar_init(&bar.done, 1);
+    bar.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(128));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncwarp();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bar.tmem;
+  if (warp == 0) {
+    if (lane == 0) {   // TMA producer
+      int nl = 0;
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % kMomStages, n = t / kMomStages;
+        if (!wait_bar(&bar.empty[s], (n & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_expect_tx(&bar.full[s], kMomTile);
+        ++nl;
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(ring + s * kMomTile + c * (kMomTile / 2), &mq, c * 64, h, r0 + kMomTcRows * t, b, &bar.full[s]);
+      }
+      for (int s = 0; s < kMomStages; ++s) {   // every armed load lands before the CTA may exit
+        const int cnt = (nl + kMomStages - 1 - s) / kMomStages;
+        if (cnt) drain_bar(&bar.full[s], (cnt - 1) & 1, a.status);
+      }
+    }
+  } else if (warp == 1) {   // MMA issuer (the whole warp; one elected lane issues)
+    constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);   // A and B both MN-major (dims contiguous)
+    bool ok = true;
+    for (int t = 0; t < ntile && ok; ++t) {
+      const int s = t % kMomStages, n = t / kMomStages;
+      ok = __all_sync(0xffffffffu, wait_bar(&bar.full[s], n & 1, abort_flag, a.status));
+      if (!ok) break;
+      fence_after();
+      // MN-major SW128: 64-dim chunks 8 KB apart (LBO), 8-row groups 1024 B apart (SBO); K = 16 rows = 2048 B
+      const uint64_t dsc = sdesc(smem_u32(ring + s * kMomTile), kMomTile / 2, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kMomTcRows / 16; ++kk)
+        mma_ss_w(tmem, dsc + (uint64_t)(kk * 128), dsc + (uint64_t)(kk * 128), id, (t > 0 || kk > 0) ? 1u : 0u);
+      mma_commit_w(&bar.empty[s]);   // the stage is free once these MMAs have read it
+    }
+    mma_commit_w(&bar.done);
+  }
+  // every warp: its 32 TMEM lanes = rows 32w .. 32w+31 of the moment, 128 columns each
+  const bool ok = __all_sync(0xffffffffu, wait_bar(&bar.done, 0, abort_flag, a.status));
+  fence_after();
+  if (ok && !*abort_flag) {
+    float* out = a.mpart + ((int64_t)bh * a.mchunks + blockIdx.x) * D * D + (int64_t)(32 * warp + lane) * D;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+    for (int c = 0; c < D / 32; ++c) {
+      float v[32];
+      tmem_ld32(lane_addr + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(out + 32 * c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    }
+  }
+  fence_before();
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(128));
+  }
 }
 
 // M = (sum of the partials, chunk order) / n_q + ridge; its lower Cholesky
@@ -263,6 +365,167 @@ __global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
       }
     }
     if (tid < kBlock && t0 + tid < a.n_v) a.ord[(int64_t)bh * a.n_v + t0 + tid] = t0 + tid;
+  }
+}
+
+// y = normalise(k L) on the tensor cores (D = 128): grid (ceil(n_v / (128 kWhTcTiles)), B*H),
+// 128 threads.  L (fp32) is split into three bf16 terms L = L1 + L2 + L3 (each the
+// rounding of what the previous ones leave, 2^-24 of L in all), laid out MN-major
+// in shared memory; every 128-row key tile is A (K-major, from TMA) and the three
+// products accumulate in TMEM in fp32: the products are exact and the split is as
+// fine as fp32's own rounding.  Each thread then takes its row (TMEM lane) for the
+// norm and writes the unit vector.  Warps 0-3 read TMEM (warp w: lanes 32w .. 32w+31),
+// warp 1 also issues the MMAs, and warp 4 alone streams the key tiles, so the
+// producer never waits inside a warp that the epilogue needs.
+constexpr int kWhTcRows = 128;
+constexpr int kWhTcTiles = 8;    // key tiles per CTA
+constexpr int kWhTcThreads = 160;
+constexpr int kWhTcStages = 2;
+struct WhBars {
+  uint64_t full[kWhTcStages], empty[kWhTcStages], acc_full, acc_free;
+  uint32_t tmem;
+  int abort_flag;
+};
+constexpr int kWhTile = kWhTcRows * 128 * 2;     // 32 KB: a K tile, or one bf16 term of L
+constexpr size_t kWhTcSmem = 1024 + (3 + kWhTcStages) * kWhTile + sizeof(WhBars);
+
+__global__ void __launch_bounds__(kWhTcThreads) rb_whiten_tc_kernel(const __grid_constant__ CUtensorMap mk, const ReblockArgs a) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t wh_smem_raw[];
+  uint8_t* Lt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wh_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = Lt + 3 * kWhTile;
+  WhBars& bar = *reinterpret_cast<WhBars*>(ring + kWhTcStages * kWhTile);
+  volatile int* abort_flag = &bar.abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t_first = blockIdx.x * kWhTcTiles;
+  const int ntile = min(kWhTcTiles, (a.n_v + kWhTcRows - 1) / kWhTcRows - t_first);
+  if (tid == 0) {
+    for (int s = 0; s < kWhTcStages; ++s) { mbar_init(&bar.full[s], 1); mbar_init(&bar.empty[s], 1); }
+    mbar_init(&bar.acc_full, 1);
+    mbar_init(&bar.acc_free, 4);
+    bar.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(128));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // L's three bf16 terms, MN-major SW128: element (i, j) in chunk j/64, row i, 16-byte unit (j%64)/8
+  // at position unit ^ (i & 7); thread tid converts units tid, tid+160, ... (8 columns each)
+  const float* Lg = a.L + (int64_t)bh * D * D;
+  for (int u = tid; u < D * D / 8; u += kWhTcThreads) {
+    const int i = u / (D / 8), j0 = (u % (D / 8)) * 8;
+    const float4 x0 = *reinterpret_cast<const float4*>(Lg + i * D + j0);
+    const float4 x1 = *reinterpret_cast<const float4*>(Lg + i * D + j0 + 4);
+    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint32_t w1[4], w2[4], w3[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float r0 = x[e], r1 = x[e + 1];
+      const __nv_bfloat162 h1 = __floats2bfloat162_rn(r0, r1);
+      r0 -= __low2float(h1); r1 -= __high2float(h1);
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(r0, r1);
+      r0 -= __low2float(h2); r1 -= __high2float(h2);
+      const __nv_bfloat162 h3 = __floats2bfloat162_rn(r0, r1);
+      w1[e / 2] = *reinterpret_cast<const uint32_t*>(&h1);
+      w2[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+      w3[e / 2] = *reinterpret_cast<const uint32_t*>(&h3);
+    }
+    const int off = (j0 / 64) * (kWhTile / 2) + i * 128 + ((((j0 % 64) / 8) ^ (i & 7)) << 4);
+    *reinterpret_cast<uint4*>(Lt + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    *reinterpret_cast<uint4*>(Lt + kWhTile + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+    *reinterpret_cast<uint4*>(Lt + 2 * kWhTile + off) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
+  fence_before();
+  __syncwarp();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bar.tmem;
+  if (warp == 4 && lane == 0) {   // TMA producer: 128-row key tiles (two 64-dim chunks)
+    int nl = 0;
+    for (int t = 0; t < ntile; ++t) {
+      const int s = t % kWhTcStages, n = t / kWhTcStages;
+      if (!wait_bar(&bar.empty[s], (n & 1) ^ 1, abort_flag, a.status)) break;
+      mbar_expect_tx(&bar.full[s], kWhTile);
+      ++nl;
+      const int row = a.n_fix + (t_first + t) * kWhTcRows;
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_4d(ring + s * kWhTile + c * (kWhTile / 2), &mk, c * 64, h, row, b, &bar.full[s]);
+    }
+    for (int s = 0; s < kWhTcStages; ++s) {
+      const int cnt = (nl + kWhTcStages - 1 - s) / kWhTcStages;
+      if (cnt) drain_bar(&bar.full[s], (cnt - 1) & 1, a.status);
+    }
+  }
+  __syncwarp();
+  constexpr uint32_t id = idesc_bf16(128, 128, 0, 1);   // A = keys K-major, B = L terms MN-major
+  const uint64_t ldsc0 = sdesc(smem_u32(Lt), kWhTile / 2, 1024);
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+  bool ok = true;
+  int issued = 0;   // tiles whose MMAs warp 1 committed
+  for (int t = 0; t < ntile && ok && warp < 4; ++t) {
+    const int s = t % kWhTcStages, n = t / kWhTcStages;
+    if (warp == 1) {   // MMAs of tile t once its keys landed and the epilogue read tile t-1
+      ok = __all_sync(0xffffffffu, wait_bar(&bar.full[s], n & 1, abort_flag, a.status) &&
+                                       (t == 0 || wait_bar(&bar.acc_free, (t - 1) & 1, abort_flag, a.status)));
+      if (ok) {
+        fence_after();
+        const uint64_t adsc = sdesc(smem_u32(ring + s * kWhTile), 16, 1024);
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t aoff = (uint64_t)(((kk >> 2) * (kWhTile / 2) + (kk & 3) * 32) >> 4);
+            const uint64_t boff = (uint64_t)((term * kWhTile + kk * 2048) >> 4);
+            mma_ss_w(tmem, adsc + aoff, ldsc0 + boff, id, (term > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit_w(&bar.empty[s]);
+        mma_commit_w(&bar.acc_full);
+        ++issued;
+      }
+    }
+    // every warp: its 32 rows of y from TMEM, the norms, the unit vectors
+    ok = __all_sync(0xffffffffu, wait_bar(&bar.acc_full, t & 1, abort_flag, a.status));
+    if (!ok) break;
+    fence_after();
+    const int row = (t_first + t) * kWhTcRows + 32 * warp + lane;   // position among the video rows
+    float* Yg = a.Y + ((int64_t)bh * a.n_v + row) * D;
+    float ss = 0.f;
+    for (int c = 0; c < D / 32; ++c) {
+      float v[32];
+      tmem_ld32(lane_addr + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+    }
+    const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+    for (int c = 0; c < D / 32; ++c) {   // second read of the row: the unit vector
+      float v[32];
+      tmem_ld32(lane_addr + 32 * c, v);
+      tmem_wait_ld();
+      if (row < a.n_v) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(Yg + 32 * c + e) = make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
+      }
+    }
+    if (row < a.n_v) a.ord[(int64_t)bh * a.n_v + row] = row;
+    fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar.acc_free);   // this warp has read tile t's accumulator
+  }
+  fence_before();
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    // every committed product has landed before TMEM is released (on the normal path
+    // the epilogue has waited for each; after an abort, wait for the last one)
+    if (issued > 0) drain_bar(&bar.acc_full, (issued - 1) & 1, a.status);
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(128));
   }
 }
 
@@ -537,16 +800,30 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(rb_factor_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, f128)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(rb_whiten_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, w128)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(rb_factor_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, f64)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(rb_whiten_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, w64)) != cudaSuccess)
+        (e = cudaFuncSetAttribute(rb_whiten_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, w64)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_moment_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMomTcSmem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_whiten_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWhTcSmem)) != cudaSuccess)
       return e;
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
   if (a.n_v > 0) {
+    // q and k as 4-D [B, N, H, D] maps (the same strides): TMA boxes of 64 dims
+    const cuuint64_t bstride = (cuuint64_t)(a.B > 1 ? a.sb : (int64_t)a.N * a.sn) * 2;
+    const cuuint64_t dims4[4] = {(cuuint64_t)D, (cuuint64_t)a.H, (cuuint64_t)a.N, (cuuint64_t)a.B};
+    const cuuint64_t str4[3] = {(cuuint64_t)a.sh * 2, (cuuint64_t)a.sn * 2, bstride};
     dim3 gm(a.mchunks, BH), gw((a.n_v + kBlock * kWhTiles - 1) / (kBlock * kWhTiles), BH);
     if (D == 128) {
-      rb_moment_kernel<128><<<gm, 256, 0, st>>>(a);
+      // the query map of the partial-moment kernel: 64 dims x 64 rows per box, SW128
+      CUtensorMap mq;
+      const cuuint32_t box4[4] = {64, 1, kMomTcRows, 1};
+      if (!make_map(&mq, a.q, 4, dims4, str4, box4, kSw128)) return cudaErrorInvalidValue;
+      rb_moment_tc_kernel<<<gm, 128, kMomTcSmem, st>>>(mq, a);
       rb_factor_kernel<128><<<BH, 256, f128, st>>>(a);
-      rb_whiten_kernel<128><<<gw, 256, w128, st>>>(a);
+      CUtensorMap mk;   // 128-row key tiles of the whitening: 64 dims x 128 rows per box, SW128
+      const cuuint32_t boxk[4] = {64, 1, kWhTcRows, 1};
+      if (!make_map(&mk, a.k, 4, dims4, str4, boxk, kSw128)) return cudaErrorInvalidValue;
+      dim3 gwt((a.n_v + kWhTcRows * kWhTcTiles - 1) / (kWhTcRows * kWhTcTiles), BH);
+      rb_whiten_tc_kernel<<<gwt, kWhTcThreads, kWhTcSmem, st>>>(mk, a);
     } else {
       rb_moment_kernel<64><<<gm, 256, 0, st>>>(a);
       rb_factor_kernel<64><<<BH, 256, f64, st>>>(a);
