@@ -302,7 +302,7 @@ sol_status sol_last_device_status(void* stream) {
 namespace {
 struct ReblockLayout {
   int n_fix, n_v, q_lo, n_q, mchunks;
-  size_t mpart, L, Y, ord, tmp, key, total;
+  size_t mpart, L, Y, ord, tmp, key, gpart, wbuf, cbuf, total;
 };
 ReblockLayout reblock_layout(const sol_params& p) {
   ReblockLayout R{};
@@ -315,12 +315,16 @@ ReblockLayout reblock_layout(const sol_params& p) {
   const size_t bh = (size_t)p.B * p.H, D = p.D;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
-  R.mpart = take(bh * R.mchunks * D * D * 4);
+  // the partial moments are dead once L is factored: the levels' Gram partials reuse them
+  R.mpart = take(std::max(bh * R.mchunks * D * D, reblock_gram_part_floats((int)bh, R.n_v, p.D)) * 4);
+  R.gpart = R.mpart;
   R.L = take(bh * D * D * 4);
   R.Y = take(bh * R.n_v * D * 4);
   R.ord = take(bh * R.n_v * 4);
   R.tmp = take(bh * R.n_v * 4);
   R.key = take(bh * R.n_v * 8);
+  R.wbuf = take(reblock_axis_floats((int)bh, R.n_v, p.D) * 4);
+  R.cbuf = take(2 * reblock_axis_floats((int)bh, R.n_v, p.D) * 4);
   R.total = R.n_v > 0 ? off : 0;
   return R;
 }
@@ -357,7 +361,9 @@ sol_status sol_reblock(const sol_params* p, const void* q, const void* k, void* 
   if (R.total > 0) {
     a.mpart = at<float>(ws, R.mpart); a.L = at<float>(ws, R.L); a.Y = at<float>(ws, R.Y);
     a.ord = at<int32_t>(ws, R.ord); a.tmp = at<int32_t>(ws, R.tmp); a.key = at<uint64_t>(ws, R.key);
+    a.gpart = at<float>(ws, R.gpart); a.wbuf = at<float>(ws, R.wbuf); a.cbuf = at<float>(ws, R.cbuf);
   }
+  a.gram_levels = reblock_gram_levels(R.n_v, p->D);
   a.perm = perm;
   a.status = status;
   const cudaError_t e = launch_reblock(a, kReblockIters, static_cast<cudaStream_t>(stream));

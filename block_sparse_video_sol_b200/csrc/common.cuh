@@ -144,9 +144,16 @@ struct ReblockArgs {
   uint64_t* key;                 // [B*H][n_v] split keys
   int32_t* perm;                 // [B*H][N] output: original row at each position
   int* status;
+  int gram_levels;               // top levels whose split axes come from Gram matrices (D = 128)
+  float* gpart;                  // Gram partials of one such level: [slots][kGramPartFloats]
+  float* wbuf;                   // split axes of one such level: [B*H << lvl][D]
+  float* cbuf;                   // [2][B*H << (levels - 1)][D]: group means, the next level's shifts
 };
 int reblock_levels(int n_v);
 int reblock_moment_chunks(int n_q);
+int reblock_gram_levels(int n_v, int D);
+size_t reblock_gram_part_floats(int BH, int n_v, int D);   // size of ReblockArgs::gpart
+size_t reblock_axis_floats(int BH, int n_v, int D);        // size of ReblockArgs::wbuf
 cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st);
 cudaError_t launch_rows(const int32_t* perm, const __nv_bfloat16* src, __nv_bfloat16* dst, int B, int H, int N, int D,
                         int64_t sb, int64_t sn, int64_t sh, bool gather, int* status, cudaStream_t st);

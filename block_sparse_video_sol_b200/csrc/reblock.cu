@@ -42,6 +42,8 @@
 // Every reduction runs in a fixed order, so the partition is deterministic.
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include <atomic>
 
 #include "common.cuh"
@@ -583,9 +585,390 @@ __device__ __forceinline__ float rb_norm(const float* v, int D, float* s_tmp) {
   return n;
 }
 
-// One level of the hierarchy: grid (2^lvl, B*H); group blockIdx.x of every head.
-template <int D, int T>
-__global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lvl, int iters) {
+__device__ inline size_t reblock_axis_floats_dev(const ReblockArgs& a) {
+  return a.gram_levels == 0 ? 0 : ((size_t)(a.B * a.H) << (a.gram_levels - 1)) * 128;
+}
+
+// The group of level lvl that holds position pos: its index s among the level's
+// 2^lvl groups (bits as in rb_segment), start and length; false if an ancestor is
+// already a leaf.
+__device__ inline bool rb_group_at(int n_v, int lvl, int pos, int& s, int& start, int& len) {
+  s = 0;
+  start = 0;
+  len = n_v;
+  for (int l = 0; l < lvl; ++l) {
+    if (len <= kBlock) return false;
+    const int left = rb_left(len);
+    if (pos < start + left) {
+      s = 2 * s;
+      len = left;
+    } else {
+      s = 2 * s + 1;
+      start += left;
+      len -= left;
+    }
+  }
+  return true;
+}
+
+// Split axes of the large groups from Gram matrices (D = 128).
+//
+// The power steps z = C w, C = sum over the group of (y - mean)(y - mean)^T,
+// need C only, so a group's C is built once instead of streaming its rows
+// once per step.  With a shift c and x = y - c,
+//   G = sum x x^T,  s1 = sum x,  C = G - s1 s1^T / n,  mean = c + s1 / n.
+// The subtraction cancels |mean - c|^2 against C's spread, so c has to lie near
+// the mean: it is the parent group's mean (computed the same way one level up),
+// and for the root the mean of 1,024 evenly spaced rows (rb_shift0_kernel).
+// (The whitened unit keys of a head are close to isotropic: shifting by one row
+// instead, |mean - c|^2 is about 100 times C's largest eigenvalue.)
+// rb_gram_tc_kernel sums G on the tensor cores: each x (fp32) is split into
+// two bf16 terms h + m (round to nearest each; the rest, below 2^-17 |x|, is
+// dropped), and G = (H + M)^T (H + M) = H^T H + H^T M + M^T H + M^T M.  The
+// dropped rest is a zero-mean rounding residual, so its share of G shrinks
+// with the number of rows.  TMEM accumulates four tiles (256 rows, 16 K steps)
+// at a time; four epilogue warps add each finished chunk into a running fp32
+// sum (round to nearest) while the MMAs fill the other chunk buffer, so no
+// accumulation in the tensor pipe runs longer than 16 steps.  The level's rows
+// are cut into 64-row tiles (tiles never straddle a group: group starts are
+// multiples of 64), the tiles of all heads split evenly over kGrCtas CTAs; each
+// CTA flushes one partial (G, s1) per group it touches into slot (group index +
+// CTA index), which is unique.  rb_axis_kernel sums a group's partials in CTA
+// order, forms C, runs the power steps from r - mean (r the group's first row)
+// and records the group's mean for the next level.
+constexpr int kGramMinRows = 2048;   // levels whose groups have at least this many rows
+constexpr int kGrCtas = 148;
+constexpr int kGrRows = 64;          // rows per tile: four K = 16 steps
+constexpr int kGrChunk = 4;          // tiles per TMEM chunk
+constexpr int kGrSlots = 3;          // fp32 staging slots per row: kGrSlots - 1 tiles in flight
+constexpr int kGrWarps = 16;         // converting warps 0-15; warp 16 issues the MMAs; 17-20 add the chunks
+constexpr int kGrMmaWarp = kGrWarps, kGrEpiWarp = kGrWarps + 1;
+constexpr int kGrThreads = 32 * (kGrWarps + 5);
+constexpr int kGrRowsPerWarp = kGrRows / kGrWarps;
+constexpr int kGrTerm = kGrRows * 128 * 2;         // 16 KB: one bf16 term, two 8 KB chunks of 64 dims
+constexpr int kGrStage = 2 * kGrTerm;              // the two terms of a tile
+constexpr int kGrStaging = kGrRows * 128 * 4;      // 32 KB: one fp32 tile
+constexpr int kGramPartFloats = 128 * 128 + 128;   // G, then s1
+struct GrBars {
+  uint64_t full[2], empty[2], accf[2], accr[2], done;
+  uint32_t tmem;
+  int abort_flag;
+};
+constexpr size_t kGrSmem = 1024 + 2 * kGrStage + kGrSlots * kGrStaging + kGrWarps * 128 * 4 + sizeof(GrBars);
+static_assert(kGrSmem <= 232448, "Gram kernel shared memory");
+
+// Means of level lvl's groups go to half (lvl + 1) & 1 of cbuf; the shifts of level
+// lvl are read from half lvl & 1: the parent's mean, or the root's sample mean.
+__device__ inline int64_t rb_shift_index(const ReblockArgs& a, int lvl, int bh, int s) {
+  const int64_t half = (int64_t)reblock_axis_floats_dev(a) * (lvl & 1);
+  return half / 128 + (lvl == 0 ? (int64_t)bh : ((int64_t)bh << (lvl - 1)) + (s >> 1));
+}
+
+// The root's shift: per head, the mean of min(n_v, 1024) evenly spaced rows;
+// grid B*H, 1024 threads: sample i goes to warp i % 32, whose lanes hold four
+// dimensions each; the 32 warp sums are added in warp order.
+__global__ void __launch_bounds__(1024) rb_shift0_kernel(const ReblockArgs a) {
+  constexpr int D = 128;
+  __shared__ __align__(16) float4 part[32][D / 4];
+  const int bh = blockIdx.x, S = min(a.n_v, 1024), warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* Yh = a.Y + (int64_t)bh * a.n_v * D;
+  float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int i = warp; i < S; i += 32) {
+    const float4 y = *reinterpret_cast<const float4*>(Yh + ((int64_t)i * a.n_v / S) * D + 4 * lane);
+    t.x += y.x; t.y += y.y; t.z += y.z; t.w += y.w;
+  }
+  part[warp][lane] = t;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float u = 0.f;
+    for (int w = 0; w < 32; ++w) u += reinterpret_cast<const float*>(part[w])[threadIdx.x];
+    a.cbuf[rb_shift_index(a, 0, bh, 0) * D + threadIdx.x] = u / (float)S;
+  }
+}
+
+// grid ceil(tiles / chunk), kGrThreads threads; tph = 64-row tiles per head.
+// TMEM columns: chunk buffers 0-127 and 128-255, the running sum 256-383.
+__global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const ReblockArgs a, int lvl, int tph, int chunk) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t gr_smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gr_smem_raw) + 1023) & ~uintptr_t(1023));
+  float* stg = reinterpret_cast<float*>(ring + 2 * kGrStage);    // [kGrSlots][kGrRows][D]
+  float* s1red = stg + kGrSlots * kGrRows * D;                    // [kGrWarps][D]
+  GrBars& bar = *reinterpret_cast<GrBars*>(s1red + kGrWarps * D);
+  volatile int* abort_flag = &bar.abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int TT = a.B * a.H * tph;
+  const int t0 = blockIdx.x * chunk, t1 = min(TT, t0 + chunk);
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.full[b], kGrWarps);
+      mbar_init(&bar.empty[b], 1);
+      mbar_init(&bar.accf[b], 1);
+      mbar_init(&bar.accr[b], 4);
+    }
+    mbar_init(&bar.done, 1);
+    bar.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kGrMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncwarp();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bar.tmem;
+  int q = 0;    // tiles through the ring so far (uniform)
+  int cc = 0;   // TMEM chunks so far (uniform)
+  bool ok = true, mma_issued = false;
+  for (int T = t0; T < t1 && ok;) {
+    const int bh = T / tph, k0 = T % tph;
+    int s, start, len;
+    const bool live = rb_group_at(a.n_v, lvl, k0 * kGrRows, s, start, len) && len > kBlock;
+    // a group that is a leaf here (or lies under one) is one tile: its start is a multiple of 64
+    const int Te = live ? min(t1, bh * tph + (start + len + kGrRows - 1) / kGrRows) : T + 1;
+    if (!live) {
+      T = Te;
+      continue;
+    }
+    const int ntile = Te - T, nchunk = (ntile + kGrChunk - 1) / kGrChunk;
+    const int p_lo = k0 * kGrRows, p_hi = min(start + len, (Te - bh * tph) * kGrRows);
+    const int32_t* ordh = a.ord + (int64_t)bh * a.n_v;
+    const float* Yh = a.Y + (int64_t)bh * a.n_v * D;
+    float* P = a.gpart + (size_t)(((int64_t)bh << lvl) + s + blockIdx.x) * kGramPartFloats;
+    if (warp < kGrWarps) {   // staging copies, the shift and the bf16 split into the ring
+      const float4 rv = *reinterpret_cast<const float4*>(a.cbuf + rb_shift_index(a, lvl, bh, s) * D + 4 * lane);
+      float4 s1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      struct Ids { int v[kGrRowsPerWarp]; };
+      auto ids_of = [&](int t) {
+        Ids id;
+#pragma unroll
+        for (int j = 0; j < kGrRowsPerWarp; ++j) {
+          const int pos = p_lo + t * kGrRows + warp * kGrRowsPerWarp + j;
+          id.v[j] = (t < ntile && pos < p_hi) ? ordh[pos] : -1;
+        }
+        return id;
+      };
+      auto issue = [&](int t, const Ids id) {   // always one commit group, possibly empty
+        float* dst = stg + ((t % kGrSlots) * kGrRows + warp * kGrRowsPerWarp) * D + 4 * lane;
+#pragma unroll
+        for (int j = 0; j < kGrRowsPerWarp; ++j)
+          if (id.v[j] >= 0) cp_async16(dst + j * D, Yh + (int64_t)id.v[j] * D + 4 * lane);
+        cp_async_commit();
+      };
+#pragma unroll
+      for (int t = 0; t < kGrSlots - 1; ++t) issue(t, ids_of(t));
+      Ids idn = ids_of(kGrSlots - 1);
+      for (int t = 0; t < ntile; ++t) {
+        issue(t + kGrSlots - 1, idn);   // empty past the segment's end
+        idn = ids_of(t + kGrSlots);     // consumed by the next iteration's issue
+        cp_async_wait<kGrSlots - 1>();  // this thread's copies of tile t have landed
+        const int st = (q + t) & 1, n = (q + t) >> 1;
+        if (!__all_sync(0xffffffffu, wait_bar(&bar.empty[st], (n & 1) ^ 1, abort_flag, a.status))) break;
+        const float* sp = stg + ((t % kGrSlots) * kGrRows + warp * kGrRowsPerWarp) * D + 4 * lane;
+        uint8_t* base = ring + st * kGrStage;
+#pragma unroll
+        for (int j = 0; j < kGrRowsPerWarp; ++j) {
+          const int R = warp * kGrRowsPerWarp + j;
+          float x[4] = {0.f, 0.f, 0.f, 0.f};
+          if (p_lo + t * kGrRows + R < p_hi) {
+            const float4 y = *reinterpret_cast<const float4*>(sp + j * D);
+            x[0] = y.x - rv.x; x[1] = y.y - rv.y; x[2] = y.z - rv.z; x[3] = y.w - rv.w;
+            s1.x += x[0]; s1.y += x[1]; s1.z += x[2]; s1.w += x[3];
+          }
+          uint32_t th[2], tm[2];
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const __nv_bfloat162 h1 = __floats2bfloat162_rn(x[e], x[e + 1]);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[e] - __low2float(h1), x[e + 1] - __high2float(h1));
+            th[e / 2] = *reinterpret_cast<const uint32_t*>(&h1);
+            tm[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          // MN-major SW128: dims 4 lane .. 4 lane + 3 are chunk lane / 16, 16-byte unit (lane % 16) / 2
+          // at position unit ^ (R & 7), half lane % 2
+          const int off = (lane >> 4) * (kGrTerm / 2) + R * 128 + ((((lane & 15) >> 1) ^ (R & 7)) << 4) + ((lane & 1) << 3);
+          *reinterpret_cast<uint2*>(base + off) = make_uint2(th[0], th[1]);
+          *reinterpret_cast<uint2*>(base + kGrTerm + off) = make_uint2(tm[0], tm[1]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.full[st]);
+      }
+      cp_async_wait<0>();
+      *reinterpret_cast<float4*>(s1red + warp * D + 4 * lane) = s1;
+    } else if (warp == kGrMmaWarp) {   // M = N = 128 (dims), K = 16 rows, A and B MN-major from the ring
+      constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);
+      for (int t = 0; t < ntile; ++t) {
+        const int kc = cc + t / kGrChunk, b = kc & 1, u = kc >> 1;
+        const bool first = t % kGrChunk == 0, last = t % kGrChunk == kGrChunk - 1 || t == ntile - 1;
+        // chunk buffer b is free once the epilogue has added its previous chunk
+        if (first && !__all_sync(0xffffffffu, wait_bar(&bar.accr[b], (u & 1) ^ 1, abort_flag, a.status))) break;
+        const int st = (q + t) & 1, n = (q + t) >> 1;
+        if (!__all_sync(0xffffffffu, wait_bar(&bar.full[st], n & 1, abort_flag, a.status))) break;
+        fence_after();
+        const uint64_t dH = sdesc(smem_u32(ring + st * kGrStage), kGrTerm / 2, 1024);
+        const uint64_t dM = dH + (uint64_t)(kGrTerm >> 4);
+        const uint32_t acc_addr = tmem + 128 * b;
+#pragma unroll
+        for (int kk = 0; kk < kGrRows / 16; ++kk) {
+          const uint64_t o = (uint64_t)(kk * 128);   // 16 rows = 2048 bytes
+          mma_ss_w(acc_addr, dH + o, dH + o, id, (!first || kk > 0) ? 1u : 0u);
+          mma_ss_w(acc_addr, dH + o, dM + o, id, 1u);
+          mma_ss_w(acc_addr, dM + o, dH + o, id, 1u);
+          mma_ss_w(acc_addr, dM + o, dM + o, id, 1u);
+        }
+        mma_issued = true;
+        mma_commit_w(&bar.empty[st]);
+        if (last) mma_commit_w(&bar.accf[b]);
+      }
+    } else {   // warps 17-20: TMEM lanes 32 (warp % 4) + lane, i.e. row i of the chunk and of the sum
+      const int i = 32 * (warp & 3) + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+      bool got = true;
+      for (int c = 0; c < nchunk && got; ++c) {
+        const int kc = cc + c, b = kc & 1, u = kc >> 1;
+        got = __all_sync(0xffffffffu, wait_bar(&bar.accf[b], u & 1, abort_flag, a.status));
+        if (!got) break;
+        fence_after();
+#pragma unroll 1
+        for (int g = 0; g < D / 16; ++g) {   // sum (+)= chunk, 16 columns at a time
+          float v[16], w2[16];
+          tmem_ld16(lane_addr + 128 * b + 16 * g, v);
+          if (c > 0) tmem_ld16(lane_addr + 256 + 16 * g, w2);
+          tmem_wait_ld();
+          if (c > 0) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += w2[e];
+          }
+          tmem_st16(lane_addr + 256 + 16 * g, reinterpret_cast<const uint32_t*>(v));
+        }
+        tmem_wait_st();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.accr[b]);
+      }
+      if (got) {   // row i of the segment's G
+#pragma unroll 1
+        for (int g = 0; g < D / 32; ++g) {
+          float v[32];
+          tmem_ld32(lane_addr + 256 + 32 * g, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(P + i * D + 32 * g + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+    }
+    __syncthreads();   // s1red complete
+    if (tid < D) {
+      float t = 0.f;
+      for (int w2 = 0; w2 < kGrWarps; ++w2) t += s1red[w2 * D + tid];
+      P[D * D + tid] = t;
+    }
+    q += ntile;
+    cc += nchunk;
+    T = Te;
+    fence_before();
+    ok = !__syncthreads_or(*abort_flag);   // the sum's reads are done before the next segment; uniform
+    fence_after();
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == kGrMmaWarp) {
+    // every issued MMA has landed before TMEM is released (after an abort the
+    // epilogue may not have waited for the last chunks)
+    if (mma_issued) {
+      mma_commit_w(&bar.done);
+      drain_bar(&bar.done, 0, a.status);
+    }
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(512));
+  }
+}
+
+// A group's split axis from its Gram partials: grid (2^lvl, B*H), 256 threads.
+// G = the sum of the partials (CTA order); C = G - s1 s1^T / n; the power
+// steps start from r - mean = -s1 / n (e_0 if that is zero).
+__global__ void __launch_bounds__(256) rb_axis_kernel(const ReblockArgs a, int lvl, int tph, int chunk, int iters) {
+  constexpr int D = 128, LD = D + 1;
+  extern __shared__ __align__(16) float G[];   // [D][LD]
+  __shared__ float s1[D], w[D], z[D];
+  __shared__ float s_tmp;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y, grp = blockIdx.x;
+  int start, len;
+  if (!rb_segment(a.n_v, lvl, grp, start, len) || len <= kBlock) return;
+  const int64_t gidx = ((int64_t)bh << lvl) + grp;
+  const int c0 = (bh * tph + start / kGrRows) / chunk, c1 = (bh * tph + (start + len - 1) / kGrRows) / chunk;
+  {   // thread tid sums float4 f = tid + 256 k (k < 16) of every partial, 16 loads in flight
+    float4 acc[D * D / 4 / 256];
+#pragma unroll
+    for (int k = 0; k < D * D / 4 / 256; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = c0; c <= c1; ++c) {
+      const float4* src = reinterpret_cast<const float4*>(a.gpart + (size_t)(gidx + c) * kGramPartFloats);
+#pragma unroll
+      for (int k = 0; k < D * D / 4 / 256; ++k) {
+        const float4 v = src[tid + 256 * k];
+        acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < D * D / 4 / 256; ++k) {
+      const int idx = 4 * (tid + 256 * k), i = idx / D, j = idx % D;
+      G[i * LD + j] = acc[k].x; G[i * LD + j + 1] = acc[k].y; G[i * LD + j + 2] = acc[k].z; G[i * LD + j + 3] = acc[k].w;
+    }
+  }
+  const float inv_n = 1.f / (float)len;
+  if (tid < D) {
+    float t = 0.f;
+    for (int c = c0; c <= c1; ++c) t += a.gpart[(size_t)(gidx + c) * kGramPartFloats + D * D + tid];
+    s1[tid] = t;
+    // r - mean = (r - c) - s1 / n; the mean c + s1 / n is the children's shift
+    const float cv = a.cbuf[rb_shift_index(a, lvl, bh, grp) * D + tid];
+    const float r = a.Y[((int64_t)bh * a.n_v + a.ord[(int64_t)bh * a.n_v + start]) * D + tid];
+    w[tid] = (r - cv) - t * inv_n;
+    a.cbuf[rb_shift_index(a, lvl + 1, bh, 2 * grp) * D + tid] = cv + t * inv_n;
+  }
+  __syncthreads();
+  {
+    const float n0 = rb_norm(w, D, &s_tmp);
+    if (tid < D) w[tid] = n0 > 0.f ? w[tid] / n0 : (tid == 0 ? 1.f : 0.f);
+    __syncthreads();
+  }
+  for (int it = 0; it < iters; ++it) {
+    if (warp == 0) {   // s1 . w
+      float t = 0.f;
+      for (int i = lane; i < D; i += 32) t = fmaf(s1[i], w[i], t);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) s_tmp = t * inv_n;
+    }
+    __syncthreads();
+    if (tid < D) {
+      float t = 0.f;
+      for (int j = 0; j < D; ++j) t = fmaf(G[tid * LD + j], w[j], t);
+      z[tid] = t - s1[tid] * s_tmp;
+    }
+    __syncthreads();
+    const float nz = rb_norm(z, D, &s_tmp);
+    if (!(nz > 0.f)) break;   // uniform
+    if (tid < D) w[tid] = z[tid] / nz;
+    __syncthreads();
+  }
+  if (tid < D) a.wbuf[gidx * D + tid] = w[tid];
+}
+
+// One level of the hierarchy: grid (2^lvl NC, B*H); group blockIdx.x / NC of every head.
+// With NC > 1 the NC CTAs of a cluster share the group: each streams the contiguous
+// slice [lo, hi) of its positions, and the block sums, the radix histograms and the
+// partition's left/right counts are summed over the cluster in rank order through
+// distributed shared memory, so every CTA holds the same mean, axis and pivot.
+// With kAxis the group's split axis is read from a.wbuf (rb_axis_kernel), and
+// only the projection pass streams the rows.
+template <int D, int T, int NC, bool kAxis>
+__device__ __forceinline__ void rb_split_group(const ReblockArgs& a, int lvl, int iters) {
   constexpr int kSplitThreads = T, kSplitWarps = T / 32;
   constexpr int LPR = D / 4, RPW = 32 / LPR, SLOTS = kSplitWarps * RPW;
   __shared__ __align__(16) float4 red[kSplitWarps][LPR];
@@ -594,12 +977,34 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
   __shared__ uint32_t hist[256];
   __shared__ int s_int[4];
   __shared__ float s_tmp;
+  __shared__ __align__(16) float part[NC > 1 ? D : 1];      // this CTA's share of a block sum
+  __shared__ uint32_t htot[NC > 1 ? 256 : 1];               // the cluster's histogram
+  __shared__ int s_cnt[2];                                  // this CTA's left / right counts
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane / LPR, fl = lane % LPR;   // row slot within the warp, lane quad of the row
   const int bh = blockIdx.y;
+  const int grp = blockIdx.x / NC, rank = blockIdx.x % NC;
   int start, len;
-  if (!rb_segment(a.n_v, lvl, blockIdx.x, start, len) || len <= kBlock) return;
+  if (!rb_segment(a.n_v, lvl, grp, start, len) || len <= kBlock) return;   // uniform over the cluster
   const int left = rb_left(len);
+  const int lo = (int)((int64_t)len * rank / NC), hi = (int)((int64_t)len * (rank + 1) / NC);
+  // a block sum of a per-lane float4 over the CTA, then over the cluster (rank order)
+  auto cluster_sum = [&](float4 v, float* out, float scale) {
+    if constexpr (NC == 1) {
+      rb_block_sum<D, kSplitWarps>(v, red, out, scale);
+    } else {
+      namespace cg = cooperative_groups;
+      cg::cluster_group cluster = cg::this_cluster();
+      rb_block_sum<D, kSplitWarps>(v, red, part, 1.f);
+      cluster.sync();
+      if (tid < D) {
+        float t = 0.f;
+        for (int r = 0; r < NC; ++r) t += cluster.map_shared_rank(part, r)[tid];
+        out[tid] = t * scale;
+      }
+      cluster.sync();   // every CTA has read every part; out is visible to the block
+    }
+  };
   int32_t* ord = a.ord + (int64_t)bh * a.n_v + start;
   const float* Y = a.Y + (int64_t)bh * a.n_v * D;
   unsigned long long* key = reinterpret_cast<unsigned long long*>(a.key) + (int64_t)bh * a.n_v + start;
@@ -607,13 +1012,13 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
   // pass over the group's rows, kSplitUnroll rows of a slot in flight
   // (the loop bound is warp-uniform, so the row dot products' shuffles see every lane)
   auto rows_pass = [&](auto&& body) {
-    for (int w0 = warp * RPW; w0 < len; w0 += SLOTS * kSplitUnroll) {
+    for (int w0 = lo + warp * RPW; w0 < hi; w0 += SLOTS * kSplitUnroll) {
       int id[kSplitUnroll];
       float4 y[kSplitUnroll];
 #pragma unroll
       for (int u = 0; u < kSplitUnroll; ++u) {
         const int m = w0 + sub + u * SLOTS;
-        id[u] = m < len ? ord[m] : -1;
+        id[u] = m < hi ? ord[m] : -1;
       }
 #pragma unroll
       for (int u = 0; u < kSplitUnroll; ++u)
@@ -624,12 +1029,16 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
     }
   };
 
+  if constexpr (kAxis) {
+    if (tid < D) w[tid] = a.wbuf[(((int64_t)bh << lvl) + grp) * D + tid];
+    __syncthreads();
+  } else {
   // mean
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   rows_pass([&](int, int id, float4 y) {
     if (id >= 0) { acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w; }
   });
-  rb_block_sum<D, kSplitWarps>(acc, red, mean, 1.f / (float)len);
+  cluster_sum(acc, mean, 1.f / (float)len);
   // start: the first row minus the mean, normalised (e_0 if that is zero)
   if (tid < D) w[tid] = Y[(int64_t)ord[0] * D + tid] - mean[tid];
   __syncthreads();
@@ -648,11 +1057,12 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
       const float p = rb_row_dot<D>(c, wq);
       if (id >= 0) { zq.x = fmaf(c.x, p, zq.x); zq.y = fmaf(c.y, p, zq.y); zq.z = fmaf(c.z, p, zq.z); zq.w = fmaf(c.w, p, zq.w); }
     });
-    rb_block_sum<D, kSplitWarps>(zq, red, z, 1.f);
+    cluster_sum(zq, z, 1.f);
     const float nz = rb_norm(z, D, &s_tmp);
     if (!(nz > 0.f)) break;   // uniform
     if (tid < D) w[tid] = z[tid] / nz;
     __syncthreads();
+  }
   }
   // projections as 64-bit keys: order-preserving float bits, then the row
   {
@@ -676,10 +1086,10 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
     __syncthreads();
     // warp-aggregated counts: the lanes holding one digit add it once (the top
     // digits of nearby projections coincide, so plain atomics would serialise)
-    for (int m0 = warp * 32; m0 < len; m0 += kSplitThreads) {
+    for (int m0 = lo + warp * 32; m0 < hi; m0 += kSplitThreads) {
       const int m = m0 + lane;
       uint32_t dig = 256u;
-      if (m < len) {
+      if (m < hi) {
         const unsigned long long k = key[m];
         if ((k & pmask) == prefix) dig = (uint32_t)((k >> shift) & 255ull);
       }
@@ -687,10 +1097,23 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
       if (dig < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
+    const uint32_t* hs = hist;
+    if constexpr (NC > 1) {   // the cluster's histogram, summed in rank order
+      namespace cg = cooperative_groups;
+      cg::cluster_group cluster = cg::this_cluster();
+      cluster.sync();
+      for (int i = tid; i < 256; i += kSplitThreads) {
+        uint32_t t = 0u;
+        for (int r = 0; r < NC; ++r) t += cluster.map_shared_rank(hist, r)[i];
+        htot[i] = t;
+      }
+      cluster.sync();   // every CTA has read every histogram before the next pass clears its own
+      hs = htot;
+    }
     // the bin holding rank `want`: a parallel exclusive scan of the 256 counts
     uint32_t c = 0u, incl = 0u;
     if (tid < 256) {   // warps 0-7, whole warps
-      c = hist[tid];
+      c = hs[tid];
       incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -715,10 +1138,29 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
   const unsigned long long pivot = prefix;
   // stable partition into tmp: rows with key <= pivot first, in their order
   int32_t* tmp = a.tmp + (int64_t)bh * a.n_v + start;
-  int base_l = 0, base_r = left;
-  for (int c0 = 0; c0 < len; c0 += kSplitThreads) {
+  int base_l = 0, base_r = left, total_l = 0;
+  if constexpr (NC > 1) {   // this CTA's offsets: the left / right counts of the ranks before it
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    int nl = 0;
+    for (int m = lo + tid; m < hi; m += kSplitThreads) nl += key[m] <= pivot ? 1 : 0;
+    nl = __reduce_add_sync(0xffffffffu, (unsigned)nl);
+    if (tid == 0) s_cnt[0] = 0;
+    __syncthreads();
+    if (lane == 0) atomicAdd(&s_cnt[0], nl);
+    __syncthreads();
+    if (tid == 0) s_cnt[1] = (hi - lo) - s_cnt[0];
+    cluster.sync();
+    for (int r = 0; r < NC; ++r) {
+      const int* rc = cluster.map_shared_rank(s_cnt, r);
+      if (r < rank) { base_l += rc[0]; base_r += rc[1]; }
+      total_l += rc[0];
+    }
+    cluster.sync();   // every CTA has read every count
+  }
+  for (int c0 = lo; c0 < hi; c0 += kSplitThreads) {
     const int m = c0 + tid;
-    const bool valid = m < len;
+    const bool valid = m < hi;
     const bool f = valid && key[m] <= pivot;
     const uint32_t bl = __ballot_sync(0xffffffffu, f), bv = __ballot_sync(0xffffffffu, valid);
     const uint32_t below = (1u << lane) - 1u;
@@ -745,9 +1187,28 @@ __global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lv
     base_r += s_int[3];
     __syncthreads();
   }
-  for (int m = tid; m < len; m += kSplitThreads) ord[m] = tmp[m];
-  if (tid == 0 && base_l != left) raise_status(a.status, SOL_ERR_INVALID_ARG);   // cannot happen: keys are distinct
+  if constexpr (NC > 1) {
+    namespace cg = cooperative_groups;
+    cg::this_cluster().sync();   // every CTA's rows are in tmp (release / acquire at cluster scope)
+  } else {
+    total_l = base_l;
+  }
+  for (int m = lo + tid; m < hi; m += kSplitThreads) ord[m] = tmp[m];
+  if (tid == 0 && total_l != left) raise_status(a.status, SOL_ERR_INVALID_ARG);   // cannot happen: keys are distinct
 }
+
+template <int D, int T, bool kAxis>
+__global__ void __launch_bounds__(T) rb_split_kernel(const ReblockArgs a, int lvl, int iters) {
+  rb_split_group<D, T, 1, kAxis>(a, lvl, iters);
+}
+
+// Groups larger than the SM count can cover: NC CTAs of 1,024 threads per group, one cluster each.
+template <int D, int NC, bool kAxis>
+__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(1024) rb_split_cluster_kernel(const ReblockArgs a, int lvl,
+                                                                                            int iters) {
+  rb_split_group<D, 1024, NC, kAxis>(a, lvl, iters);
+}
+
 
 __global__ void rb_perm_kernel(const ReblockArgs a) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -786,6 +1247,24 @@ int reblock_levels(int n_v) {
 
 int reblock_moment_chunks(int n_q) { return (n_q + kMomRows - 1) / kMomRows; }
 
+int reblock_gram_levels(int n_v, int D) {
+  if (D != 128) return 0;
+  const int levels = reblock_levels(n_v);
+  int g = 0;
+  while (g < levels && (n_v >> g) >= kGramMinRows) ++g;
+  return g;
+}
+
+size_t reblock_gram_part_floats(int BH, int n_v, int D) {
+  const int g = reblock_gram_levels(n_v, D);
+  return g == 0 ? 0 : (((size_t)BH << (g - 1)) + kGrCtas) * kGramPartFloats;
+}
+
+size_t reblock_axis_floats(int BH, int n_v, int D) {
+  const int g = reblock_gram_levels(n_v, D);
+  return g == 0 ? 0 : ((size_t)BH << (g - 1)) * 128;
+}
+
 cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
   const int BH = a.B * a.H;
   if (BH == 0 || a.N == 0) return cudaSuccess;
@@ -802,7 +1281,9 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
         (e = cudaFuncSetAttribute(rb_factor_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, f64)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(rb_whiten_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, w64)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(rb_moment_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMomTcSmem)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(rb_whiten_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWhTcSmem)) != cudaSuccess)
+        (e = cudaFuncSetAttribute(rb_whiten_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWhTcSmem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGrSmem)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(rb_axis_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 129 * 4)) != cudaSuccess)
       return e;
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
@@ -831,15 +1312,27 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int levels = reblock_levels(a.n_v);
+    const int tph = (a.n_v + kGrRows - 1) / kGrRows;   // 64-row tiles per head
+    const int chunk = (BH * tph + kGrCtas - 1) / kGrCtas, ngr = (BH * tph + chunk - 1) / chunk;
     for (int lvl = 0; lvl < levels; ++lvl) {
       dim3 gs(1u << lvl, BH);
       const bool wide = (a.n_v >> lvl) > 4096;   // large groups: 1024 threads; small ones: 256, more CTAs per SM
-      if (D == 128) {
-        if (wide) rb_split_kernel<128, 1024><<<gs, 1024, 0, st>>>(a, lvl, iters);
-        else rb_split_kernel<128, 256><<<gs, 256, 0, st>>>(a, lvl, iters);
+      // fewer groups than SMs: two CTAs of one cluster per group
+      const bool pair = wide && (int64_t)BH << lvl < 148;
+      if (lvl < a.gram_levels) {   // D = 128: axes from Gram matrices, then one projection pass
+        if (lvl == 0) rb_shift0_kernel<<<BH, 1024, 0, st>>>(a);
+        rb_gram_tc_kernel<<<ngr, kGrThreads, kGrSmem, st>>>(a, lvl, tph, chunk);
+        rb_axis_kernel<<<gs, 256, 128 * 129 * 4, st>>>(a, lvl, tph, chunk, iters);
+        if (pair) rb_split_cluster_kernel<128, 2, true><<<dim3(2u << lvl, BH), 1024, 0, st>>>(a, lvl, iters);
+        else if (wide) rb_split_kernel<128, 1024, true><<<gs, 1024, 0, st>>>(a, lvl, iters);
+        else rb_split_kernel<128, 256, true><<<gs, 256, 0, st>>>(a, lvl, iters);
+      } else if (D == 128) {
+        if (pair) rb_split_cluster_kernel<128, 2, false><<<dim3(2u << lvl, BH), 1024, 0, st>>>(a, lvl, iters);
+        else if (wide) rb_split_kernel<128, 1024, false><<<gs, 1024, 0, st>>>(a, lvl, iters);
+        else rb_split_kernel<128, 256, false><<<gs, 256, 0, st>>>(a, lvl, iters);
       } else {
-        if (wide) rb_split_kernel<64, 1024><<<gs, 1024, 0, st>>>(a, lvl, iters);
-        else rb_split_kernel<64, 256><<<gs, 256, 0, st>>>(a, lvl, iters);
+        if (wide) rb_split_kernel<64, 1024, false><<<gs, 1024, 0, st>>>(a, lvl, iters);
+        else rb_split_kernel<64, 256, false><<<gs, 256, 0, st>>>(a, lvl, iters);
       }
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
