@@ -636,11 +636,11 @@ __device__ inline bool rb_group_at(int n_v, int lvl, int pos, int& s, int& start
 // CTA index), which is unique.  rb_axis_kernel sums a group's partials in CTA
 // order, forms C, runs the power steps from r - mean (r the group's first row)
 // and records the group's mean for the next level.
-constexpr int kGramMinRows = 2048;   // levels whose groups have at least this many rows
+constexpr int kGramMinRows = 512;    // levels whose groups have at least this many rows
 constexpr int kGrCtas = 148;
 constexpr int kGrRows = 64;          // rows per tile: four K = 16 steps
 constexpr int kGrChunk = 4;          // tiles per TMEM chunk
-constexpr int kGrSlots = 3;          // fp32 staging slots per row: kGrSlots - 1 tiles in flight
+constexpr int kGrSlots = 4;          // fp32 staging slots per row: kGrSlots - 1 tiles in flight
 constexpr int kGrWarps = 16;         // converting warps 0-15; warp 16 issues the MMAs; 17-20 add the chunks
 constexpr int kGrMmaWarp = kGrWarps, kGrEpiWarp = kGrWarps + 1;
 constexpr int kGrThreads = 32 * (kGrWarps + 5);
@@ -1077,7 +1077,9 @@ __device__ __forceinline__ void rb_split_group(const ReblockArgs& a, int lvl, in
     });
   }
   __syncthreads();
-  // radix select of the key of rank left-1 (keys are distinct: the row is in them)
+  // radix select of the key of rank left-1 (keys are distinct: the row is in them);
+  // once the chosen digit's bin holds one key, that key is the only one with the
+  // prefix, so "key <= prefix with every lower bit set" selects the same rows
   unsigned long long prefix = 0ull, pmask = 0ull;
   int want = left - 1;
   for (int pass = 0; pass < 8; ++pass) {
@@ -1127,15 +1129,21 @@ __device__ __forceinline__ void rb_split_group(const ReblockArgs& a, int lvl, in
       uint32_t base = 0u;
       for (int w2 = 0; w2 < warp; ++w2) base += wsum[w2];
       const uint32_t excl = base + incl - c;
-      if (excl <= (uint32_t)want && (uint32_t)want < excl + c) { s_int[0] = tid; s_int[1] = want - (int)excl; }
+      if (excl <= (uint32_t)want && (uint32_t)want < excl + c) {
+        s_int[0] = tid;
+        s_int[1] = want - (int)excl;
+        s_int[2] = (int)c;
+      }
     }
     __syncthreads();
     prefix |= (unsigned long long)s_int[0] << shift;
     pmask |= 255ull << shift;
     want = s_int[1];
+    const bool single = s_int[2] == 1;   // uniform (over the cluster too: the histograms are the same)
     __syncthreads();
+    if (single) break;
   }
-  const unsigned long long pivot = prefix;
+  const unsigned long long pivot = prefix | ~pmask;
   // stable partition into tmp: rows with key <= pivot first, in their order
   int32_t* tmp = a.tmp + (int64_t)bh * a.n_v + start;
   int base_l = 0, base_r = left, total_l = 0;
