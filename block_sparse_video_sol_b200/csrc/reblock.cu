@@ -624,9 +624,9 @@ __device__ inline bool rb_group_at(int n_v, int lvl, int pos, int& s, int& start
 // instead, |mean - c|^2 is about 100 times C's largest eigenvalue.)
 // rb_gram_tc_kernel sums G on the tensor cores: each x (fp32) is split into
 // two bf16 terms h + m (round to nearest each; the rest, below 2^-17 |x|, is
-// dropped), and G = (H + M)^T (H + M) = H^T H + H^T M + M^T H + M^T M.  The
-// dropped rest is a zero-mean rounding residual, so its share of G shrinks
-// with the number of rows.  TMEM accumulates four tiles (256 rows, 16 K steps)
+// dropped), and G = H^T H + H^T M + M^T H.  The dropped rest is a zero-mean
+// rounding residual, so its share of G shrinks with the number of rows; the
+// dropped M^T M is below 2^-18 of H^T H and sits mostly on the diagonal.  TMEM accumulates four tiles (256 rows, 16 K steps)
 // at a time; four epilogue warps add each finished chunk into a running fp32
 // sum (round to nearest) while the MMAs fill the other chunk buffer, so no
 // accumulation in the tensor pipe runs longer than 16 steps.  The level's rows
@@ -640,9 +640,16 @@ constexpr int kGramMinRows = 512;    // levels whose groups have at least this m
 constexpr int kGrCtas = 148;
 constexpr int kGrRows = 64;          // rows per tile: four K = 16 steps
 constexpr int kGrChunk = 4;          // tiles per TMEM chunk
-constexpr int kGrSlots = 4;          // fp32 staging slots per row: kGrSlots - 1 tiles in flight
+#ifndef SOL_GR_SLOTS
+#define SOL_GR_SLOTS 3
+#endif
+#ifndef SOL_GR_STAGES
+#define SOL_GR_STAGES 4
+#endif
+constexpr int kGrSlots = SOL_GR_SLOTS;     // fp32 staging slots per row: kGrSlots - 1 tiles in flight
+constexpr int kGrStages = SOL_GR_STAGES;   // bf16 term stages between the converting warps and the MMAs
 constexpr int kGrWarps = 16;         // converting warps 0-15; warp 16 issues the MMAs; 17-20 add the chunks
-constexpr int kGrMmaWarp = kGrWarps, kGrEpiWarp = kGrWarps + 1;
+constexpr int kGrMmaWarp = kGrWarps;
 constexpr int kGrThreads = 32 * (kGrWarps + 5);
 constexpr int kGrRowsPerWarp = kGrRows / kGrWarps;
 constexpr int kGrTerm = kGrRows * 128 * 2;         // 16 KB: one bf16 term, two 8 KB chunks of 64 dims
@@ -650,11 +657,11 @@ constexpr int kGrStage = 2 * kGrTerm;              // the two terms of a tile
 constexpr int kGrStaging = kGrRows * 128 * 4;      // 32 KB: one fp32 tile
 constexpr int kGramPartFloats = 128 * 128 + 128;   // G, then s1
 struct GrBars {
-  uint64_t full[2], empty[2], accf[2], accr[2], done;
+  uint64_t full[kGrStages], empty[kGrStages], accf[2], accr[2], done;
   uint32_t tmem;
   int abort_flag;
 };
-constexpr size_t kGrSmem = 1024 + 2 * kGrStage + kGrSlots * kGrStaging + kGrWarps * 128 * 4 + sizeof(GrBars);
+constexpr size_t kGrSmem = 1024 + kGrStages * kGrStage + kGrSlots * kGrStaging + sizeof(GrBars);
 static_assert(kGrSmem <= 232448, "Gram kernel shared memory");
 
 // Means of level lvl's groups go to half (lvl + 1) & 1 of cbuf; the shifts of level
@@ -693,17 +700,20 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
   constexpr int D = 128;
   extern __shared__ uint8_t gr_smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gr_smem_raw) + 1023) & ~uintptr_t(1023));
-  float* stg = reinterpret_cast<float*>(ring + 2 * kGrStage);    // [kGrSlots][kGrRows][D]
-  float* s1red = stg + kGrSlots * kGrRows * D;                    // [kGrWarps][D]
-  GrBars& bar = *reinterpret_cast<GrBars*>(s1red + kGrWarps * D);
+  float* stg = reinterpret_cast<float*>(ring + kGrStages * kGrStage);   // [kGrSlots][kGrRows][D]
+  GrBars& bar = *reinterpret_cast<GrBars*>(stg + kGrSlots * kGrRows * D);
+  // a converting warp's s1 goes to the first of its own staging rows once its copies are done
+  auto s1_row = [&](int w) { return stg + w * kGrRowsPerWarp * D; };
   volatile int* abort_flag = &bar.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int TT = a.B * a.H * tph;
   const int t0 = blockIdx.x * chunk, t1 = min(TT, t0 + chunk);
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kGrStages; ++b) {
       mbar_init(&bar.full[b], kGrWarps);
       mbar_init(&bar.empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&bar.accf[b], 1);
       mbar_init(&bar.accr[b], 4);
     }
@@ -765,7 +775,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
         issue(t + kGrSlots - 1, idn);   // empty past the segment's end
         idn = ids_of(t + kGrSlots);     // consumed by the next iteration's issue
         cp_async_wait<kGrSlots - 1>();  // this thread's copies of tile t have landed
-        const int st = (q + t) & 1, n = (q + t) >> 1;
+        const int st = (q + t) % kGrStages, n = (q + t) / kGrStages;
         if (!__all_sync(0xffffffffu, wait_bar(&bar.empty[st], (n & 1) ^ 1, abort_flag, a.status))) break;
         const float* sp = stg + ((t % kGrSlots) * kGrRows + warp * kGrRowsPerWarp) * D + 4 * lane;
         uint8_t* base = ring + st * kGrStage;
@@ -797,7 +807,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
         if (lane == 0) mbar_arrive(&bar.full[st]);
       }
       cp_async_wait<0>();
-      *reinterpret_cast<float4*>(s1red + warp * D + 4 * lane) = s1;
+      *reinterpret_cast<float4*>(s1_row(warp) + 4 * lane) = s1;
     } else if (warp == kGrMmaWarp) {   // M = N = 128 (dims), K = 16 rows, A and B MN-major from the ring
       constexpr uint32_t id = idesc_bf16(128, 128, 1, 1);
       for (int t = 0; t < ntile; ++t) {
@@ -805,7 +815,7 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
         const bool first = t % kGrChunk == 0, last = t % kGrChunk == kGrChunk - 1 || t == ntile - 1;
         // chunk buffer b is free once the epilogue has added its previous chunk
         if (first && !__all_sync(0xffffffffu, wait_bar(&bar.accr[b], (u & 1) ^ 1, abort_flag, a.status))) break;
-        const int st = (q + t) & 1, n = (q + t) >> 1;
+        const int st = (q + t) % kGrStages, n = (q + t) / kGrStages;
         if (!__all_sync(0xffffffffu, wait_bar(&bar.full[st], n & 1, abort_flag, a.status))) break;
         fence_after();
         const uint64_t dH = sdesc(smem_u32(ring + st * kGrStage), kGrTerm / 2, 1024);
@@ -817,7 +827,6 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
           mma_ss_w(acc_addr, dH + o, dH + o, id, (!first || kk > 0) ? 1u : 0u);
           mma_ss_w(acc_addr, dH + o, dM + o, id, 1u);
           mma_ss_w(acc_addr, dM + o, dH + o, id, 1u);
-          mma_ss_w(acc_addr, dM + o, dM + o, id, 1u);
         }
         mma_issued = true;
         mma_commit_w(&bar.empty[st]);
@@ -861,10 +870,10 @@ __global__ void __launch_bounds__(kGrThreads, 1) rb_gram_tc_kernel(const Reblock
         }
       }
     }
-    __syncthreads();   // s1red complete
+    __syncthreads();   // the warps' s1 rows are complete
     if (tid < D) {
       float t = 0.f;
-      for (int w2 = 0; w2 < kGrWarps; ++w2) t += s1red[w2 * D + tid];
+      for (int w2 = 0; w2 < kGrWarps; ++w2) t += s1_row(w2)[tid];
       P[D * D + tid] = t;
     }
     q += ntile;
