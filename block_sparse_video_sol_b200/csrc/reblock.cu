@@ -243,10 +243,27 @@ __global__ void __launch_bounds__(256) rb_factor_kernel(const ReblockArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, bh = blockIdx.x;
   const float* part = a.mpart + (int64_t)bh * a.mchunks * D * D;
   const float inv_n = 1.f / (float)a.n_q;
-  for (int idx = tid; idx < D * D; idx += 256) {
-    float s = 0.f;
-    for (int c = 0; c < a.mchunks; ++c) s += part[(int64_t)c * D * D + idx];
-    M[(idx / D) * LD + idx % D] = s * inv_n;
+  {   // thread tid sums float4 f = tid + 256 k of every chunk's partial, all k's loads in flight
+    constexpr int KF = D * D / 4 / 256;
+    float4 acc[KF];
+#pragma unroll
+    for (int k = 0; k < KF; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < a.mchunks; ++c) {
+      const float4* src = reinterpret_cast<const float4*>(part + (int64_t)c * D * D);
+#pragma unroll
+      for (int k = 0; k < KF; ++k) {
+        const float4 v = src[tid + 256 * k];
+        acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < KF; ++k) {
+      const int idx = 4 * (tid + 256 * k), i = idx / D, j = idx % D;
+      M[i * LD + j] = acc[k].x * inv_n;
+      M[i * LD + j + 1] = acc[k].y * inv_n;
+      M[i * LD + j + 2] = acc[k].z * inv_n;
+      M[i * LD + j + 3] = acc[k].w * inv_n;
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -274,9 +291,19 @@ __global__ void __launch_bounds__(256) rb_factor_kernel(const ReblockArgs a) {
     __syncthreads();
     const float ljj = M[j * LD + j];
     for (int i = j + 1 + tid; i < D; i += 256) {
-      float t = M[i * LD + j];
-      for (int c = 0; c < j; ++c) t = fmaf(-M[i * LD + c], M[j * LD + c], t);
-      M[i * LD + j] = t / ljj;
+      // sum_c<j L[i][c] L[j][c] in four interleaved partial sums (c mod 4), then added in order
+      float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
+      const float* Li = M + i * LD;
+      const float* Lj = M + j * LD;
+      int c = 0;
+      for (; c + 4 <= j; c += 4) {
+        t0 = fmaf(Li[c], Lj[c], t0);
+        t1 = fmaf(Li[c + 1], Lj[c + 1], t1);
+        t2 = fmaf(Li[c + 2], Lj[c + 2], t2);
+        t3 = fmaf(Li[c + 3], Lj[c + 3], t3);
+      }
+      for (; c < j; ++c) t0 = fmaf(Li[c], Lj[c], t0);
+      M[i * LD + j] = (M[i * LD + j] - ((t0 + t1) + (t2 + t3))) / ljj;
     }
     __syncthreads();
   }
@@ -370,164 +397,197 @@ __global__ void __launch_bounds__(256) rb_whiten_kernel(const ReblockArgs a) {
   }
 }
 
-// y = normalise(k L) on the tensor cores (D = 128): grid (ceil(n_v / (128 kWhTcTiles)), B*H),
-// 128 threads.  L (fp32) is split into three bf16 terms L = L1 + L2 + L3 (each the
-// rounding of what the previous ones leave, 2^-24 of L in all), laid out MN-major
-// in shared memory; every 128-row key tile is A (K-major, from TMA) and the three
-// products accumulate in TMEM in fp32: the products are exact and the split is as
-// fine as fp32's own rounding.  Each thread then takes its row (TMEM lane) for the
-// norm and writes the unit vector.  Warps 0-3 read TMEM (warp w: lanes 32w .. 32w+31),
-// warp 1 also issues the MMAs, and warp 4 alone streams the key tiles, so the
-// producer never waits inside a warp that the epilogue needs.
+// y = normalise(k L) on the tensor cores (D = 128).  L (fp32) is split into three
+// bf16 terms L = L1 + L2 + L3 (each the rounding of what the previous ones leave,
+// 2^-24 of L in all), laid out MN-major in shared memory; every 128-row key tile
+// is A (K-major, from TMA) and the three products accumulate in TMEM in fp32: the
+// products are exact and the split is as fine as fp32's own rounding.
+// Persistent: grid min(148, tiles), the tiles of all heads (head-major) split
+// evenly over the CTAs; a CTA converts L again where its range enters a new head.
+// Warp 4 streams the key tiles through a kWhTcStages ring, warp 5 issues the 24
+// MMAs of a tile into one of two TMEM accumulators, and warps 0-3 (warp w: TMEM
+// lanes 32w .. 32w+31) take each row's norm and write the unit vector while the
+// MMAs of the next tile fill the other accumulator.
 constexpr int kWhTcRows = 128;
-constexpr int kWhTcTiles = 8;    // key tiles per CTA
-constexpr int kWhTcThreads = 160;
-constexpr int kWhTcStages = 2;
+constexpr int kWhTcCtas = 148;
+constexpr int kWhTcThreads = 192;
+constexpr int kWhTcStages = 3;
 struct WhBars {
-  uint64_t full[kWhTcStages], empty[kWhTcStages], acc_full, acc_free;
+  uint64_t full[kWhTcStages], empty[kWhTcStages], acc_full[2], acc_free[2], done;
   uint32_t tmem;
   int abort_flag;
 };
 constexpr int kWhTile = kWhTcRows * 128 * 2;     // 32 KB: a K tile, or one bf16 term of L
-constexpr size_t kWhTcSmem = 1024 + (3 + kWhTcStages) * kWhTile + sizeof(WhBars);
+constexpr int kWhStw = 4 * 32 * 33 * 4;          // the epilogue warps' row transposes (padded)
+constexpr size_t kWhTcSmem = 1024 + (3 + kWhTcStages) * kWhTile + kWhStw + sizeof(WhBars);
+static_assert(kWhTcSmem <= 232448, "whitening kernel shared memory");
 
-__global__ void __launch_bounds__(kWhTcThreads) rb_whiten_tc_kernel(const __grid_constant__ CUtensorMap mk, const ReblockArgs a) {
+// grid ceil(tiles / chunk), kWhTcThreads threads; tph = 128-row tiles per head
+__global__ void __launch_bounds__(kWhTcThreads, 1) rb_whiten_tc_kernel(const __grid_constant__ CUtensorMap mk,
+                                                                        const ReblockArgs a, int tph, int chunk) {
   constexpr int D = 128;
   extern __shared__ uint8_t wh_smem_raw[];
   uint8_t* Lt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wh_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = Lt + 3 * kWhTile;
-  WhBars& bar = *reinterpret_cast<WhBars*>(ring + kWhTcStages * kWhTile);
+  float* stw = reinterpret_cast<float*>(ring + kWhTcStages * kWhTile);   // [4][32][33]
+  WhBars& bar = *reinterpret_cast<WhBars*>(reinterpret_cast<uint8_t*>(stw) + kWhStw);
   volatile int* abort_flag = &bar.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-  const int t_first = blockIdx.x * kWhTcTiles;
-  const int ntile = min(kWhTcTiles, (a.n_v + kWhTcRows - 1) / kWhTcRows - t_first);
+  const int TT = a.B * a.H * tph;
+  const int t0 = blockIdx.x * chunk, t1 = min(TT, t0 + chunk);
   if (tid == 0) {
     for (int s = 0; s < kWhTcStages; ++s) { mbar_init(&bar.full[s], 1); mbar_init(&bar.empty[s], 1); }
-    mbar_init(&bar.acc_full, 1);
-    mbar_init(&bar.acc_free, 4);
+    for (int b2 = 0; b2 < 2; ++b2) { mbar_init(&bar.acc_full[b2], 1); mbar_init(&bar.acc_free[b2], 4); }
+    mbar_init(&bar.done, 1);
     bar.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(128));
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(256));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // L's three bf16 terms, MN-major SW128: element (i, j) in chunk j/64, row i, 16-byte unit (j%64)/8
-  // at position unit ^ (i & 7); thread tid converts units tid, tid+160, ... (8 columns each)
-  const float* Lg = a.L + (int64_t)bh * D * D;
-  for (int u = tid; u < D * D / 8; u += kWhTcThreads) {
-    const int i = u / (D / 8), j0 = (u % (D / 8)) * 8;
-    const float4 x0 = *reinterpret_cast<const float4*>(Lg + i * D + j0);
-    const float4 x1 = *reinterpret_cast<const float4*>(Lg + i * D + j0 + 4);
-    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    uint32_t w1[4], w2[4], w3[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      float r0 = x[e], r1 = x[e + 1];
-      const __nv_bfloat162 h1 = __floats2bfloat162_rn(r0, r1);
-      r0 -= __low2float(h1); r1 -= __high2float(h1);
-      const __nv_bfloat162 h2 = __floats2bfloat162_rn(r0, r1);
-      r0 -= __low2float(h2); r1 -= __high2float(h2);
-      const __nv_bfloat162 h3 = __floats2bfloat162_rn(r0, r1);
-      w1[e / 2] = *reinterpret_cast<const uint32_t*>(&h1);
-      w2[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-      w3[e / 2] = *reinterpret_cast<const uint32_t*>(&h3);
-    }
-    const int off = (j0 / 64) * (kWhTile / 2) + i * 128 + ((((j0 % 64) / 8) ^ (i & 7)) << 4);
-    *reinterpret_cast<uint4*>(Lt + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-    *reinterpret_cast<uint4*>(Lt + kWhTile + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-    *reinterpret_cast<uint4*>(Lt + 2 * kWhTile + off) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
   fence_before();
   __syncwarp();
   __syncthreads();
   fence_after();
   const uint32_t tmem = bar.tmem;
-  if (warp == 4 && lane == 0) {   // TMA producer: 128-row key tiles (two 64-dim chunks)
-    int nl = 0;
-    for (int t = 0; t < ntile; ++t) {
-      const int s = t % kWhTcStages, n = t / kWhTcStages;
-      if (!wait_bar(&bar.empty[s], (n & 1) ^ 1, abort_flag, a.status)) break;
-      mbar_expect_tx(&bar.full[s], kWhTile);
-      ++nl;
-      const int row = a.n_fix + (t_first + t) * kWhTcRows;
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(ring + s * kWhTile + c * (kWhTile / 2), &mk, c * 64, h, row, b, &bar.full[s]);
+  int q = 0;   // tiles of this CTA so far (uniform)
+  bool ok = true, mma_issued = false;
+  for (int T = t0; T < t1 && ok;) {   // one segment: the range's tiles of one head
+    const int bh = T / tph, b = bh / a.H, h = bh % a.H;
+    const int Te = min(t1, (bh + 1) * tph), ntile = Te - T, k0 = T - bh * tph;
+    // L's three bf16 terms, MN-major SW128: element (i, j) in chunk j/64, row i, 16-byte unit
+    // (j%64)/8 at position unit ^ (i & 7); thread tid converts units tid, tid+192, ... (8 columns each)
+    const float* Lg = a.L + (int64_t)bh * D * D;
+    for (int u = tid; u < D * D / 8; u += kWhTcThreads) {
+      const int i = u / (D / 8), j0 = (u % (D / 8)) * 8;
+      const float4 x0 = *reinterpret_cast<const float4*>(Lg + i * D + j0);
+      const float4 x1 = *reinterpret_cast<const float4*>(Lg + i * D + j0 + 4);
+      const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      uint32_t w1[4], w2[4], w3[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float r0 = x[e], r1 = x[e + 1];
+        const __nv_bfloat162 h1 = __floats2bfloat162_rn(r0, r1);
+        r0 -= __low2float(h1); r1 -= __high2float(h1);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(r0, r1);
+        r0 -= __low2float(h2); r1 -= __high2float(h2);
+        const __nv_bfloat162 h3 = __floats2bfloat162_rn(r0, r1);
+        w1[e / 2] = *reinterpret_cast<const uint32_t*>(&h1);
+        w2[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+        w3[e / 2] = *reinterpret_cast<const uint32_t*>(&h3);
+      }
+      const int off = (j0 / 64) * (kWhTile / 2) + i * 128 + ((((j0 % 64) / 8) ^ (i & 7)) << 4);
+      *reinterpret_cast<uint4*>(Lt + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      *reinterpret_cast<uint4*>(Lt + kWhTile + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+      *reinterpret_cast<uint4*>(Lt + 2 * kWhTile + off) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
     }
-    for (int s = 0; s < kWhTcStages; ++s) {
-      const int cnt = (nl + kWhTcStages - 1 - s) / kWhTcStages;
-      if (cnt) drain_bar(&bar.full[s], (cnt - 1) & 1, a.status);
-    }
-  }
-  __syncwarp();
-  constexpr uint32_t id = idesc_bf16(128, 128, 0, 1);   // A = keys K-major, B = L terms MN-major
-  const uint64_t ldsc0 = sdesc(smem_u32(Lt), kWhTile / 2, 1024);
-  const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-  bool ok = true;
-  int issued = 0;   // tiles whose MMAs warp 1 committed
-  for (int t = 0; t < ntile && ok && warp < 4; ++t) {
-    const int s = t % kWhTcStages, n = t / kWhTcStages;
-    if (warp == 1) {   // MMAs of tile t once its keys landed and the epilogue read tile t-1
-      ok = __all_sync(0xffffffffu, wait_bar(&bar.full[s], n & 1, abort_flag, a.status) &&
-                                       (t == 0 || wait_bar(&bar.acc_free, (t - 1) & 1, abort_flag, a.status)));
-      if (ok) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
+    __syncthreads();
+    if (warp == 4) {   // TMA producer: 128-row key tiles (two 64-dim chunks)
+      if (lane == 0) {
+        int nl = 0;
+        for (int t = 0; t < ntile; ++t) {
+          const int g = q + t, s = g % kWhTcStages, n = g / kWhTcStages;
+          if (!wait_bar(&bar.empty[s], (n & 1) ^ 1, abort_flag, a.status)) break;
+          mbar_expect_tx(&bar.full[s], kWhTile);
+          ++nl;
+          const int row = a.n_fix + (k0 + t) * kWhTcRows;
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(ring + s * kWhTile + c * (kWhTile / 2), &mk, c * 64, h, row, b, &bar.full[s]);
+        }
+        if (nl < ntile) {   // after an abort: every armed load lands before the CTA moves on
+          for (int t = max(0, nl - kWhTcStages); t < nl; ++t) {   // each stage's last load
+            const int g = q + t;
+            drain_bar(&bar.full[g % kWhTcStages], (g / kWhTcStages) & 1, a.status);
+          }
+        }
+      }
+      __syncwarp();
+    } else if (warp == 5) {   // MMA issuer
+      constexpr uint32_t id = idesc_bf16(128, 128, 0, 1);   // A = keys K-major, B = L terms MN-major
+      const uint64_t ldsc0 = sdesc(smem_u32(Lt), kWhTile / 2, 1024);
+      for (int t = 0; t < ntile; ++t) {
+        const int g = q + t, s = g % kWhTcStages, n = g / kWhTcStages, bb = g & 1, u = g >> 1;
+        // tile g's keys have landed, and accumulator bb's previous tile (g - 2) has been read
+        if (!__all_sync(0xffffffffu, wait_bar(&bar.full[s], n & 1, abort_flag, a.status) &&
+                                         wait_bar(&bar.acc_free[bb], (u & 1) ^ 1, abort_flag, a.status)))
+          break;
         fence_after();
         const uint64_t adsc = sdesc(smem_u32(ring + s * kWhTile), 16, 1024);
+        const uint32_t acc = tmem + 128 * bb;
 #pragma unroll
         for (int term = 0; term < 3; ++term) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t aoff = (uint64_t)(((kk >> 2) * (kWhTile / 2) + (kk & 3) * 32) >> 4);
             const uint64_t boff = (uint64_t)((term * kWhTile + kk * 2048) >> 4);
-            mma_ss_w(tmem, adsc + aoff, ldsc0 + boff, id, (term > 0 || kk > 0) ? 1u : 0u);
+            mma_ss_w(acc, adsc + aoff, ldsc0 + boff, id, (term > 0 || kk > 0) ? 1u : 0u);
           }
         }
+        mma_issued = true;
         mma_commit_w(&bar.empty[s]);
-        mma_commit_w(&bar.acc_full);
-        ++issued;
+        mma_commit_w(&bar.acc_full[bb]);
+      }
+    } else {   // warps 0-3: row 32 warp + lane of each tile from TMEM: its norm, then the unit vector
+      const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+      for (int t = 0; t < ntile; ++t) {
+        const int g = q + t, bb = g & 1, u = g >> 1;
+        if (!__all_sync(0xffffffffu, wait_bar(&bar.acc_full[bb], u & 1, abort_flag, a.status))) break;
+        fence_after();
+        const int row = (k0 + t) * kWhTcRows + 32 * warp + lane;   // position among the video rows
+        float ss = 0.f;
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(lane_addr + 128 * bb + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+        }
+        const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        // second read of the row: the unit vector, 32 columns at a time, turned through shared
+        // memory so that each store writes four whole 128-byte row pieces
+        float* sw = stw + warp * 32 * 33;
+        const int row0 = (k0 + t) * kWhTcRows + 32 * warp;   // the warp's first row
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(lane_addr + 128 * bb + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sw[lane * 33 + e] = v[e] * inv;
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {   // rows 4k + lane / 8, columns 32c + 4 (lane % 8) .. + 3
+            const int r = 4 * k + (lane >> 3), cc = 4 * (lane & 7);
+            if (row0 + r < a.n_v)
+              *reinterpret_cast<float4*>(a.Y + ((int64_t)bh * a.n_v + row0 + r) * D + 32 * c + cc) =
+                  make_float4(sw[r * 33 + cc], sw[r * 33 + cc + 1], sw[r * 33 + cc + 2], sw[r * 33 + cc + 3]);
+          }
+          __syncwarp();
+        }
+        if (row < a.n_v) a.ord[(int64_t)bh * a.n_v + row] = row;
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.acc_free[bb]);   // this warp has read tile g's accumulator
       }
     }
-    // every warp: its 32 rows of y from TMEM, the norms, the unit vectors
-    ok = __all_sync(0xffffffffu, wait_bar(&bar.acc_full, t & 1, abort_flag, a.status));
-    if (!ok) break;
-    fence_after();
-    const int row = (t_first + t) * kWhTcRows + 32 * warp + lane;   // position among the video rows
-    float* Yg = a.Y + ((int64_t)bh * a.n_v + row) * D;
-    float ss = 0.f;
-    for (int c = 0; c < D / 32; ++c) {
-      float v[32];
-      tmem_ld32(lane_addr + 32 * c, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
-    }
-    const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
-    for (int c = 0; c < D / 32; ++c) {   // second read of the row: the unit vector
-      float v[32];
-      tmem_ld32(lane_addr + 32 * c, v);
-      tmem_wait_ld();
-      if (row < a.n_v) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(Yg + 32 * c + e) = make_float4(v[e] * inv, v[e + 1] * inv, v[e + 2] * inv, v[e + 3] * inv);
-      }
-    }
-    if (row < a.n_v) a.ord[(int64_t)bh * a.n_v + row] = row;
+    q += ntile;
+    T = Te;
     fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar.acc_free);   // this warp has read tile t's accumulator
+    ok = !__syncthreads_or(*abort_flag);   // every MMA of the segment has been read: L may change
+    fence_after();
   }
   fence_before();
-  __syncwarp();
   __syncthreads();
-  if (warp == 1) {
-    // every committed product has landed before TMEM is released (on the normal path
-    // the epilogue has waited for each; after an abort, wait for the last one)
-    if (issued > 0) drain_bar(&bar.acc_full, (issued - 1) & 1, a.status);
+  if (warp == 5) {
+    // every issued MMA has landed before TMEM is released (after an abort the
+    // epilogue may not have waited for the last ones)
+    if (mma_issued) {
+      mma_commit_w(&bar.done);
+      drain_bar(&bar.done, 0, a.status);
+    }
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(128));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(256));
   }
 }
 
@@ -1320,8 +1380,9 @@ cudaError_t launch_reblock(const ReblockArgs& a, int iters, cudaStream_t st) {
       CUtensorMap mk;   // 128-row key tiles of the whitening: 64 dims x 128 rows per box, SW128
       const cuuint32_t boxk[4] = {64, 1, kWhTcRows, 1};
       if (!make_map(&mk, a.k, 4, dims4, str4, boxk, kSw128)) return cudaErrorInvalidValue;
-      dim3 gwt((a.n_v + kWhTcRows * kWhTcTiles - 1) / (kWhTcRows * kWhTcTiles), BH);
-      rb_whiten_tc_kernel<<<gwt, kWhTcThreads, kWhTcSmem, st>>>(mk, a);
+      const int wtph = (a.n_v + kWhTcRows - 1) / kWhTcRows;
+      const int wchunk = (BH * wtph + kWhTcCtas - 1) / kWhTcCtas;
+      rb_whiten_tc_kernel<<<(BH * wtph + wchunk - 1) / wchunk, kWhTcThreads, kWhTcSmem, st>>>(mk, a, wtph, wchunk);
     } else {
       rb_moment_kernel<64><<<gm, 256, 0, st>>>(a);
       rb_factor_kernel<64><<<BH, 256, f64, st>>>(a);
