@@ -1078,23 +1078,25 @@ __device__ __forceinline__ void rb_split_group(const ReblockArgs& a, int lvl, in
   const float* Y = a.Y + (int64_t)bh * a.n_v * D;
   unsigned long long* key = reinterpret_cast<unsigned long long*>(a.key) + (int64_t)bh * a.n_v + start;
 
-  // pass over the group's rows, kSplitUnroll rows of a slot in flight
-  // (the loop bound is warp-uniform, so the row dot products' shuffles see every lane)
+  // pass over the group's rows, U rows of a slot in flight (8 when the projections are the
+  // only pass: fewer live values then); the loop bound is warp-uniform, so the row dot
+  // products' shuffles see every lane
+  constexpr int U = kAxis ? 2 * kSplitUnroll : kSplitUnroll;
   auto rows_pass = [&](auto&& body) {
-    for (int w0 = lo + warp * RPW; w0 < hi; w0 += SLOTS * kSplitUnroll) {
-      int id[kSplitUnroll];
-      float4 y[kSplitUnroll];
+    for (int w0 = lo + warp * RPW; w0 < hi; w0 += SLOTS * U) {
+      int id[U];
+      float4 y[U];
 #pragma unroll
-      for (int u = 0; u < kSplitUnroll; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int m = w0 + sub + u * SLOTS;
         id[u] = m < hi ? ord[m] : -1;
       }
 #pragma unroll
-      for (int u = 0; u < kSplitUnroll; ++u)
+      for (int u = 0; u < U; ++u)
         y[u] = id[u] >= 0 ? *reinterpret_cast<const float4*>(Y + (int64_t)id[u] * D + 4 * fl)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < kSplitUnroll; ++u) body(w0 + sub + u * SLOTS, id[u], y[u]);
+      for (int u = 0; u < U; ++u) body(w0 + sub + u * SLOTS, id[u], y[u]);
     }
   };
 
