@@ -237,10 +237,12 @@ sol_status sol_route(const sol_params* p, void* ws, size_t ws_bytes, int32_t* ro
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SOL_ERR_INVALID_ARG, "sol_route: workspace not 256-byte aligned");
   const WsLayout L = ws_layout(*p);
   if (ws_bytes < L.total) return fail(SOL_ERR_WORKSPACE, "sol_route: workspace %zu < %zu bytes", ws_bytes, L.total);
-  if ((s = check_arch()) != SOL_OK) return s;
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   RouteArgs a = route_args(p, L, ws);
   a.mask = at<uint32_t>(ws, L.mask); a.counts = at<int32_t>(ws, L.counts);
+  a.status = status;
   cudaError_t e = launch_route(a, p->D, st);
   if (e != cudaSuccess) return cuda_fail(e, "sol_route launch");
   e = launch_scan_compact(a.mask, a.counts, p->B * p->H * L.nqb, L.mask_words, row_ptr, col_idx, st);
@@ -497,13 +499,15 @@ extern "C" sol_status sol_route_static(const sol_params* p, const void* ws, size
     return fail(SOL_ERR_UNSUPPORTED,
                 "sol_route_static: this problem needs %zu bytes of routing scratch; the built-in array holds %zu "
                 "(use sol_route with a caller-allocated workspace)", need, kRouteScratchBytes);
-  if ((s = check_arch()) != SOL_OK) return s;
+  int* status = nullptr;
+  if ((s = check_arch(&status)) != SOL_OK) return s;
   unsigned char* scratch = nullptr;
   if ((s = route_scratch(&scratch)) != SOL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   RouteArgs a = route_args(p, L, ws);
   a.mask = reinterpret_cast<uint32_t*>(scratch);
   a.counts = reinterpret_cast<int32_t*>(scratch + mask_bytes);
+  a.status = status;
   cudaError_t e = launch_route(a, p->D, st);
   if (e != cudaSuccess) return cuda_fail(e, "sol_route_static launch");
   e = launch_scan_compact(a.mask, a.counts, (int)rows, L.mask_words, row_ptr, col_idx, st);

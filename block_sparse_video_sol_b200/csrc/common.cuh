@@ -97,6 +97,7 @@ struct RouteArgs {
   int topk;                      // > 0: Top-K routing keeping topk key blocks (0: threshold)
   int q128;                      // Top-K query rows are 128-row blocks (both 64-row halves share a list)
   uint32_t* mask; int32_t* counts;
+  int* status;                   // device status word (bounded waits of the tensor-core scores)
 };
 
 struct AttnArgs {

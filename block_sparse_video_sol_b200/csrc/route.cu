@@ -266,6 +266,175 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   }
 }
 
+// Threshold routing with the scores on the tensor cores (D = 128, n_kb <= 512):
+// grid (ceil(n_qb / 128), B*H), 512 threads; thread r < 128 owns query block i0 + r.
+// q̄ and k̄ (fp32) are each split into two bf16 terms, h = bf16(x) and
+// m = bf16(x - h), and S = s·(qh·kh + qh·km + qm·kh) accumulates in fp32 in TMEM:
+// the products of bf16 values are exact, and what is left out (the rest of each
+// operand below 2^-17 of it, and qm·km below 2^-18) is under 4·10^-6 of |q̄||k̄|s,
+// far inside the 10^-4 band in which the routing decision is allowed to differ
+// from the fp64 reading.  The 128 × n_kb score tile fills at most the 512 TMEM
+// columns, so the row statistics and the mask are taken from TMEM, one row per
+// thread: the mean, the population std (two passes, as in route_kernel), then the
+// mask words of the row, 32 columns at a time.  k̄ is converted in chunks of 128
+// key blocks into two shared-memory buffers, so the next chunk's conversion runs
+// beside the current chunk's MMAs.
+constexpr int kRtRows = 128;
+constexpr int kRtThreads = 512;              // all convert; warps 0-3 (TMEM lanes 0-127) take the rows
+constexpr int kRtTerm = kRtRows * 128 * 2;   // 32 KB: one bf16 term of a 128-row tile (two 16 KB chunks of 64 dims)
+struct RtBars {
+  uint64_t mma[2];
+  uint32_t tmem;
+  int abort_flag;
+};
+constexpr size_t kRtSmem = 1024 + 2 * kRtTerm + 2 * 2 * kRtTerm + sizeof(RtBars);
+
+// rows [r0, r0 + 128) of x (fp32 [rows][128], rows >= nrows read as zeros) as two bf16 terms,
+// K-major SW128: row r's dims 8u .. 8u+7 in chunk u / 8 at 16-byte position (u % 8) ^ (r & 7)
+// (kRtThreads threads, each with all four of its 8-dim units' loads in flight at once)
+__device__ __forceinline__ void rt_split_tile(const float* x, int r0, int nrows, uint8_t* th, uint8_t* tm) {
+  constexpr int kPer = kRtRows * 16 / kRtThreads;
+  float4 ld[kPer][2];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = threadIdx.x + kRtThreads * k, r = idx >> 4, u = idx & 15;
+    ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < nrows) {
+      ld[k][0] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u);
+      ld[k][1] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u + 4);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = threadIdx.x + kRtThreads * k, r = idx >> 4, u = idx & 15;
+    const float v[8] = {ld[k][0].x, ld[k][0].y, ld[k][0].z, ld[k][0].w, ld[k][1].x, ld[k][1].y, ld[k][1].z, ld[k][1].w};
+    uint32_t wh[4], wm[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[e], v[e + 1]);
+      const __nv_bfloat162 m = __floats2bfloat162_rn(v[e] - __low2float(h), v[e + 1] - __high2float(h));
+      wh[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+      wm[e / 2] = *reinterpret_cast<const uint32_t*>(&m);
+    }
+    const int off = (u >> 3) * (kRtTerm / 2) + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(th + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4*>(tm + off) = make_uint4(wm[0], wm[1], wm[2], wm[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs a) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t rt_smem_raw[];
+  uint8_t* qt = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* kt = qt + 2 * kRtTerm;   // [2 buffers][2 terms]
+  RtBars& bar = *reinterpret_cast<RtBars*>(kt + 4 * kRtTerm);
+  volatile int* abort_flag = &bar.abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRtRows;
+  const int nch = (a.nkb + kRtRows - 1) / kRtRows;   // 128-block chunks of k̄ (<= 4)
+  const float* qbar = a.qbar + (int64_t)bh * a.nqb * D;
+  const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
+  if (tid == 0) {
+    mbar_init(&bar.mma[0], 1);
+    mbar_init(&bar.mma[1], 1);
+    bar.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  rt_split_tile(qbar, i0, a.nqb, qt, qt + kRtTerm);
+  rt_split_tile(kbar, 0, a.nkb, kt, kt + kRtTerm);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bar.tmem;
+  constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);   // A = q̄ terms, B = k̄ terms, both K-major
+  const uint64_t dqh = sdesc(smem_u32(qt), 16, 1024), dqm = dqh + (uint64_t)(kRtTerm >> 4);
+  bool ok = true;
+  for (int j = 0; j < nch; ++j) {
+    if (warp == 0) {   // chunk j's scores into TMEM columns 128 j .. 128 j + 127
+      const uint64_t dkh = sdesc(smem_u32(kt + (j & 1) * 2 * kRtTerm), 16, 1024), dkm = dkh + (uint64_t)(kRtTerm >> 4);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t o = (uint64_t)(((kk >> 2) * (kRtTerm / 2) + (kk & 3) * 32) >> 4);
+        mma_ss_w(tmem + 128 * j, dqh + o, dkh + o, id, kk > 0 ? 1u : 0u);
+        mma_ss_w(tmem + 128 * j, dqh + o, dkm + o, id, 1u);
+        mma_ss_w(tmem + 128 * j, dqm + o, dkh + o, id, 1u);
+      }
+      mma_commit_w(&bar.mma[j & 1]);
+    }
+    if (j + 1 < nch) {   // chunk j+1 into the other buffer, once chunk j-1's MMAs have read it
+      if (j >= 1) ok = ok && wait_bar(&bar.mma[(j + 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status);
+      if (ok) rt_split_tile(kbar, (j + 1) * kRtRows, a.nkb, kt + ((j + 1) & 1) * 2 * kRtTerm, kt + ((j + 1) & 1) * 2 * kRtTerm + kRtTerm);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_before();
+      ok = !__syncthreads_or(!ok);
+      fence_after();
+      if (!ok) break;
+    }
+  }
+  // every chunk's MMAs have landed (commits complete in order: the last one covers all)
+  ok = ok && wait_bar(&bar.mma[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_flag, a.status);
+  ok = !__syncthreads_or(!ok);   // uniform: the TMEM loads below are warp-collective
+  fence_after();
+  const int i = i0 + tid;
+  // whole warps read TMEM (the loads are warp-collective); rows past n_qb only skip the writes
+  if (ok && warp < 4 && i0 + 32 * warp < a.nqb) {
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
+    const float inv_n = 1.f / (float)a.nkb;
+    const int npiece = (a.nkb + 31) / 32;
+    float sum = 0.f;
+    for (int pc = 0; pc < npiece; ++pc) {
+      float v[32];
+      tmem_ld32(lane_addr + 32 * pc, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sum += (32 * pc + e < a.nkb) ? a.scale * v[e] : 0.f;
+    }
+    const float mu = sum * inv_n;
+    float ss = 0.f;
+    for (int pc = 0; pc < npiece; ++pc) {
+      float v[32];
+      tmem_ld32(lane_addr + 32 * pc, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float t = a.scale * v[e] - mu;
+        ss = (32 * pc + e < a.nkb) ? fmaf(t, t, ss) : ss;
+      }
+    }
+    const float sd = sqrtf(ss * inv_n);
+    const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
+    const bool dense = i < a.n_dense;
+    const int64_t row = (int64_t)bh * a.nqb + i;
+    int cnt = 0;
+    for (int pc = 0; pc < npiece; ++pc) {
+      float v[32];
+      tmem_ld32(lane_addr + 32 * pc, v);
+      tmem_wait_ld();
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int j = 32 * pc + e;
+        const bool sel = j < a.nkb && (dense || j < a.n_sink || a.scale * v[e] > thr);
+        bits |= sel ? (1u << e) : 0u;
+      }
+      if (i < a.nqb) a.mask[row * a.mask_words + pc] = bits;
+      cnt += __popc(bits);
+    }
+    if (i < a.nqb) a.counts[row] = cnt;
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(512));
+  }
+}
+
 // Exclusive scan of the row counts in (b, h, i) order by one CTA.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int rows, int32_t* row_ptr) {
   __shared__ int warp_tot[32];
@@ -332,11 +501,14 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
   if (dev < 0 || dev >= 64 || !prepared[dev].load(std::memory_order_acquire)) {
     const int max128 = (int)route_smem_bytes(128, kMaxKeyBlocks), max64 = (int)route_smem_bytes(64, kMaxKeyBlocks);
     if ((e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, max128)) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, max64)) != cudaSuccess)
+        (e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, max64)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtSmem)) != cudaSuccess)
       return e;
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
-  if (D == 128) route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
+  if (D == 128 && !a.topk && a.nkb <= 4 * kRtRows)   // threshold routing: scores on the tensor cores
+    route_tc_kernel<<<dim3((a.nqb + kRtRows - 1) / kRtRows, a.B * a.H), kRtThreads, kRtSmem, st>>>(a);
+  else if (D == 128) route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
   else route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
   return cudaGetLastError();
 }
