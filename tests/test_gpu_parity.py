@@ -61,6 +61,24 @@ def test_tau_sweep_n8192(tau, lmb):
     assert (0.2 < dens < 0.5) if tau == 0.5 else (0.005 < dens < 0.1)
 
 
+@pytest.mark.parametrize("B,N,H,prefix,tau,grid", [(1, 30001, 2, 200, 1.0, (1, 17, 1753)),
+                                                   (2, 5000, 3, 0, 0.5, (5, 20, 50)),
+                                                   (1, 32768, 1, 64, 2.0, (8, 8, 511))])
+def test_tensor_core_routing_ragged(B, N, H, prefix, tau, grid):
+    """Threshold routing takes its scores from the tensor cores for D = 128 and up to 512 key
+    blocks.  Cases: a partial last 128-block chunk of k-bar and a partial last mask word (469
+    key blocks), a partial last 128-row query tile, two batch entries, sinks and dense rows, and
+    the full 512 key blocks.  The mask must match the oracle outside the 1e-4 band."""
+    w = synth.Workload("rt", B=B, H=H, N=N, D=128, grid=grid, n_topics=8, prefix=prefix, tau=tau, seed=31)
+    q, k, v = synth.generate(w)
+    p, buf = parity.run_gpu(parity.to_dev(q), parity.to_dev(k), parity.to_dev(v), tau, prefix, 0)
+    heads = list(range(H))
+    Qd, Kd, Vd = (synth.bf16_bits_to_f64(x) for x in (q, k, v))
+    qbar, kbar, _ = parity.check_pool(p, buf, Qd, Kd, Vd, heads, 0, prefix)
+    _, flips = parity.check_route(p, buf, qbar, kbar, heads, tau, prefix)
+    print(f"decisions that differ inside the band: {flips}")
+
+
 def test_all_exact_matches_dense_sdpa():
     w = synth.Workload("dense", B=1, H=2, N=700, D=128, grid=(7, 10, 10), n_topics=4, tau=-math.inf, seed=9)
     q, k, v = synth.generate(w)
