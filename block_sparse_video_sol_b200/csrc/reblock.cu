@@ -30,11 +30,20 @@
 //                        three bf16 terms (D = 128; rb_whiten_kernel, fp32
 //                        FMAs with L loaded once per 8 tiles, for D = 64), and
 //                        the initial (identity) order;
-//   rb_split_kernel   -- one launch per level of the hierarchy, one CTA per
-//                        group: mean, power steps, projections as 64-bit keys
-//                        (order-preserving float bits, row index), the split
-//                        rank found by an 8-pass radix select, then a stable
-//                        partition of the group's rows;
+//   per level of the hierarchy, for the levels whose groups hold at least
+//   512 rows (D = 128):
+//     rb_shift0_kernel -- (root only) a sample mean per head, the root's shift;
+//     rb_gram_tc_kernel -- each group's shifted Gram matrix on the tensor cores
+//                        (partials per CTA and group);
+//     rb_axis_kernel  -- one CTA per group: the covariance from the partials,
+//                        the power steps, the group's mean for the next level;
+//     rb_split_kernel / rb_split_cluster_kernel with the axis given -- the
+//                        projection pass, the select and the partition;
+//   for the other levels, rb_split_kernel -- one CTA per group: mean, power
+//                        steps and projections as 64-bit keys (order-
+//                        preserving float bits, row index), the split rank
+//                        found by a radix select, then a stable partition of
+//                        the group's rows;
 //   rb_perm_kernel    -- perm[pos] = original row at position pos;
 //   gather / scatter  -- rows of a BTHD tensor into / out of a head-major
 //                        [B, H, N, D] copy in the partition's order.
