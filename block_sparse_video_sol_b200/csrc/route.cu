@@ -7,12 +7,15 @@
 // Attention Acceleration", section 工作原理 > Sol (Q64/K64 threshold routing,
 // prefix KV sink, dense prefix query rows).
 //
-// The score S = s * qbar kbar^T is a small fp32 contraction (2*nqb*nkb*D flop
-// per head).  It stays on the fp32 FMA pipe: TF32 tensor cores would put
-// ~1e-3 relative error on scores that are compared against a threshold.
-// One CTA owns 32 query blocks of one (b, h) and all key blocks; it keeps
-// its 32 x nkb score rows in shared memory so that the mean, the population
-// std and the mask come from one evaluation of S.
+// The score S = s * qbar kbar^T is a small contraction (2*nqb*nkb*D flop per
+// head) compared against a threshold, so it needs fp32 accuracy: TF32 would
+// put ~1e-3 relative error on it.  Threshold routing with D = 128 and at most
+// 512 key blocks (route_tc_kernel) runs it on the tensor cores with each
+// operand split into two bf16 terms, the score tile held in TMEM.  The other
+// cases (Top-K, D = 64, longer key sequences) use route_kernel on the fp32
+// FMA pipe: one CTA owns 32 query blocks of one (b, h) and all key blocks and
+// keeps its 32 x nkb score rows in shared memory, so that the mean, the
+// population std and the mask come from one evaluation of S.
 //
 // The same kernel does Top-K routing: a warp finds each row's k-th largest
 // score exactly by a bitwise binary search over order-preserving integer
