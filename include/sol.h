@@ -177,7 +177,9 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
  *            the two halves of a 128-row block carry the same list).
  *   col_idx  int32 device, capacity sol_col_capacity(p); row r's exact key
  *            blocks, ascending, at [row_ptr[r], row_ptr[r+1]).
- * Routing 0: S_ij = s * qbar_i . kbar_j in fp32; block j is exact for row i
+ * Routing 0: S_ij = s * qbar_i . kbar_j to fp32 accuracy (for D = 128 and at
+ * most 512 key blocks from bf16 hi/lo terms on the tensor cores, within
+ * 4e-6 * |qbar_i||kbar_j| s of the fp32 dot product); block j is exact for row i
  * iff S_ij > mean_j S_ij + tau * std_j S_ij (population std over all key
  * blocks), or j is a sink block, or i is a dense (prefix) query block.
  * Routing 1: qbar_i over 128 rows; row i keeps its k largest S_ij (equal
@@ -269,7 +271,8 @@ sol_status sol_last_device_status(void* stream);
  * other fields must still pass the common validation.  The workspace (device,
  * 256-byte aligned, >= sol_reblock_workspace_bytes, which may be 0 when
  * every row is a prefix-block row) holds fp32 whitened keys, partial
- * moments, the factor and the split scratch (about 1.03 GB at B=1, H=56,
+ * moments (reused for the levels' Gram partials), the factor, the split
+ * scratch, the split axes and the group means (about 1.22 GB at B=1, H=56,
  * N=32768, D=128); it may be reused once the stream has passed the call.
  *
  * A reblocked forward pass: sol_reblock; sol_gather_rows of q, k and v into
