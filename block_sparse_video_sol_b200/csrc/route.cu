@@ -293,24 +293,29 @@ struct RtBars {
 constexpr size_t kRtSmem = 1024 + 2 * kRtTerm + 2 * 2 * kRtTerm + sizeof(RtBars);
 
 // rows [r0, r0 + 128) of x (fp32 [rows][128], rows >= nrows read as zeros) as two bf16 terms,
-// K-major SW128: row r's dims 8u .. 8u+7 in chunk u / 8 at 16-byte position (u % 8) ^ (r & 7)
-// (kRtThreads threads, each with all four of its 8-dim units' loads in flight at once)
-__device__ __forceinline__ void rt_split_tile(const float* x, int r0, int nrows, uint8_t* th, uint8_t* tm) {
-  constexpr int kPer = kRtRows * 16 / kRtThreads;
-  float4 ld[kPer][2];
+// K-major SW128: row r's dims 8u .. 8u+7 in chunk u / 8 at 16-byte position (u % 8) ^ (r & 7).
+// Thread t handles the 8-dim units t + kRtThreads k; rt_load issues all of its loads at once
+// and rt_store splits and writes them, so other work can sit between the two.
+constexpr int kRtPer = kRtRows * 16 / kRtThreads;
+struct RtLoad { float4 v[kRtPer][2]; };
+__device__ __forceinline__ RtLoad rt_load(const float* x, int r0, int nrows) {
+  RtLoad l;
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
+  for (int k = 0; k < kRtPer; ++k) {
     const int idx = threadIdx.x + kRtThreads * k, r = idx >> 4, u = idx & 15;
-    ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    l.v[k][0] = l.v[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + r < nrows) {
-      ld[k][0] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u);
-      ld[k][1] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u + 4);
+      l.v[k][0] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u);
+      l.v[k][1] = *reinterpret_cast<const float4*>(x + (int64_t)(r0 + r) * 128 + 8 * u + 4);
     }
   }
+  return l;
+}
+__device__ __forceinline__ void rt_store(const RtLoad& l, uint8_t* th, uint8_t* tm) {
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
+  for (int k = 0; k < kRtPer; ++k) {
     const int idx = threadIdx.x + kRtThreads * k, r = idx >> 4, u = idx & 15;
-    const float v[8] = {ld[k][0].x, ld[k][0].y, ld[k][0].z, ld[k][0].w, ld[k][1].x, ld[k][1].y, ld[k][1].z, ld[k][1].w};
+    const float v[8] = {l.v[k][0].x, l.v[k][0].y, l.v[k][0].z, l.v[k][0].w, l.v[k][1].x, l.v[k][1].y, l.v[k][1].z, l.v[k][1].w};
     uint32_t wh[4], wm[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
@@ -347,8 +352,12 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  rt_split_tile(qbar, i0, a.nqb, qt, qt + kRtTerm);
-  rt_split_tile(kbar, 0, a.nkb, kt, kt + kRtTerm);
+  {
+    const RtLoad lq = rt_load(qbar, i0, a.nqb);
+    const RtLoad lk = rt_load(kbar, 0, a.nkb);
+    rt_store(lq, qt, qt + kRtTerm);
+    rt_store(lk, kt, kt + kRtTerm);
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
   fence_before();
   __syncthreads();
@@ -370,8 +379,9 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
       mma_commit_w(&bar.mma[j & 1]);
     }
     if (j + 1 < nch) {   // chunk j+1 into the other buffer, once chunk j-1's MMAs have read it
+      const RtLoad lk = rt_load(kbar, (j + 1) * kRtRows, a.nkb);   // in flight during the wait
       if (j >= 1) ok = ok && wait_bar(&bar.mma[(j + 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status);
-      if (ok) rt_split_tile(kbar, (j + 1) * kRtRows, a.nkb, kt + ((j + 1) & 1) * 2 * kRtTerm, kt + ((j + 1) & 1) * 2 * kRtTerm + kRtTerm);
+      if (ok) rt_store(lk, kt + ((j + 1) & 1) * 2 * kRtTerm, kt + ((j + 1) & 1) * 2 * kRtTerm + kRtTerm);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       fence_before();
       ok = !__syncthreads_or(!ok);
