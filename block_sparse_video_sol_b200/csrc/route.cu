@@ -270,16 +270,16 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
 }
 
 // Threshold routing with the scores on the tensor cores (D = 128, n_kb <= 512):
-// grid (ceil(n_qb / 128), B*H), 512 threads; thread r < 128 owns query block i0 + r.
+// grid (ceil(n_qb / 128), B*H), 512 threads; query block i0 + r is TMEM lane r.
 // q̄ and k̄ (fp32) are each split into two bf16 terms, h = bf16(x) and
 // m = bf16(x - h), and S = s·(qh·kh + qh·km + qm·kh) accumulates in fp32 in TMEM:
 // the products of bf16 values are exact, and what is left out (the rest of each
 // operand below 2^-17 of it, and qm·km below 2^-18) is under 4·10^-6 of |q̄||k̄|s,
 // far inside the 10^-4 band in which the routing decision is allowed to differ
 // from the fp64 reading.  The 128 × n_kb score tile fills at most the 512 TMEM
-// columns, so the row statistics and the mask are taken from TMEM, one row per
-// thread: the mean, the population std (two passes, as in route_kernel), then the
-// mask words of the row, 32 columns at a time.  k̄ is converted in chunks of 128
+// columns, so the row statistics and the mask are taken from TMEM, four threads
+// per row (a quarter of its columns each): the mean, the population std (two
+// passes, as in route_kernel), then the mask words of the row, 32 columns at a time.  k̄ is converted in chunks of 128
 // key blocks into two shared-memory buffers, so the next chunk's conversion runs
 // beside the current chunk's MMAs.
 constexpr int kRtRows = 128;
@@ -393,38 +393,53 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
   ok = ok && wait_bar(&bar.mma[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_flag, a.status);
   ok = !__syncthreads_or(!ok);   // uniform: the TMEM loads below are warp-collective
   fence_after();
-  const int i = i0 + tid;
-  // whole warps read TMEM (the loads are warp-collective); rows past n_qb only skip the writes
-  if (ok && warp < 4 && i0 + 32 * warp < a.nqb) {
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16);
-    const float inv_n = 1.f / (float)a.nkb;
-    const int npiece = (a.nkb + 31) / 32;
-    float sum = 0.f;
-    for (int pc = 0; pc < npiece; ++pc) {
+  // Every warp takes part: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows), and of each row
+  // the 32-column pieces pc with pc % 4 == w / 4.  The four partial sums of a row are added in
+  // shared memory in a fixed order.  Whole warps read TMEM (the loads are warp-collective);
+  // rows past n_qb only skip the writes.
+  __shared__ float rsum[4][kRtRows];
+  __shared__ int rcnt[4][kRtRows];
+  const int quad = warp & 3, part = warp >> 2, rr = 32 * quad + lane, i = i0 + rr;
+  const bool live = ok && i0 + 32 * quad < a.nqb;   // uniform per warp
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * quad) << 16);
+  const float inv_n = 1.f / (float)a.nkb;
+  const int npiece = (a.nkb + 31) / 32;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (live) {
+    for (int pc = part; pc < npiece; pc += 4) {
       float v[32];
       tmem_ld32(lane_addr + 32 * pc, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) sum += (32 * pc + e < a.nkb) ? a.scale * v[e] : 0.f;
+      for (int e = 0; e < 32; ++e) acc[e & 3] += (32 * pc + e < a.nkb) ? a.scale * v[e] : 0.f;
     }
-    const float mu = sum * inv_n;
-    float ss = 0.f;
-    for (int pc = 0; pc < npiece; ++pc) {
+  }
+  rsum[part][rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  __syncthreads();
+  const float mu = ((rsum[0][rr] + rsum[1][rr]) + (rsum[2][rr] + rsum[3][rr])) * inv_n;
+  __syncthreads();
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  if (live) {
+    for (int pc = part; pc < npiece; pc += 4) {
       float v[32];
       tmem_ld32(lane_addr + 32 * pc, v);
       tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float t = a.scale * v[e] - mu;
-        ss = (32 * pc + e < a.nkb) ? fmaf(t, t, ss) : ss;
+        acc[e & 3] = (32 * pc + e < a.nkb) ? fmaf(t, t, acc[e & 3]) : acc[e & 3];
       }
     }
-    const float sd = sqrtf(ss * inv_n);
-    const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
-    const bool dense = i < a.n_dense;
-    const int64_t row = (int64_t)bh * a.nqb + i;
-    int cnt = 0;
-    for (int pc = 0; pc < npiece; ++pc) {
+  }
+  rsum[part][rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  __syncthreads();
+  const float sd = sqrtf(((rsum[0][rr] + rsum[1][rr]) + (rsum[2][rr] + rsum[3][rr])) * inv_n);
+  const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
+  const bool dense = i < a.n_dense;
+  const int64_t row = (int64_t)bh * a.nqb + i;
+  int cnt = 0;
+  if (live) {
+    for (int pc = part; pc < npiece; pc += 4) {
       float v[32];
       tmem_ld32(lane_addr + 32 * pc, v);
       tmem_wait_ld();
@@ -438,8 +453,10 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
       if (i < a.nqb) a.mask[row * a.mask_words + pc] = bits;
       cnt += __popc(bits);
     }
-    if (i < a.nqb) a.counts[row] = cnt;
   }
+  rcnt[part][rr] = cnt;
+  __syncthreads();
+  if (live && part == 0 && i < a.nqb) a.counts[row] = (rcnt[0][rr] + rcnt[1][rr]) + (rcnt[2][rr] + rcnt[3][rr]);
   fence_before();
   __syncthreads();
   if (warp == 0) {
