@@ -465,21 +465,21 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
   }
 }
 
-// Exclusive scan of the row counts in (b, h, i) order by one CTA.
+// Exclusive scan of the row counts in (b, h, i) order by one CTA: warp w owns
+// the rows [w c, (w + 1) c) (c a multiple of 32), read 32 at a time (coalesced);
+// pass 1 sums them, the warp totals are scanned, pass 2 scans each 32-row step
+// with shuffles and carries the running offset.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int rows, int32_t* row_ptr) {
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (rows + 1023) / 1024;
-  const int lo = min(rows, tid * per), hi = min(rows, lo + per);
+  const int c = ((rows + 1023) / 1024) * 32;
+  const int lo = min(rows, warp * c), hi = min(rows, lo + c);
   int s = 0;
-  for (int r = lo; r < hi; ++r) s += counts[r];
-  int incl = s;
+#pragma unroll 4
+  for (int r = lo + lane; r < hi; r += 32) s += counts[r];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) warp_tot[warp] = s;
   __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
   __syncthreads();
   if (warp == 0) {
@@ -489,13 +489,25 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* counts, int r
       const int y = __shfl_up_sync(0xffffffffu, ti, o);
       if (lane >= o) ti += y;
     }
-    warp_tot[lane] = ti - t;  // exclusive warp offsets
+    warp_tot[lane] = ti - t;   // exclusive warp offsets
+    if (lane == 31) row_ptr[rows] = ti;
   }
-  __syncwarp();   // re-converge the warp first: bar.sync is an aligned barrier
+  __syncwarp();
   __syncthreads();
-  int run = warp_tot[warp] + incl - s;
-  for (int r = lo; r < hi; ++r) { row_ptr[r] = run; run += counts[r]; }
-  if (tid == 1023) row_ptr[rows] = warp_tot[31] + incl;
+  int carry = warp_tot[warp];
+#pragma unroll 4
+  for (int r0 = lo; r0 < hi; r0 += 32) {   // warp-uniform bounds
+    const int r = r0 + lane;
+    const int v = r < hi ? counts[r] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (r < hi) row_ptr[r] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
 }
 
 // One warp per row: bitmap words -> ascending column indices at row_ptr[row].
