@@ -190,6 +190,18 @@ def test_ragged_reblocked_forward(N, D, prefix):
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
 
 
+def test_batch2_gram_levels_split_like_the_oracle():
+    """B = 2 through the Gram-axis levels (groups of 512 rows or more, D = 128): 2,036 video
+    rows per head (three Gram levels, then the streamed levels), a prefix that is not block
+    aligned, and two heads per batch entry; every split is checked on its own members."""
+    B, N, H, D, prefix = 2, 2100, 2, 128, 40
+    q, k = (synth.random_bf16((B, N, H, D), seed=s) for s in (41, 42))
+    perm = _gpu_perm(to_dev(q), to_dev(k), prefix, D)
+    _valid(perm, N, prefix)
+    rep = _check_every_split(synth.bf16_bits_to_f64(q), synth.bf16_bits_to_f64(k), perm, prefix, 0.95)
+    assert rep.levels == 5 and rep.groups == B * H * 31
+
+
 def test_all_prefix_and_empty_partitions():
     """P = N: nothing to partition, the order is the identity; N = 0: nothing runs."""
     from block_sparse_video_sol_b200 import sol
