@@ -10,9 +10,9 @@
 // The score S = s * qbar kbar^T is a small contraction (2*nqb*nkb*D flop per
 // head) compared against a threshold, so it needs fp32 accuracy: TF32 would
 // put ~1e-3 relative error on it.  Threshold routing with D = 128 and at most
-// 512 key blocks (route_tc_kernel) runs it on the tensor cores with each
+// 1024 key blocks (route_tc_kernel) runs it on the tensor cores with each
 // operand split into two bf16 terms, the score tile held in TMEM.  The other
-// cases (Top-K, D = 64, longer key sequences) use route_kernel on the fp32
+// cases (Top-K, D = 64) use route_kernel on the fp32
 // FMA pipe: one CTA owns 32 query blocks of one (b, h) and all key blocks and
 // keeps its 32 x nkb score rows in shared memory, so that the mean, the
 // population std and the mask come from one evaluation of S.
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
   }
 }
 
-// Threshold routing with the scores on the tensor cores (D = 128, n_kb <= 512):
+// Threshold routing with the scores on the tensor cores (D = 128, n_kb <= 1024):
 // grid (ceil(n_qb / 128), B*H), 512 threads; query block i0 + r is TMEM lane r.
 // q̄ and k̄ (fp32) are each split into two bf16 terms, h = bf16(x) and
 // m = bf16(x - h), and S = s·(qh·kh + qh·km + qm·kh) accumulates in fp32 in TMEM:
@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(256) route_kernel(const RouteArgs a, int ldS) 
 // from the fp64 reading.  The 128 × n_kb score tile fills at most the 512 TMEM
 // columns, so the row statistics and the mask are taken from TMEM, four threads
 // per row (a quarter of its columns each): the mean, the population std (two
-// passes, as in route_kernel), then the mask words of the row, 32 columns at a time.  k̄ is converted in chunks of 128
+// passes, as in route_kernel), then the mask words of the row, 32 columns at a time.
+// Past 512 key blocks TMEM holds one half of the row at a time, and each half's
+// scores are computed again where a pass needs them (four MMA passes in all).  k̄ is converted in chunks of 128
 // key blocks into two shared-memory buffers, so the next chunk's conversion runs
 // beside the current chunk's MMAs.
 constexpr int kRtRows = 128;
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
   volatile int* abort_flag = &bar.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y, i0 = blockIdx.x * kRtRows;
-  const int nch = (a.nkb + kRtRows - 1) / kRtRows;   // 128-block chunks of k̄ (<= 4)
+  const int nch = (a.nkb + kRtRows - 1) / kRtRows;   // 128-block chunks of k̄ (<= 8)
   const float* qbar = a.qbar + (int64_t)bh * a.nqb * D;
   const float* kbar = a.kbar + (int64_t)bh * a.nkb * D;
   if (tid == 0) {
@@ -354,11 +356,8 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
   }
   {
     const RtLoad lq = rt_load(qbar, i0, a.nqb);
-    const RtLoad lk = rt_load(kbar, 0, a.nkb);
     rt_store(lq, qt, qt + kRtTerm);
-    rt_store(lk, kt, kt + kRtTerm);
   }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
   fence_before();
   __syncthreads();
   fence_after();
@@ -366,100 +365,153 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
   constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);   // A = q̄ terms, B = k̄ terms, both K-major
   const uint64_t dqh = sdesc(smem_u32(qt), 16, 1024), dqm = dqh + (uint64_t)(kRtTerm >> 4);
   bool ok = true;
-  for (int j = 0; j < nch; ++j) {
-    if (warp == 0) {   // chunk j's scores into TMEM columns 128 j .. 128 j + 127
-      const uint64_t dkh = sdesc(smem_u32(kt + (j & 1) * 2 * kRtTerm), 16, 1024), dkm = dkh + (uint64_t)(kRtTerm >> 4);
+  int gc = 0;   // chunk instances run so far: instance g converts into buffer g & 1, commits to mma[g & 1]
+  // The scores of key blocks [512 h, 512 h + 512) into TMEM columns 0 .. 511 (chunk j of the
+  // half at columns 128 j); every MMA of the half has completed on return (ok uniform).
+  int ncommit = 0;   // chunk instances whose MMAs were committed (uniform)
+  auto run_half = [&](int h) {
+    if (!ok) return;   // uniform
+    const int j0 = 4 * h, j1 = min(nch, 4 * h + 4);
+    {   // the half's first chunk (its buffer was last read by instance gc - 2, complete by now)
+      const RtLoad lk = rt_load(kbar, j0 * kRtRows, a.nkb);
+      rt_store(lk, kt + (gc & 1) * 2 * kRtTerm, kt + (gc & 1) * 2 * kRtTerm + kRtTerm);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
+    fence_before();
+    __syncthreads();   // also: the previous passes' TMEM reads are done before these MMAs
+    fence_after();
+    for (int j = j0; j < j1; ++j) {
+      const int g = gc + (j - j0);
+      if (warp == 0) {
+        const uint64_t dkh = sdesc(smem_u32(kt + (g & 1) * 2 * kRtTerm), 16, 1024), dkm = dkh + (uint64_t)(kRtTerm >> 4);
+        const uint32_t col = tmem + 128 * (j - j0);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t o = (uint64_t)(((kk >> 2) * (kRtTerm / 2) + (kk & 3) * 32) >> 4);
-        mma_ss_w(tmem + 128 * j, dqh + o, dkh + o, id, kk > 0 ? 1u : 0u);
-        mma_ss_w(tmem + 128 * j, dqh + o, dkm + o, id, 1u);
-        mma_ss_w(tmem + 128 * j, dqm + o, dkh + o, id, 1u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t o = (uint64_t)(((kk >> 2) * (kRtTerm / 2) + (kk & 3) * 32) >> 4);
+          mma_ss_w(col, dqh + o, dkh + o, id, kk > 0 ? 1u : 0u);
+          mma_ss_w(col, dqh + o, dkm + o, id, 1u);
+          mma_ss_w(col, dqm + o, dkh + o, id, 1u);
+        }
+        mma_commit_w(&bar.mma[g & 1]);
       }
-      mma_commit_w(&bar.mma[j & 1]);
+      ncommit = g + 1;
+      if (j + 1 < j1) {   // chunk j+1 into the other buffer, once instance g-1's MMAs have read it
+        const RtLoad lk = rt_load(kbar, (j + 1) * kRtRows, a.nkb);   // in flight during the wait
+        if (g >= 1) ok = ok && wait_bar(&bar.mma[(g + 1) & 1], ((g - 1) >> 1) & 1, abort_flag, a.status);
+        if (ok) rt_store(lk, kt + ((g + 1) & 1) * 2 * kRtTerm, kt + ((g + 1) & 1) * 2 * kRtTerm + kRtTerm);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        fence_before();
+        ok = !__syncthreads_or(!ok);
+        fence_after();
+        if (!ok) break;
+      }
     }
-    if (j + 1 < nch) {   // chunk j+1 into the other buffer, once chunk j-1's MMAs have read it
-      const RtLoad lk = rt_load(kbar, (j + 1) * kRtRows, a.nkb);   // in flight during the wait
-      if (j >= 1) ok = ok && wait_bar(&bar.mma[(j + 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status);
-      if (ok) rt_store(lk, kt + ((j + 1) & 1) * 2 * kRtTerm, kt + ((j + 1) & 1) * 2 * kRtTerm + kRtTerm);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      fence_before();
-      ok = !__syncthreads_or(!ok);
-      fence_after();
-      if (!ok) break;
-    }
-  }
-  // every chunk's MMAs have landed (commits complete in order: the last one covers all)
-  ok = ok && wait_bar(&bar.mma[(nch - 1) & 1], ((nch - 1) >> 1) & 1, abort_flag, a.status);
-  ok = !__syncthreads_or(!ok);   // uniform: the TMEM loads below are warp-collective
-  fence_after();
-  // Every warp takes part: warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows), and of each row
-  // the 32-column pieces pc with pc % 4 == w / 4.  The four partial sums of a row are added in
-  // shared memory in a fixed order.  Whole warps read TMEM (the loads are warp-collective);
-  // rows past n_qb only skip the writes.
+    // every chunk's MMAs have landed (commits complete in order: the last one covers all)
+    const int gl = gc + (j1 - j0) - 1;
+    ok = ok && wait_bar(&bar.mma[gl & 1], (gl >> 1) & 1, abort_flag, a.status);
+    ok = !__syncthreads_or(!ok);   // uniform: the TMEM loads that follow are warp-collective
+    fence_after();
+    gc += j1 - j0;
+  };
+  // Row passes over the half in TMEM.  Every warp takes part: warp w reads TMEM lanes
+  // 32 (w % 4) .. + 31 (rows), and of each row the 32-column pieces pc with pc % 4 == w / 4.
+  // The four partial sums of a row are added in shared memory in a fixed order.  Whole
+  // warps read TMEM (the loads are warp-collective); rows past n_qb only skip the writes.
   __shared__ float rsum[4][kRtRows];
   __shared__ int rcnt[4][kRtRows];
   const int quad = warp & 3, part = warp >> 2, rr = 32 * quad + lane, i = i0 + rr;
-  const bool live = ok && i0 + 32 * quad < a.nqb;   // uniform per warp
   const uint32_t lane_addr = tmem + ((uint32_t)(32 * quad) << 16);
   const float inv_n = 1.f / (float)a.nkb;
-  const int npiece = (a.nkb + 31) / 32;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (live) {
-    for (int pc = part; pc < npiece; pc += 4) {
-      float v[32];
-      tmem_ld32(lane_addr + 32 * pc, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) acc[e & 3] += (32 * pc + e < a.nkb) ? a.scale * v[e] : 0.f;
-    }
-  }
-  rsum[part][rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  __syncthreads();
-  const float mu = ((rsum[0][rr] + rsum[1][rr]) + (rsum[2][rr] + rsum[3][rr])) * inv_n;
-  __syncthreads();
-  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-  if (live) {
-    for (int pc = part; pc < npiece; pc += 4) {
-      float v[32];
-      tmem_ld32(lane_addr + 32 * pc, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float t = a.scale * v[e] - mu;
-        acc[e & 3] = (32 * pc + e < a.nkb) ? fmaf(t, t, acc[e & 3]) : acc[e & 3];
-      }
-    }
-  }
-  rsum[part][rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  __syncthreads();
-  const float sd = sqrtf(((rsum[0][rr] + rsum[1][rr]) + (rsum[2][rr] + rsum[3][rr])) * inv_n);
-  const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
   const bool dense = i < a.n_dense;
   const int64_t row = (int64_t)bh * a.nqb + i;
-  int cnt = 0;
-  if (live) {
-    for (int pc = part; pc < npiece; pc += 4) {
-      float v[32];
-      tmem_ld32(lane_addr + 32 * pc, v);
-      tmem_wait_ld();
-      uint32_t bits = 0u;
+  const int nh = (nch + 3) / 4;   // halves of up to 512 key blocks (TMEM holds one)
+  auto live = [&]() { return ok && i0 + 32 * quad < a.nqb; };   // uniform per warp
+  auto pieces = [&](int h) { return (min(a.nkb - 512 * h, 512) + 31) / 32; };
+  auto row_total = [&](float x) {   // the four quarters of each row, in order
+    rsum[part][rr] = x;
+    __syncthreads();
+    const float t = (rsum[0][rr] + rsum[1][rr]) + (rsum[2][rr] + rsum[3][rr]);
+    __syncthreads();
+    return t;
+  };
+  auto pass_sum = [&](int h) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live()) {
+      for (int pc = part; pc < pieces(h); pc += 4) {
+        float v[32];
+        tmem_ld32(lane_addr + 32 * pc, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = 32 * pc + e;
-        const bool sel = j < a.nkb && (dense || j < a.n_sink || a.scale * v[e] > thr);
-        bits |= sel ? (1u << e) : 0u;
+        for (int e = 0; e < 32; ++e) acc[e & 3] += (512 * h + 32 * pc + e < a.nkb) ? a.scale * v[e] : 0.f;
       }
-      if (i < a.nqb) a.mask[row * a.mask_words + pc] = bits;
-      cnt += __popc(bits);
     }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  };
+  auto pass_ss = [&](int h, float mu) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live()) {
+      for (int pc = part; pc < pieces(h); pc += 4) {
+        float v[32];
+        tmem_ld32(lane_addr + 32 * pc, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float t = a.scale * v[e] - mu;
+          acc[e & 3] = (512 * h + 32 * pc + e < a.nkb) ? fmaf(t, t, acc[e & 3]) : acc[e & 3];
+        }
+      }
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  };
+  auto pass_mask = [&](int h, float thr) {
+    int cnt = 0;
+    if (live()) {
+      for (int pc = part; pc < pieces(h); pc += 4) {
+        float v[32];
+        tmem_ld32(lane_addr + 32 * pc, v);
+        tmem_wait_ld();
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = 512 * h + 32 * pc + e;
+          const bool sel = j < a.nkb && (dense || j < a.n_sink || a.scale * v[e] > thr);
+          bits |= sel ? (1u << e) : 0u;
+        }
+        if (i < a.nqb) a.mask[row * a.mask_words + 16 * h + pc] = bits;
+        cnt += __popc(bits);
+      }
+    }
+    return cnt;
+  };
+  float mu, sd;
+  int cnt;
+  if (nh == 1) {   // up to 512 key blocks: one MMA pass, three row passes
+    run_half(0);
+    mu = row_total(pass_sum(0)) * inv_n;
+    sd = sqrtf(row_total(pass_ss(0, mu)) * inv_n);
+    const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
+    cnt = pass_mask(0, thr);
+  } else {         // 513-1024: the halves' scores are taken again where a pass needs them
+    run_half(0);
+    const float s0 = pass_sum(0);
+    run_half(1);
+    mu = row_total(s0 + pass_sum(1)) * inv_n;
+    const float q1 = pass_ss(1, mu);
+    run_half(0);
+    sd = sqrtf(row_total(pass_ss(0, mu) + q1) * inv_n);
+    const float thr = (a.tau == -INFINITY) ? -INFINITY : fmaf(a.tau, sd, mu);
+    cnt = pass_mask(0, thr);
+    run_half(1);
+    cnt += pass_mask(1, thr);
   }
   rcnt[part][rr] = cnt;
   __syncthreads();
-  if (live && part == 0 && i < a.nqb) a.counts[row] = (rcnt[0][rr] + rcnt[1][rr]) + (rcnt[2][rr] + rcnt[3][rr]);
+  if (live() && part == 0 && i < a.nqb) a.counts[row] = (rcnt[0][rr] + rcnt[1][rr]) + (rcnt[2][rr] + rcnt[3][rr]);
   fence_before();
   __syncthreads();
   if (warp == 0) {
+    // after an abort the last committed MMAs may still run: they land before TMEM is released
+    if (!ok && ncommit > 0) drain_bar(&bar.mma[(ncommit - 1) & 1], ((ncommit - 1) >> 1) & 1, a.status);
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(512));
   }
@@ -548,7 +600,7 @@ cudaError_t launch_route(const RouteArgs& a, int D, cudaStream_t st) {
       return e;
     if (dev >= 0 && dev < 64) prepared[dev].store(1, std::memory_order_release);
   }
-  if (D == 128 && !a.topk && a.nkb <= 4 * kRtRows)   // threshold routing: scores on the tensor cores
+  if (D == 128 && !a.topk && a.nkb <= 8 * kRtRows)   // threshold routing: scores on the tensor cores
     route_tc_kernel<<<dim3((a.nqb + kRtRows - 1) / kRtRows, a.B * a.H), kRtThreads, kRtSmem, st>>>(a);
   else if (D == 128) route_kernel<128><<<grid, 256, smem, st>>>(a, ldS);
   else route_kernel<64><<<grid, 256, smem, st>>>(a, ldS);
