@@ -354,6 +354,7 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&bar.tmem)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  RtLoad lk0 = rt_load(kbar, 0, a.nkb);   // the first chunk, in flight beside q̄'s tile
   {
     const RtLoad lq = rt_load(qbar, i0, a.nqb);
     rt_store(lq, qt, qt + kRtTerm);
@@ -373,8 +374,11 @@ __global__ void __launch_bounds__(kRtThreads, 1) route_tc_kernel(const RouteArgs
     if (!ok) return;   // uniform
     const int j0 = 4 * h, j1 = min(nch, 4 * h + 4);
     {   // the half's first chunk (its buffer was last read by instance gc - 2, complete by now)
-      const RtLoad lk = rt_load(kbar, j0 * kRtRows, a.nkb);
-      rt_store(lk, kt + (gc & 1) * 2 * kRtTerm, kt + (gc & 1) * 2 * kRtTerm + kRtTerm);
+      if (gc == 0) rt_store(lk0, kt, kt + kRtTerm);
+      else {
+        const RtLoad lk = rt_load(kbar, j0 * kRtRows, a.nkb);
+        rt_store(lk, kt + (gc & 1) * 2 * kRtTerm, kt + (gc & 1) * 2 * kRtTerm + kRtTerm);
+      }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the terms feed the tensor cores
     fence_before();
