@@ -177,9 +177,9 @@ sol_status sol_pool(const sol_params* p, const void* q, const void* k, const voi
  *            the two halves of a 128-row block carry the same list).
  *   col_idx  int32 device, capacity sol_col_capacity(p); row r's exact key
  *            blocks, ascending, at [row_ptr[r], row_ptr[r+1]).
- * Routing 0: S_ij = s * qbar_i . kbar_j to fp32 accuracy (for D = 128 and at
- * most 512 key blocks from bf16 hi/lo terms on the tensor cores, within
- * 4e-6 * |qbar_i||kbar_j| s of the fp32 dot product); block j is exact for row i
+ * Routing 0: S_ij = s * qbar_i . kbar_j to fp32 accuracy (for D = 128 from
+ * bf16 hi/lo terms on the tensor cores, within 4e-6 * |qbar_i||kbar_j| s of
+ * the fp32 dot product); block j is exact for row i
  * iff S_ij > mean_j S_ij + tau * std_j S_ij (population std over all key
  * blocks), or j is a sink block, or i is a dense (prefix) query block.
  * Routing 1: qbar_i over 128 rows; row i keeps its k largest S_ij (equal
