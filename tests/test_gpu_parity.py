@@ -64,13 +64,15 @@ def test_tau_sweep_n8192(tau, lmb):
 @pytest.mark.parametrize("B,N,H,prefix,tau,grid", [(1, 30001, 2, 200, 1.0, (1, 17, 1753)),
                                                    (2, 5000, 3, 0, 0.5, (5, 20, 50)),
                                                    (1, 32768, 1, 64, 2.0, (8, 8, 511)),
-                                                   (2, 40000, 1, 300, 1.0, (4, 25, 397))])
+                                                   (2, 40000, 1, 300, 1.0, (4, 25, 397)),
+                                                   (1, 40000, 2, 0, -math.inf, (16, 25, 100))])
 def test_tensor_core_routing_ragged(B, N, H, prefix, tau, grid):
     """Threshold routing takes its scores from the tensor cores for D = 128 and up to 1024 key
     blocks.  Cases: a partial last 128-block chunk of k-bar and a partial last mask word (469
     key blocks), a partial last 128-row query tile, two batch entries, sinks and dense rows, the
     full 512 key blocks, and 625 key blocks (two halves of the row, the second one a single
-    partial chunk).  The mask must match the oracle outside the 1e-4 band."""
+    partial chunk), also with tau = -inf (every block exact).  The mask must match the oracle
+    outside the 1e-4 band."""
     w = synth.Workload("rt", B=B, H=H, N=N, D=128, grid=grid, n_topics=8, prefix=prefix, tau=tau, seed=31)
     q, k, v = synth.generate(w)
     p, buf = parity.run_gpu(parity.to_dev(q), parity.to_dev(k), parity.to_dev(v), tau, prefix, 0)
